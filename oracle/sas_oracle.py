@@ -1,0 +1,374 @@
+"""fp64 CPU oracle of SAS gated block-sparse causal attention.
+
+TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and bench.py's
+CPU-baseline / reference arm may import this module. The library's kernels
+never call it and share no code with it.
+
+Plain, slow and written to be checked by eye against the pages:
+
+* SAS close reading (liuzhao09.github.io, "SAS: learning context ranking
+  under a finite attention budget"), section 2.1: the history is cut into
+  contiguous blocks B_m of b tokens; s = R(q, {K_Bm}); I = TopK(s, k);
+  S = B0 + the selected blocks; the current block B0 is always kept and is
+  causally masked inside.
+* same page, section 2.2: g_m = exp(s_m) / sum_l exp(s_l) over the C history
+  blocks, g0 = 1, log g_m = s_m - LSE(s); o = softmax(q K_S^T + log g_S) V_S.
+* SAS reproduction note (daiwk.github.io), core formula: the logit carries the
+  1/sqrt(d) scale, o = softmax(q K_S^T / sqrt(d) + log g_S) V_S.
+* SAS close reading, section 2.4: the backward pass recomputes the
+  probabilities, forms the logit gradients from dO and sums them over each
+  selected block into the block's log-gate gradient.
+* SAS close reading, section 2.1 (Algorithm 2 as described there): at
+  inference the continuous bias may be dropped and plain softmax attention
+  runs over the Top-K blocks and the current block (`gated=0`).
+
+Readings where the pages leave a step open (each listed in the design doc):
+* block size b = 64 (section 3.1); the selector is parameter-free:
+  s_m = scale * qbar . kbar_m, kbar_m = mean of block m's 64 keys,
+  qbar = mean of the kv group's query heads (and, in prefill, of the query
+  block's tokens), scale = 1/sqrt(d);
+* the gate softmax runs over all C causally visible complete history blocks;
+* Top-K order is (score descending, block index ascending); the kept indices
+  are listed in ascending block order, padded with -1; kk = min(k, C);
+* prefill selects one block set per (sequence, kv group, 64-token query
+  block); query block t sees history blocks 0..t-1 (C = t);
+* decode: the query sits at position n-1, t = (n-1)//64, C = t and all n-64t
+  tokens of the current block are visible.
+
+Layouts: q/o/dO [B][Hq][N][d]; k/v [B][Hkv][N][d]; summaries [B][Hkv][nblk][d];
+idx/logg/dlogg [B][Hkv][T][k] with T = ceil(N/64); cnt [B][Hkv][T];
+lse [B][Hq][N]. All arithmetic in float64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 64
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a torch tensor: upcast its stored values
+        x = x.detach().cpu().double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# Block summaries (section 2.1: summaries compress each block's keys; the
+# summary is the mean of the block's 64 keys).
+# --------------------------------------------------------------------------
+def block_summary(k, lens=None) -> np.ndarray:
+    """kbar[b, r, m] = mean of the 64 keys of complete block m.
+
+    With `lens`, blocks that are not complete within lens[b] are zero.
+    """
+    k = _f64(k)
+    B, H, N, d = k.shape
+    nblk = N // BLOCK
+    out = np.zeros((B, H, nblk, d))
+    for b in range(B):
+        nb = nblk if lens is None else min(nblk, int(lens[b]) // BLOCK)
+        for m in range(nb):
+            out[b, :, m] = k[b, :, m * BLOCK:(m + 1) * BLOCK].mean(axis=1)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Selector score, normalised gate, Top-K (sections 2.1 and 2.2).
+# --------------------------------------------------------------------------
+def gate_and_topk(s: np.ndarray, topk: int):
+    """For one row's scores s[0..C-1]: (idx ascending, log g of idx, log g of all).
+
+    log g_m = s_m - LSE(s) with the max shift; Top-K keeps the kk = min(k, C)
+    largest scores, ties to the lower block index.
+    """
+    C = s.shape[0]
+    kk = min(topk, C)
+    if C == 0:
+        return np.zeros(0, dtype=np.int64), np.zeros(0), np.zeros(0)
+    mx = s.max()
+    lse = mx + np.log(np.exp(s - mx).sum())
+    logg_all = s - lse
+    order = np.lexsort((np.arange(C), -s))  # primary: -s ascending; then index
+    chosen = np.sort(order[:kk])
+    return chosen, logg_all[chosen], logg_all
+
+
+def _pack_rows(B, Hkv, T, topk):
+    idx = np.full((B, Hkv, T, topk), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hkv, T), dtype=np.int32)
+    logg = np.zeros((B, Hkv, T, topk))
+    return idx, cnt, logg
+
+
+def select_prefill(q, ksum, Hkv: int, topk: int, scale: float | None = None):
+    """Per (b, kv group r, query block t): scores, gate and Top-K.
+
+    qbar = mean over the group's heads and the query block's tokens; C = t.
+    Returns idx int32, cnt int32, logg (fp64), scores list-of-arrays.
+    """
+    q = _f64(q)
+    ksum = _f64(ksum)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    T = -(-N // BLOCK)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    idx, cnt, logg = _pack_rows(B, Hkv, T, topk)
+    scores = {}
+    for b in range(B):
+        for r in range(Hkv):
+            for t in range(T):
+                rows = q[b, r * G:(r + 1) * G, t * BLOCK:min(N, (t + 1) * BLOCK)]
+                qbar = rows.reshape(-1, d).mean(axis=0)
+                C = t
+                s = scale * (ksum[b, r, :C] @ qbar)
+                chosen, lg, _ = gate_and_topk(s, topk)
+                kk = chosen.shape[0]
+                idx[b, r, t, :kk] = chosen
+                cnt[b, r, t] = kk
+                logg[b, r, t, :kk] = lg
+                scores[(b, r, t)] = s
+    return idx, cnt, logg, scores
+
+
+def select_decode(q, ksum, lens, Hkv: int, topk: int, scale: float | None = None):
+    """Per (b, kv group r): the decode query at position n-1, C = (n-1)//64.
+
+    qbar = mean over the group's heads of q[b, h]. Returns idx [B][Hkv][k],
+    cnt [B][Hkv], logg [B][Hkv][k] and the scores.
+    """
+    q = _f64(q)
+    ksum = _f64(ksum)
+    B, Hq, d = q.shape
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    idx = np.full((B, Hkv, topk), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hkv), dtype=np.int32)
+    logg = np.zeros((B, Hkv, topk))
+    scores = {}
+    for b in range(B):
+        C = (int(lens[b]) - 1) // BLOCK
+        for r in range(Hkv):
+            qbar = q[b, r * G:(r + 1) * G].mean(axis=0)
+            s = scale * (ksum[b, r, :C] @ qbar)
+            chosen, lg, _ = gate_and_topk(s, topk)
+            kk = chosen.shape[0]
+            idx[b, r, :kk] = chosen
+            cnt[b, r] = kk
+            logg[b, r, :kk] = lg
+            scores[(b, r)] = s
+    return idx, cnt, logg, scores
+
+
+# --------------------------------------------------------------------------
+# Gated sparse attention, forward (section 2.2; reproduction note's formula)
+# and backward (section 2.4: recompute the probabilities, form the logit
+# gradients from dO, sum them per selected block into d(log g)).
+# --------------------------------------------------------------------------
+def _token_set(t, N, sel, sel_logg):
+    """Key positions and their bias for query block t: the selected history
+    blocks (all 64 tokens, bias log g_m) followed by the current block
+    (bias 0, g0 = 1). Returns positions, bias, and the current block's
+    positions."""
+    pos, bias = [], []
+    for m, lg in zip(sel, sel_logg):
+        pos.append(np.arange(m * BLOCK, (m + 1) * BLOCK))
+        bias.append(np.full(BLOCK, float(lg)))
+    cur = np.arange(t * BLOCK, min(N, (t + 1) * BLOCK))
+    pos.append(cur)
+    bias.append(np.zeros(cur.shape[0]))
+    return np.concatenate(pos), np.concatenate(bias), cur
+
+
+def _block_rows(qt, kS, vS, bias, cur, dot=None, scale=1.0):
+    """Forward (and, with dot, backward) for the rows of one query block.
+
+    qt [nr][d] are the rows i = cur[0..nr-1]; kS, vS [ns][d] the token set
+    whose last len(cur) entries are the current block. Row i sees every
+    history token and the current tokens j <= i (section 2.1, B0 causal).
+    z = scale * q k^T + bias; p = softmax(z); o = p V; lse = log sum e^z.
+    Backward of L = sum(dO * o): D_i = dO_i . o_i, dp = dO V^T,
+    dz = p (dp - D), dq = scale dz K, dK = scale dz^T Q, dV = p^T dO.
+    """
+    nr = qt.shape[0]
+    nhist = kS.shape[0] - cur.shape[0]
+    z = scale * (qt @ kS.T) + bias[None, :]
+    causal = cur[None, :] <= cur[:, None]               # [row i][current j]
+    z[:, nhist:] = np.where(causal, z[:, nhist:], -np.inf)
+    mx = z.max(axis=1, keepdims=True)
+    e = np.exp(z - mx)
+    ssum = e.sum(axis=1, keepdims=True)
+    p = e / ssum
+    o = p @ vS
+    lse = (mx + np.log(ssum))[:, 0]
+    if dot is None:
+        return o, lse
+    D = (dot * o).sum(axis=1, keepdims=True)
+    dp = dot @ vS.T
+    dz = p * (dp - D)
+    dq = scale * (dz @ kS)
+    dkS = scale * (dz.T @ qt)
+    dvS = p.T @ dot
+    return o, lse, dq, dkS, dvS, dz
+
+
+def _scale(d, scale):
+    return 1.0 / np.sqrt(d) if scale is None else scale
+
+
+def attn_fwd(q, k, v, idx, cnt, logg, scale: float | None = None):
+    """o[b,h,i] = sum_j softmax_j(z_ij) v_j and lse[b,h,i] = log sum_j e^z_ij,
+    z_ij = scale * q_i . k_j + log g of j's block (0 in the current block),
+    over the selected blocks and the causal part of the current block."""
+    q, k, v, logg = _f64(q), _f64(k), _f64(v), _f64(logg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    T = -(-N // BLOCK)
+    scale = _scale(d, scale)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            r = h // G
+            for t in range(T):
+                kk = int(cnt[b, r, t])
+                pos, bias, cur = _token_set(t, N, idx[b, r, t, :kk], logg[b, r, t, :kk])
+                o[b, h, cur], lse[b, h, cur] = _block_rows(
+                    q[b, h, cur], k[b, r, pos], v[b, r, pos], bias, cur, scale=scale)
+    return o, lse
+
+
+def attn_bwd(q, k, v, do, idx, cnt, logg, scale: float | None = None):
+    """Gradients of L = sum(dO * o) with o from attn_fwd.
+
+    dlogg[b, r, t, slot] = sum over the group's heads, the rows of query
+    block t and the slot's 64 keys of the logit gradient dz (section 2.4).
+    Returns dq, dk, dv, dlogg.
+    """
+    q, k, v, do, logg = _f64(q), _f64(k), _f64(v), _f64(do), _f64(logg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    T = -(-N // BLOCK)
+    scale = _scale(d, scale)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dlogg = np.zeros(logg.shape)
+    for b in range(B):
+        for h in range(Hq):
+            r = h // G
+            for t in range(T):
+                kk = int(cnt[b, r, t])
+                pos, bias, cur = _token_set(t, N, idx[b, r, t, :kk], logg[b, r, t, :kk])
+                _, _, dqt, dkS, dvS, dz = _block_rows(
+                    q[b, h, cur], k[b, r, pos], v[b, r, pos], bias, cur,
+                    dot=do[b, h, cur], scale=scale)
+                dq[b, h, cur] = dqt
+                np.add.at(dk[b, r], pos, dkS)
+                np.add.at(dv[b, r], pos, dvS)
+                for slot in range(kk):
+                    dlogg[b, r, t, slot] += dz[:, slot * BLOCK:(slot + 1) * BLOCK].sum()
+    return dq, dk, dv, dlogg
+
+
+def query_block(q, k, v, do, idx, cnt, logg, b: int, r: int, t: int,
+                scale: float | None = None):
+    """Forward and backward restricted to query block t of kv group r.
+
+    The same definitions as attn_fwd / attn_bwd, for sampled checks of
+    full-size workloads. Returns per head of the group: o, lse, dq (rows of
+    block t), and dlogg[slot] summed over the group's heads, plus this
+    block's dk/dv contributions {position array, dk rows, dv rows}.
+    """
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    scale = _scale(d, scale)
+    kk = int(cnt[b, r, t])
+    lg = _f64(logg[b, r, t, :kk])
+    pos, bias, cur = _token_set(t, N, np.asarray(idx[b, r, t, :kk]), lg)
+    kS, vS = _f64(k[b, r, pos]), _f64(v[b, r, pos])
+    out = dict(o=[], lse=[], dq=[], dlogg=np.zeros(kk), pos=pos,
+               dk=np.zeros_like(kS), dv=np.zeros_like(vS))
+    for h in range(r * G, (r + 1) * G):
+        o, lse, dq, dkS, dvS, dz = _block_rows(
+            _f64(q[b, h, cur]), kS, vS, bias, cur, dot=_f64(do[b, h, cur]), scale=scale)
+        out["o"].append(o)
+        out["lse"].append(lse)
+        out["dq"].append(dq)
+        out["dk"] += dkS
+        out["dv"] += dvS
+        for slot in range(kk):
+            out["dlogg"][slot] += dz[:, slot * BLOCK:(slot + 1) * BLOCK].sum()
+    return out
+
+
+def key_block_grads(q, k, v, do, idx, cnt, logg, b: int, r: int, j: int,
+                    scale: float | None = None):
+    """dk, dv of key block j of kv group r: the sum of the contributions of
+    every query block that selected j, and of query block j itself (for
+    which j is the current block)."""
+    N = q.shape[2]
+    T = -(-N // BLOCK)
+    dk = np.zeros((BLOCK, q.shape[3]))
+    dv = np.zeros((BLOCK, q.shape[3]))
+    lo = j * BLOCK
+    for t in range(T):
+        kk = int(cnt[b, r, t])
+        if t != j and j not in set(int(x) for x in idx[b, r, t, :kk]):
+            continue
+        res = query_block(q, k, v, do, idx, cnt, logg, b, r, t, scale)
+        hit = (res["pos"] >= lo) & (res["pos"] < lo + BLOCK)
+        np.add.at(dk, res["pos"][hit] - lo, res["dk"][hit])
+        np.add.at(dv, res["pos"][hit] - lo, res["dv"][hit])
+    return dk, dv
+
+
+# --------------------------------------------------------------------------
+# Decode (section 2.1/2.4 serving: one query token per sequence, GQA groups
+# share one block set).
+# --------------------------------------------------------------------------
+def decode(q, kc, vc, lens, ksum, Hkv: int, topk: int, gated: int = 1,
+           scale: float | None = None):
+    """One decode step. q [B][Hq][d]; kc, vc [B][Hkv][Lmax][d]; ksum the
+    block summaries. Each (b, kv group) selects with select_decode; every
+    head of the group attends over the selected blocks (bias log g when
+    gated=1, none when gated=0) and the n-64t tokens of the current block.
+    Returns o [B][Hq][d], idx [B][Hkv][k], cnt [B][Hkv], lse [B][Hq]."""
+    q = _f64(q)
+    B, Hq, d = q.shape
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    idx, cnt, logg, _ = select_decode(q, ksum, lens, Hkv, topk, scale)
+    o = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        n = int(lens[b])
+        t = (n - 1) // BLOCK
+        for r in range(Hkv):
+            kk = int(cnt[b, r])
+            pos, bias = [], []
+            for slot in range(kk):
+                m = int(idx[b, r, slot])
+                pos.append(np.arange(m * BLOCK, (m + 1) * BLOCK))
+                bias.append(np.full(BLOCK, logg[b, r, slot] if gated else 0.0))
+            cur = np.arange(t * BLOCK, n)
+            pos.append(cur)
+            bias.append(np.zeros(cur.shape[0]))
+            pos = np.concatenate(pos)
+            bias = np.concatenate(bias)
+            kr = _f64(kc[b, r][pos])
+            vr = _f64(vc[b, r][pos])
+            for h in range(r * G, (r + 1) * G):
+                z = scale * (kr @ q[b, h]) + bias
+                mx = z.max()
+                e = np.exp(z - mx)
+                o[b, h] = (e / e.sum()) @ vr
+                lse[b, h] = mx + np.log(e.sum())
+    return o, idx, cnt, lse

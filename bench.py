@@ -1,0 +1,577 @@
+#!/usr/bin/env python
+"""Benchmark of the SAS gated block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c4|c5|c3|c1]
+                    [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). A step is one pass of the hot path over one
+batch of the named synthetic workload:
+  decode configs (c2 default, c4, c5): block selection over the summaries
+    (scores, gate, Top-K) and split-K attention over the kept blocks plus the
+    current block, for every sequence and kv group; the summaries are built
+    when blocks complete, outside the step. Metric: GB/s of algorithmic bytes
+    (summaries scanned + kept K/V read + q/o).
+  prefill configs (c3, c1): summaries, selection, gated sparse forward and
+    backward. Metric: TFLOP/s of algorithmic FLOPs (kept block pairs, causal
+    pairs exact on the diagonal block, forward 4d and backward 10d per pair).
+
+Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs and
+bracketed by CUDA events on the launching stream (barrier + synchronize on
+both sides, max over ranks). Decode steps rotate over L copies of the layer's
+cache and summaries so that the bytes touched between reuses exceed 3x L2.
+With N > 1 every rank runs its own replica (independent sequences, no
+data-path collective): weak scaling.
+
+--impl reference times the fp64 CPU oracle on the host cores, on bounded
+samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode GB/s vs HBM peak; prefill fwd+bwd TFLOP/s vs bf16 peak"
+DEFAULT_STEPS = {"c1": 200, "c2": 100000, "c3": 10, "c4": 4000, "c5": 20000}
+DEFAULT_WARMUP = {"c1": 10, "c2": 1000, "c3": 3, "c4": 100, "c5": 500}
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    sm_max=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max=1965.0, source="fallback")
+
+
+def source_sha(name: str) -> str:
+    p = os.path.join(ROOT, "gated_block_sparse_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, source: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("source_sha") != source_sha(source):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples every 100 ms; summarised over a wall-clock window."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        rows = []
+        try:
+            for r in csv.reader(open(self.f.name)):
+                if len(r) < 9:
+                    continue
+                ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + r[0].strip().split(".")[1]) if "." in r[0] else 0.0
+                rows.append((ts + frac, [x.strip() for x in r[1:]]))
+        except Exception:
+            rows = []
+        win = [x for t, x in rows if t0 - 0.15 <= t <= t1 + 0.15] or \
+              [x for t, x in rows if t >= t0][:1] or rows[-1:]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for x in win for n, v in zip(names, x[4:8]) if v.lower() == "active"})
+        sm = [float(x[0]) for x in win if x[0].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(win[0][1]) if win[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: int = 512,
+                 clocks: ClockSampler | None = None):
+    """Capture fn_step(i) for i in [0, chunk) into a graph (plus a tail graph)
+    and time exactly n_steps steps after `warmup` untimed ones. Returns
+    (ms total, max over ranks; clock summary)."""
+    import torch
+    chunk = max(1, min(chunk, n_steps))
+    graphs = {}
+
+    def graph_of(n):
+        if n not in graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    fn_step(i)
+            graphs[n] = g
+        return graphs[n]
+
+    def run(n):
+        full, tail = divmod(n, chunk)
+        for _ in range(full):
+            graph_of(chunk).replay()
+        if tail:
+            graph_of(tail).replay()
+
+    with torch.cuda.stream(stream):
+        run(max(3, warmup))
+        graph_of(chunk)
+        if n_steps % chunk:
+            graph_of(n_steps % chunk)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        start.record(stream)
+        run(n_steps)
+        end.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        barrier(world)
+    ms = max_over_ranks(world, start.elapsed_time(end))
+    return ms, (clocks.summary(t0, t1) if clocks else None)
+
+
+# ----------------------------------------------------------------- decode
+class DecodeWorkload:
+    def __init__(self, name: str):
+        from gated_block_sparse_b200 import inputs
+        self.name = name
+        self.c = inputs.CONFIGS[name]
+        self.host = inputs.gen_config(name)
+        c = self.c
+        lens = self.host["lens"].numpy()
+        self.rows = c["B"] * c["Hkv"]
+        self.C = [(int(n) - 1) // 64 for n in lens]
+        kk = [min(c["topk"], C) for C in self.C]
+        ncur = [int(n) - 64 * C for n, C in zip(lens, self.C)]
+        d, Hkv, es = c["d"], c["Hkv"], 2 if c["dtype"] == "bf16" else 4
+        # algorithmic bytes per step, by kernel
+        self.sel_bytes = sum(Hkv * C * d * 4 for C in self.C) + c["B"] * c["Hq"] * d * es
+        self.att_bytes = (sum(Hkv * (k * 64 + nc) * d * es * 2 for k, nc in zip(kk, ncur))
+                          + 2 * c["B"] * c["Hq"] * d * es)
+        self.step_bytes = self.sel_bytes + self.att_bytes - c["B"] * c["Hq"] * d * es  # q once
+
+    def describe(self):
+        from gated_block_sparse_b200 import inputs
+        c = self.c
+        return {"workload": f"{self.name}: {inputs.DESCRIPTIONS[self.name]}", "batch": c["B"],
+                "q_heads": c["Hq"], "kv_heads": c["Hkv"], "head_dim": c["d"],
+                "context": c["Lmax"] if c["lens"][0] == c["lens"][1] else list(c["lens"]),
+                "topk": c["topk"], "gated": c["gated"], "block": 64,
+                "bytes_per_step": self.step_bytes}
+
+
+def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
+    import torch
+
+    from gated_block_sparse_b200 import sas
+    c = w.c
+    dev = torch.device("cuda", local if world > 1 else 0)
+    h = w.host
+    q = h["q"].to(dev)
+    lens = h["lens"].to(dev)
+    kc0, vc0 = h["kc"].to(dev), h["vc"].to(dev)
+    ks0 = sas.sas_block_summary(kc0)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_layer = kc0.numel() * kc0.element_size() * 2 + ks0.numel() * 4
+    free = torch.cuda.mem_get_info(dev)[0]
+    L = max(2, math.ceil(3 * l2 / w.step_bytes))
+    L = min(L, max(2, int(0.6 * free // per_layer)))
+    if args.layers:
+        L = args.layers
+    kcs, vcs, kss = [kc0], [vc0], [ks0]
+    for _ in range(L - 1):
+        kcs.append(kc0.clone())
+        vcs.append(vc0.clone())
+        kss.append(ks0.clone())
+    topk, Hkv = c["topk"], c["Hkv"]
+    o = torch.empty_like(q)
+    ws = torch.empty(sas.sas_decode_workspace_size(c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    K, W = args.steps, args.warmup
+
+    def step(i):
+        j = i % L
+        sas.sas_decode(q, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=o, ws=ws)
+
+    ms, clk = timed_graphs(step, K, W, world, stream, clocks=clocks)
+    clocks.stop()
+
+    # per-kernel timing for the roofline: selection alone, attention alone
+    sel = [sas.sas_select(q, kss[j], Hkv, topk, "decode", lens=lens) for j in range(L)]
+    sel_ws = torch.empty(max(16, sas.load_library().sas_select_workspace_size(
+        c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk, 1)), dtype=torch.uint8, device=dev)
+    att_ws = torch.empty(max(16, sas.load_library().sas_decode_attend_workspace_size(
+        c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk)), dtype=torch.uint8, device=dev)
+    sel_out = [(torch.empty_like(a), torch.empty_like(b), torch.empty_like(cc)) for a, b, cc in sel]
+    Kk = min(K, 20000)
+
+    def sel_step(i):
+        j = i % L
+        sas.sas_select(q, kss[j], Hkv, topk, "decode", lens=lens, out=sel_out[j], ws=sel_ws)
+
+    def att_step(i):
+        j = i % L
+        sas.sas_decode_attend(q, kcs[j], vcs[j], lens, *sel[j], gated=c["gated"], out=o, ws=att_ws)
+
+    ms_sel, _ = timed_graphs(sel_step, Kk, 10, world, stream)
+    ms_att, _ = timed_graphs(att_step, Kk, 10, world, stream)
+    t_sel, t_att = ms_sel / Kk * 1e-3, ms_att / Kk * 1e-3
+    peaks = measured_peaks()
+    if t_sel >= t_att:
+        kern, kb, kt, src = "k_select_decode", w.sel_bytes, t_sel, "k_select.cu"
+    else:
+        kern, kb, kt, src = "k_decode_attend", w.att_bytes, t_att, "k_decode.cu"
+    ach = kb / kt / 1e9
+    roof = {"bound": "hbm", "kernel": kern, "achieved": round(ach, 1), "peak": peaks["hbm"],
+            "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
+            "traffic": recorded_traffic(kern, src),
+            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+            "algorithmic_bytes_per_launch": kb, "launch_us": round(kt * 1e6, 3),
+            "other_kernel": {"k_select_decode": {"us": round(t_sel * 1e6, 3),
+                                                 "GBps": round(w.sel_bytes / t_sel / 1e9, 1)},
+                             "k_decode_attend": {"us": round(t_att * 1e6, 3),
+                                                 "GBps": round(w.att_bytes / t_att / 1e9, 1)}}}
+
+    # end to end through the public API: pinned host q in, o out, every step
+    qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    qh.copy_(q.cpu())
+    oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    qd = torch.empty_like(q)
+    E = min(K, 2000)
+    with torch.cuda.stream(stream):
+        for i in range(20):
+            qd.copy_(qh, non_blocking=True)
+            sas.sas_decode(qd, kcs[i % L], vcs[i % L], lens, kss[i % L], topk, gated=c["gated"],
+                           out=o, ws=ws)
+            oh.copy_(o, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(E):
+            qd.copy_(qh, non_blocking=True)
+            sas.sas_decode(qd, kcs[i % L], vcs[i % L], lens, kss[i % L], topk, gated=c["gated"],
+                           out=o, ws=ws)
+            oh.copy_(o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
+    nb = q.numel() * q.element_size()
+
+    value = w.step_bytes * K * world / (ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if c["dtype"] == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) with planted relevant blocks)",
+        "config": {**w.describe(), "parallelism": f"replicas x{world}",
+                   "l2": f"rotating {L} layer copies of cache + summaries "
+                         f"({w.step_bytes * L / 1e6:.0f} MB touched per rotation, L2 {l2 / 1e6:.0f} MB)"},
+        "roofline": roof,
+        "e2e": {"value": round(w.step_bytes * E * world / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb,
+                "path": "pinned host q -> sas_decode (Python binding, C ABI) -> pinned host o"},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    return res
+
+
+def one_thread():
+    """Limit numpy's BLAS to one thread (the oracle baseline runs on 1 core)."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
+
+
+def cpu_baseline_decode(name: str, seconds: float, w: "DecodeWorkload | None" = None) -> dict:
+    """The fp64 oracle on whole decode steps of the workload, for ~`seconds`."""
+    from oracle import sas_oracle as O
+    w = DecodeWorkload(name) if w is None else w
+    c = w.c
+    h = w.host
+    with one_thread():
+        ks = O.block_summary(h["kc"])  # summaries are built outside the step, as on the GPU
+        lens = h["lens"].numpy()
+        n, t0 = 0, time.perf_counter()
+        while True:
+            O.decode(h["q"], h["kc"], h["vc"], lens, ks, c["Hkv"], c["topk"], gated=c["gated"])
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return {"value": round(w.step_bytes * n / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "steps": n, "seconds": round(el, 2),
+            "sample": f"{n} whole decode steps of {name} (all {w.rows} rows), fp64 numpy oracle, "
+                      f"1 BLAS thread; summaries precomputed as on the GPU"}
+
+
+# ----------------------------------------------------------------- prefill
+def prefill_flops(idx_cnt, N: int, Hq: int, Hkv: int, d: int):
+    """Algorithmic FLOPs of one forward and one backward (per sequence sum)."""
+    import numpy as np
+    cnt = np.asarray(idx_cnt)  # [B][Hkv][T]
+    G = Hq // Hkv
+    T = cnt.shape[-1]
+    pairs = 0
+    for t in range(T):
+        nr = min(64, N - 64 * t)
+        pairs += int(cnt[..., t].sum()) * G * nr * 64 + cnt.shape[0] * Hq * nr * (nr + 1) // 2
+    return 4 * d * pairs, 10 * d * pairs
+
+
+def bench_prefill_ours(args, world, rank, local) -> dict:
+    import torch
+
+    from gated_block_sparse_b200 import inputs, sas
+    name = args.config
+    c = inputs.CONFIGS[name]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    h = inputs.gen_config(name)
+    q, k, v, do = (h[n].to(dev) for n in ("q", "k", "v", "do"))
+    topk, Hkv = c["topk"], c["Hkv"]
+    B, Hq, N, d = q.shape
+    ks = sas.sas_block_summary(k)
+    idx, cnt, logg = sas.sas_select(q, ks, Hkv, topk, "prefill")
+    o, lse = sas.sas_attn_fwd(q, k, v, idx, cnt, logg)
+    grads = sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg)
+    torch.cuda.synchronize()
+    f_fwd, f_bwd = prefill_flops(cnt.cpu().numpy(), N, Hq, Hkv, d)
+    lib = sas.load_library()
+    dt = 1 if c["dtype"] == "bf16" else 0
+    sel_ws = torch.empty(max(16, lib.sas_select_workspace_size(B, Hq, Hkv, N, d, topk, 0)),
+                         dtype=torch.uint8, device=dev)
+    bwd_ws = torch.empty(max(16, lib.sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt)),
+                         dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+
+    def step(i):
+        sas.sas_block_summary(k, out=ks)
+        sas.sas_select(q, ks, Hkv, topk, "prefill", out=(idx, cnt, logg), ws=sel_ws)
+        sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
+        sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+
+    K, W = args.steps, args.warmup
+    ms, clk = timed_graphs(step, K, W, world, stream, chunk=8, clocks=clocks)
+    clocks.stop()
+
+    def fwd_step(i):
+        sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
+
+    def bwd_step(i):
+        sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+
+    ms_f, _ = timed_graphs(fwd_step, max(3, K), 2, world, stream, chunk=8)
+    ms_b, _ = timed_graphs(bwd_step, max(3, K), 2, world, stream, chunk=8)
+    tf, tb = ms_f / max(3, K) * 1e-3, ms_b / max(3, K) * 1e-3
+    peaks = measured_peaks()
+    simt_peak = 148 * 128 * 2 * peaks["sm_max"] * 1e6 / 1e12  # fp32 FMA lanes x 2 x clock
+    if tb >= tf:
+        kern, kf, kt = "k_attn_bwd_simt", f_bwd, tb
+    else:
+        kern, kf, kt = "k_attn_fwd_simt", f_fwd, tf
+    ach = kf / kt / 1e12
+    roof = {"bound": "alu", "kernel": kern, "achieved": round(ach, 3), "peak": round(simt_peak, 1),
+            "unit": "TFLOP/s", "frac": round(ach / simt_peak, 4),
+            "traffic": recorded_traffic(kern, "k_attn_simt.cu"),
+            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock "
+                           "(fp32 CUDA-core path)",
+            "algorithmic_flops_per_launch": kf, "launch_ms": round(kt * 1e3, 4),
+            "fwd_ms": round(tf * 1e3, 4), "bwd_ms": round(tb * 1e3, 4),
+            "bf16_tensor_peak_for_reference": peaks["bf16"]}
+
+    # end to end: pinned host inputs in, gradients out
+    pin = {n: torch.empty(h[n].shape, dtype=h[n].dtype, pin_memory=True) for n in ("q", "k", "v", "do")}
+    for n in pin:
+        pin[n].copy_(h[n])
+    outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o,) + tuple(grads)]
+    E = max(2, min(K, 5))
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(E):
+            q.copy_(pin["q"], non_blocking=True)
+            k.copy_(pin["k"], non_blocking=True)
+            v.copy_(pin["v"], non_blocking=True)
+            do.copy_(pin["do"], non_blocking=True)
+            step(0)
+            for dst, src in zip(outs, (o,) + tuple(grads)):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    total = f_fwd + f_bwd
+    return {
+        "metric": METRIC, "value": round(total * K * world / (ms * 1e-3) / 1e12, 4),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if c["dtype"] == "bf16" else "f32", "data": "synthetic (seeded N(0,1), planted)",
+        "config": {"workload": f"{name}: {inputs.DESCRIPTIONS[name]}", "batch": B, "seq_len": N,
+                   "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "topk": topk,
+                   "flops_fwd": f_fwd, "flops_bwd": f_bwd, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 (q+k+v+dO = {h2d / 1e6:.0f} MB)"},
+        "roofline": roof,
+        "e2e": {"value": round(total * E * world / (ms_e2e * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 7 * K,
+        "clocks": clk,
+    }
+
+
+def cpu_baseline_prefill(name: str, seconds: float) -> dict:
+    """The oracle's forward+backward on whole query blocks of the workload."""
+    import numpy as np
+
+    from gated_block_sparse_b200 import inputs
+    from oracle import sas_oracle as O
+    c = inputs.CONFIGS[name]
+    h = inputs.gen_config(name)
+    N, d = c["N"], c["d"]
+    G = c["Hq"] // c["Hkv"]
+    with one_thread():
+        ks = O.block_summary(h["k"])
+        idx, cnt, logg, _ = O.select_prefill(h["q"], ks, c["Hkv"], c["topk"])
+        T = idx.shape[2]
+        n, flops, t0 = 0, 0, time.perf_counter()
+        order = [(b, r, t) for t in range(T - 1, -1, -1) for b in range(c["B"])
+                 for r in range(c["Hkv"])]
+        for (b, r, t) in order:
+            O.query_block(h["q"], h["k"], h["v"], h["do"], idx, cnt, logg, b, r, t)
+            nr = min(64, N - 64 * t)
+            pairs = int(cnt[b, r, t]) * G * nr * 64 + G * nr * (nr + 1) // 2
+            flops += 14 * d * pairs
+            n += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        el = time.perf_counter() - t0
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "seconds": round(el, 2),
+            "sample": f"{n} of {len(order)} (sequence, kv group, query block) units of {name} "
+                      "(forward + backward, all heads of the group), fp64 numpy oracle, 1 BLAS thread"}
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="decode: number of rotated layer copies (default: enough for 3x L2)")
+    args = ap.parse_args()
+    args.steps = args.steps or DEFAULT_STEPS[args.config]
+    args.warmup = max(3, args.warmup if args.warmup is not None else DEFAULT_WARMUP[args.config])
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    decode = args.config in ("c2", "c4", "c5")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        base = (cpu_baseline_decode(args.config, args.cpu_seconds) if decode
+                else cpu_baseline_prefill(args.config, args.cpu_seconds))
+        from gated_block_sparse_b200 import inputs
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
+            "n_gpus": args.gpus, "steps": base.get("steps"), "warmup": 0,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded, same generator)",
+            "config": {"workload": f"{args.config}: {inputs.DESCRIPTIONS[args.config]}"},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": base["unit"], "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    if decode:
+        w = DecodeWorkload(args.config)
+        res = bench_decode_ours(args, world, rank, local, w)
+    else:
+        res = bench_prefill_ours(args, world, rank, local)
+    if rank == 0:
+        res["cpu_baseline"] = (cpu_baseline_decode(args.config, args.cpu_seconds, w) if decode
+                               else cpu_baseline_prefill(args.config, args.cpu_seconds))
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

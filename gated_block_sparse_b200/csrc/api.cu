@@ -1,0 +1,324 @@
+// C ABI of libsas (declared in include/sas.h): argument validation, workspace
+// carving and kernel launches. Host code only; the kernels live in k_*.cu.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "../../include/sas.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sas_status fail(sas_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+sas_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return SAS_OK;
+  return fail(SAS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, st, ...) \
+  do {                         \
+    if (!(cond)) return fail(st, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p)                                                                   \
+  do {                                                                                   \
+    if ((p) == nullptr) return fail(SAS_ERR_INVALID_ARG, "%s must not be NULL", #p);     \
+    if (!aligned16(p)) return fail(SAS_ERR_INVALID_ARG, "%s must be 16-byte aligned", #p); \
+  } while (0)
+
+sas_status check_common(sas_dtype dt, int B, int Hq, int Hkv, int N, int d, int topk) {
+  REQUIRE(dt == SAS_F32 || dt == SAS_BF16, SAS_ERR_INVALID_ARG, "dtype must be SAS_F32 or SAS_BF16");
+  REQUIRE(B >= 0 && N >= 0, SAS_ERR_INVALID_ARG, "B and N must be >= 0 (B=%d N=%d)", B, N);
+  REQUIRE(Hq >= 1 && Hkv >= 1, SAS_ERR_INVALID_ARG, "head counts must be >= 1 (Hq=%d Hkv=%d)", Hq, Hkv);
+  REQUIRE(Hq % Hkv == 0, SAS_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  REQUIRE(Hq / Hkv <= 8, SAS_ERR_UNSUPPORTED, "at most 8 query heads per kv head (got %d)", Hq / Hkv);
+  REQUIRE(d == 64 || d == 128, SAS_ERR_UNSUPPORTED, "head dim must be 64 or 128 (got %d)", d);
+  REQUIRE(topk >= 0, SAS_ERR_INVALID_ARG, "topk must be >= 0 (got %d)", topk);
+  REQUIRE(topk <= 128, SAS_ERR_UNSUPPORTED, "topk must be <= 128 (got %d)", topk);
+  return SAS_OK;
+}
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
+
+size_t a16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// Decode workspace: counters [2 * rows] | select partials | attend partials |
+// idx [rows][topk] | cnt [rows] | logg [rows][topk].
+struct DecodeLayout {
+  size_t counters, sel, att, idx, cnt, logg, total;
+};
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int d, int topk) {
+  DecodeLayout L;
+  const int rows = B * Hkv;
+  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, Lmax, topk);
+  size_t off = 0;
+  L.counters = off; off += a16(sizeof(int) * 2 * (size_t)rows);
+  L.sel = off; off += a16(sas::decode_select_ws_bytes(p));
+  L.att = off; off += a16(sas::decode_attend_ws_bytes(B, Hq, Hkv, topk, d));
+  L.idx = off; off += a16(sizeof(int32_t) * (size_t)rows * topk);
+  L.cnt = off; off += a16(sizeof(int32_t) * (size_t)rows);
+  L.logg = off; off += a16(sizeof(float) * (size_t)rows * topk);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sas_strerror(sas_status s) {
+  switch (s) {
+    case SAS_OK: return "ok";
+    case SAS_ERR_INVALID_ARG: return "invalid argument";
+    case SAS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SAS_ERR_CUDA: return "CUDA error";
+    case SAS_ERR_TIMEOUT: return "device wait timed out";
+    case SAS_ERR_INTERNAL: return "internal error";
+  }
+  return "unknown status";
+}
+
+const char* sas_last_error_message(void) { return g_last_error.c_str(); }
+
+int sas_version(void) { return 100; }
+
+sas_status sas_block_summary(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                             const int32_t* lens, float* ksum, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, H, H, N, d, 0);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N / 64 == 0) return SAS_OK;
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(ksum);
+  if (lens) REQUIRE(aligned16(lens), SAS_ERR_INVALID_ARG, "lens must be 16-byte aligned");
+  return cuda_status(sas::launch_block_summary(k, dt == SAS_BF16, B, H, N, d, lens, ksum,
+                                               (cudaStream_t)stream),
+                     "sas_block_summary launch");
+}
+
+size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_mode mode) {
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || topk < 0) return 0;
+  if (mode == SAS_PREFILL) return a16(sas::select_prefill_ws_bytes(B, Hkv, N, d));
+  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, N, topk);
+  return a16(sizeof(int) * (size_t)B * Hkv) + a16(sas::decode_select_ws_bytes(p));
+}
+
+sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
+                      int N, int d, int topk, sas_mode mode, const int32_t* lens, float scale,
+                      int32_t* idx, int32_t* cnt, float* logg, void* ws, size_t ws_bytes,
+                      sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE(mode == SAS_PREFILL || mode == SAS_DECODE, SAS_ERR_INVALID_ARG, "bad mode");
+  if (B == 0 || N == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(cnt);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  if (N / 64 > 0) REQUIRE_PTR(ksum);
+  const size_t need = sas_select_workspace_size(B, Hq, Hkv, N, d, topk, mode);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  const float sc = resolve_scale(scale, d);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (mode == SAS_PREFILL) {
+    REQUIRE(lens == nullptr, SAS_ERR_INVALID_ARG, "lens must be NULL in prefill mode");
+    REQUIRE((N + 63) / 64 - 1 <= 256 * 64, SAS_ERR_UNSUPPORTED, "prefill N too long for selection");
+    return cuda_status(sas::launch_select_prefill(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
+                                                  sc, idx, cnt, logg, ws, st),
+                       "sas_select launch");
+  }
+  REQUIRE_PTR(lens);
+  REQUIRE(N % 64 == 0 && N >= 64, SAS_ERR_INVALID_ARG, "decode needs Lmax a positive multiple of 64");
+  REQUIRE(topk > 0 || idx == nullptr || aligned16(idx), SAS_ERR_INVALID_ARG, "idx alignment");
+  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, N, topk);
+  int* counters = static_cast<int*>(ws);
+  void* rest = static_cast<char*>(ws) + a16(sizeof(int) * (size_t)B * Hkv);
+  cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)B * Hkv, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_select memset");
+  return cuda_status(sas::launch_select_decode(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
+                                               lens, sc, idx, cnt, logg, p, counters, rest, st),
+                     "sas_select launch");
+}
+
+size_t sas_attn_fwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_dtype dt) {
+  (void)B; (void)Hq; (void)Hkv; (void)N; (void)d; (void)topk; (void)dt;
+  return 0;
+}
+
+static sas_status check_attn_ptrs(const void* q, const void* k, const void* v, const int32_t* idx,
+                                  const int32_t* cnt, const float* logg, int topk) {
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(cnt);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  return SAS_OK;
+}
+
+sas_status sas_attn_fwd(const void* q, const void* k, const void* v, sas_dtype dt, int B, int Hq,
+                        int Hkv, int N, int d, const int32_t* idx, const int32_t* cnt,
+                        const float* logg, int topk, float scale, void* o, float* lse, void* ws,
+                        size_t ws_bytes, sas_stream_t stream) {
+  g_last_error.clear();
+  (void)ws; (void)ws_bytes;
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N == 0) return SAS_OK;
+  s = check_attn_ptrs(q, k, v, idx, cnt, logg, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(lse);
+  return cuda_status(sas::launch_attn_fwd_simt(q, k, v, dt == SAS_BF16, B, Hq, Hkv, N, d, idx, cnt,
+                                               logg, topk, resolve_scale(scale, d), o, lse,
+                                               (cudaStream_t)stream),
+                     "sas_attn_fwd launch");
+}
+
+size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_dtype dt) {
+  (void)Hq; (void)topk; (void)dt;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return 0;
+  return a16(sas::attn_bwd_simt_ws_bytes(B, Hkv, N, d));
+}
+
+sas_status sas_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, sas_dtype dt, int B, int Hq, int Hkv, int N, int d,
+                        const float* lse, const int32_t* idx, const int32_t* cnt,
+                        const float* logg, int topk, float scale, void* dq, void* dk, void* dv,
+                        float* dlogg, void* ws, size_t ws_bytes, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N == 0) return SAS_OK;
+  s = check_attn_ptrs(q, k, v, idx, cnt, logg, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(lse);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  if (topk > 0) REQUIRE_PTR(dlogg);
+  const size_t need = sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  return cuda_status(sas::launch_attn_bwd_simt(q, k, v, o, dout, dt == SAS_BF16, B, Hq, Hkv, N, d,
+                                               lse, idx, cnt, logg, topk, resolve_scale(scale, d),
+                                               dq, dk, dv, dlogg, ws, (cudaStream_t)stream),
+                     "sas_attn_bwd launch");
+}
+
+static sas_status check_decode(sas_dtype dt, int B, int Hq, int Hkv, int Lmax, int d, int topk,
+                               int gated) {
+  sas_status s = check_common(dt, B, Hq, Hkv, Lmax, d, topk);
+  if (s != SAS_OK) return s;
+  const int G = Hq / Hkv;
+  REQUIRE(G == 1 || G == 2 || G == 4 || G == 8, SAS_ERR_UNSUPPORTED,
+          "decode supports 1, 2, 4 or 8 query heads per kv head (got %d)", G);
+  REQUIRE(Lmax % 64 == 0 && Lmax >= 64, SAS_ERR_INVALID_ARG, "Lmax must be a positive multiple of 64");
+  REQUIRE(gated == 0 || gated == 1, SAS_ERR_INVALID_ARG, "gated must be 0 or 1");
+  return SAS_OK;
+}
+
+size_t sas_decode_attend_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk) {
+  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || d <= 0 || topk < 0) return 0;
+  return a16(sizeof(int) * (size_t)B * Hkv) + a16(sas::decode_attend_ws_bytes(B, Hq, Hkv, topk, d));
+}
+
+sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_dtype dt, int B,
+                             int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                             const int32_t* idx, const int32_t* cnt, const float* logg, int topk,
+                             int gated, float scale, void* o, void* ws, size_t ws_bytes,
+                             sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_decode(dt, B, Hq, Hkv, Lmax, d, topk, gated);
+  if (s != SAS_OK) return s;
+  if (B == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kc);
+  REQUIRE_PTR(vc);
+  REQUIRE_PTR(lens);
+  REQUIRE_PTR(cnt);
+  REQUIRE_PTR(o);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  const size_t need = sas_decode_attend_workspace_size(B, Hq, Hkv, Lmax, d, topk);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  int* counters = static_cast<int*>(ws);
+  cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)B * Hkv, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_decode_attend memset");
+  e = sas::launch_decode_attend(q, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, idx, cnt,
+                                logg, topk, gated, resolve_scale(scale, d), o, counters,
+                                static_cast<char*>(ws) + a16(sizeof(int) * (size_t)B * Hkv), st,
+                                false);
+  return cuda_status(e, "sas_decode_attend launch");
+}
+
+size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk) {
+  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || d <= 0 || topk < 0) return 0;
+  return decode_layout(B, Hq, Hkv, Lmax, d, topk).total;
+}
+
+sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype dt, int B, int Hq,
+                      int Hkv, int Lmax, int d, const int32_t* lens, const float* ksum, int topk,
+                      int gated, float scale, void* o, int32_t* idx_out, void* ws,
+                      size_t ws_bytes, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_decode(dt, B, Hq, Hkv, Lmax, d, topk, gated);
+  if (s != SAS_OK) return s;
+  if (B == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kc);
+  REQUIRE_PTR(vc);
+  REQUIRE_PTR(lens);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(o);
+  if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
+  const DecodeLayout L = decode_layout(B, Hq, Hkv, Lmax, d, topk);
+  REQUIRE(ws_bytes >= L.total, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, L.total);
+  REQUIRE_PTR(ws);
+  char* w = static_cast<char*>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int rows = B * Hkv;
+  int* counters = reinterpret_cast<int*>(w + L.counters);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  int32_t* cnt = reinterpret_cast<int32_t*>(w + L.cnt);
+  float* logg = reinterpret_cast<float*>(w + L.logg);
+  const float sc = resolve_scale(scale, d);
+  cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * 2 * (size_t)rows, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_decode memset");
+  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, Lmax, topk);
+  e = sas::launch_select_decode(q, dt == SAS_BF16, ksum, B, Hq, Hkv, Lmax, d, topk, lens, sc, idx,
+                                cnt, logg, p, counters, w + L.sel, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_decode select launch");
+  e = sas::launch_decode_attend(q, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, idx, cnt,
+                                logg, topk, gated, sc, o, counters + rows, w + L.att, st, true);
+  return cuda_status(e, "sas_decode attend launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,489 @@
+// Selector scores, softmax gate and Top-K over the history blocks (SAS close
+// reading, liuzhao09.github.io, sections 2.1-2.2: s = R(q, {K_Bm}),
+// I = TopK(s, k), g = softmax(s) over the C history blocks, log g = s - LSE).
+// The selector is parameter-free: s_m = scale * qbar . kbar_m.
+//
+// Top-K is exact and deterministic for any tie pattern. A candidate's order
+// key is (score descending, block index ascending), packed into one 64-bit
+// integer. Each chunk of up to 256 history blocks is scored into shared
+// memory and reduced to its own best-first list of min(k, n) candidates by
+// rank counting. The merge takes theta = the best k-th entry among the full
+// lists; every global Top-K member is at or above theta (the list that gives
+// theta alone holds k keys >= theta), so only entries >= theta are ranked,
+// each by binary searches in the sorted lists. The kept blocks are then
+// written in ascending block order. (The MSA notes, papercache, Top-K kernel
+// section, use per-lane heaps and a shuffle merge on H800; chunk lists plus a
+// threshold merge suit wide CTAs and need no heap.)
+//
+// Prefill: one CTA per (b, kv group, query block). Decode: one CTA per
+// (b, kv group, chunk); the last CTA to finish a row (atomic counter, no
+// waiting) merges, writes the row and resets the counter.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sas {
+
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_CHUNK_MAX = 256;      // prefill chunk
+constexpr int DEC_CHUNK_MAX = 512;      // decode chunk upper bound
+constexpr int DEC_NCHUNK_MAX = 128;     // decode chunks per row upper bound
+
+__device__ __forceinline__ unsigned long long cand_key(float s, int m) {
+  uint32_t u = __float_as_uint(s);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving map
+  return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)m);
+}
+
+__device__ __forceinline__ float block_reduce_max(float v, float* red) {
+  v = warp_max(v);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float r = -FLT_MAX;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+__device__ __forceinline__ float block_reduce_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r += red[i];
+  return r;
+}
+
+// s[j] = scale * qbar . ksum_row[m0 + j] for j < n. Warp-per-block with the
+// d dimension split over the lanes (D/32 floats each), four blocks in flight
+// per warp. A -0 score is stored as +0 so that exact ties compare equal.
+template <int D>
+__device__ void score_chunk(const float* __restrict__ ks_row, int m0, int n,
+                            const float* qbar_s, float scale, float* sc) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  float qv[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) qv[i] = qbar_s[lane * PER + i];
+  for (int base = w; base < n; base += nw * 4) {
+    float part[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * nw;
+      float acc = 0.f;
+      if (j < n) {
+        const float* p = ks_row + (size_t)(m0 + j) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+          acc = x.x * qv[0] + x.y * qv[1] + x.z * qv[2] + x.w * qv[3];
+        } else {
+          const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+          acc = x.x * qv[0] + x.y * qv[1];
+        }
+      }
+      part[u] = acc;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) part[u] = warp_sum(part[u]);
+    if (lane == 0) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = base + u * nw;
+        if (j < n) sc[j] = part[u] * scale + 0.0f;
+      }
+    }
+  }
+}
+
+// Best-first list of the min(k, n) best entries of sc[0..n) (blocks m0..).
+template <bool kGlobalOut>
+__device__ void chunk_topk(const float* sc, int m0, int n, int k, float* ls, int* li) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float si = sc[i];
+    int r = 0;
+    for (int j = 0; j < n; ++j) {
+      const float sj = sc[j];
+      r += (sj > si) || (sj == si && j < i);
+    }
+    if (r < k) {
+      ls[r] = si;
+      li[r] = m0 + i;
+    }
+  }
+}
+
+// Merge nchunk best-first lists (list c: len[c] entries at ls/li + c*k) into
+// the kk best entries, written to out_idx/out_logg in ascending block order
+// (log g = s - lse), padded to k with -1 / 0. sel_s/sel_m: kk-entry scratch
+// in shared memory. Loads go through L2 (.cg) because the lists may have
+// been written by other CTAs of the grid.
+template <typename X>
+__device__ __forceinline__ X ld_list(const X* p, bool global) {
+  return global ? __ldcg(p) : *p;
+}
+
+template <bool kGlobal>
+__device__ void merge_lists(const float* ls, const int* li, const int* len, int nchunk, int k,
+                            int kk, float lse, float* sel_s, int* sel_m,
+                            unsigned long long* theta_s, int32_t* out_idx, float* out_logg) {
+  const int tid = threadIdx.x;
+  if (tid == 0) *theta_s = 0ull;
+  __syncthreads();
+  for (int c = tid; c < nchunk; c += blockDim.x) {
+    const int L = ld_list(len + c, kGlobal);
+    if (L == k && k > 0) {
+      const unsigned long long key = cand_key(ld_list(ls + (size_t)c * k + k - 1, kGlobal),
+                                              ld_list(li + (size_t)c * k + k - 1, kGlobal));
+      atomicMax(theta_s, key);
+    }
+  }
+  __syncthreads();
+  const unsigned long long theta = *theta_s;
+  const int total = nchunk * k;
+  for (int e = tid; e < total; e += blockDim.x) {
+    const int c = e / k, p = e - c * k;
+    if (p >= ld_list(len + c, kGlobal)) continue;
+    const float s = ld_list(ls + e, kGlobal);
+    const int m = ld_list(li + e, kGlobal);
+    const unsigned long long key = cand_key(s, m);
+    if (key < theta) continue;
+    int rank = 0;
+    for (int c2 = 0; c2 < nchunk && rank < kk; ++c2) {
+      int lo = 0, hi = ld_list(len + c2, kGlobal);  // count entries of list c2 with a larger key
+      const float* s2 = ls + (size_t)c2 * k;
+      const int* m2 = li + (size_t)c2 * k;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const unsigned long long km = cand_key(ld_list(s2 + mid, kGlobal), ld_list(m2 + mid, kGlobal));
+        if (km > key) lo = mid + 1; else hi = mid;
+      }
+      rank += lo;
+    }
+    if (rank < kk) {
+      sel_s[rank] = s;
+      sel_m[rank] = m;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < kk; i += blockDim.x) {
+    const int mi = sel_m[i];
+    int pos = 0;
+    for (int j = 0; j < kk; ++j) pos += sel_m[j] < mi;
+    out_idx[pos] = mi;
+    out_logg[pos] = sel_s[i] - lse;
+  }
+  for (int i = kk + tid; i < k; i += blockDim.x) {
+    out_idx[i] = -1;
+    out_logg[i] = 0.f;
+  }
+}
+
+// ------------------------------------------------------------------ prefill
+// qbar[b, r, t] = mean of q over the group's G heads and query block t's rows.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_qbar_prefill(const T* __restrict__ q, int Hq, int Hkv,
+                                                      int N, float* __restrict__ qbar) {
+  constexpr int VEC = Vec16<T>::N;
+  constexpr int TPR = D / VEC;
+  constexpr int RP = 256 / TPR;
+  __shared__ float red[RP][D];
+  const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z, T_ = gridDim.x;
+  const int G = Hq / Hkv;
+  const int tid = threadIdx.x, c = tid % TPR, rg = tid / TPR;
+  const int row0 = t * SAS_BLOCK, nr = min(SAS_BLOCK, N - row0);
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+  for (int g = 0; g < G; ++g) {
+    const T* base = q + (((size_t)b * Hq + r * G + g) * N + row0) * D + c * VEC;
+    for (int i = rg; i < nr; i += RP) {
+      float x[VEC];
+      Vec16<T>::load_nc(base + (size_t)i * D, x);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) acc[u] += x[u];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) red[rg][c * VEC + i] = acc[i];
+  __syncthreads();
+  const float inv = 1.0f / (float)(G * nr);
+  float* out = qbar + (((size_t)b * Hkv + r) * T_ + t) * D;
+  for (int col = tid; col < D; col += 256) {
+    float s = 0.f;
+    for (int i = 0; i < RP; ++i) s += red[i][col];
+    out[col] = s * inv;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
+    const float* __restrict__ qbar, const float* __restrict__ ksum, int Hkv, int nblk, int topk,
+    float scale, int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z, T_ = gridDim.x;
+  const int C = t;
+  const int nchunk = (C + SEL_CHUNK_MAX - 1) / SEL_CHUNK_MAX;
+  float* q_s = reinterpret_cast<float*>(smem_raw);
+  float* sc = q_s + D;
+  float* red = sc + SEL_CHUNK_MAX;
+  float* sel_s = red + 32;
+  int* sel_m = reinterpret_cast<int*>(sel_s + 128);
+  unsigned long long* theta_s = reinterpret_cast<unsigned long long*>(sel_m + 128);
+  int* len = reinterpret_cast<int*>(theta_s + 1);
+  float* ls = reinterpret_cast<float*>(len + ((nchunk + 3) & ~3));
+  int* li = reinterpret_cast<int*>(ls + (size_t)nchunk * topk);
+
+  const size_t row = ((size_t)b * Hkv + r) * T_ + t;
+  const float* qrow = qbar + row * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) q_s[i] = qrow[i];
+  __syncthreads();
+  const float* ks_row = ksum + ((size_t)b * Hkv + r) * nblk * D;
+  float run_m = -FLT_MAX, run_s = 0.f;
+  for (int c = 0; c < nchunk; ++c) {
+    const int m0 = c * SEL_CHUNK_MAX, n = min(SEL_CHUNK_MAX, C - m0);
+    score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
+    __syncthreads();
+    if (topk > 0) chunk_topk<false>(sc, m0, n, topk, ls + (size_t)c * topk, li + (size_t)c * topk);
+    float lm = -FLT_MAX;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) lm = fmaxf(lm, sc[i]);
+    lm = block_reduce_max(lm, red);
+    float le = 0.f;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) le += __expf(sc[i] - lm);
+    le = block_reduce_sum(le, red);
+    const float nm = fmaxf(run_m, lm);
+    run_s = run_s * __expf(run_m - nm) + le * __expf(lm - nm);
+    run_m = nm;
+    if (threadIdx.x == 0) len[c] = min(topk, n);
+    __syncthreads();
+  }
+  const int kk = min(topk, C);
+  const float lse = (C > 0) ? run_m + __logf(run_s) : 0.f;
+  if (topk > 0)
+    merge_lists<false>(ls, li, len, nchunk, topk, kk, lse, sel_s, sel_m, theta_s, idx + row * topk,
+                logg + row * topk);
+  if (threadIdx.x == 0) cnt[row] = kk;
+}
+
+size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d) {
+  const int T_ = (N + SAS_BLOCK - 1) / SAS_BLOCK;
+  return (size_t)B * Hkv * T_ * d * sizeof(float);
+}
+
+static size_t prefill_select_smem(int d, int nchunk, int topk) {
+  size_t n = (size_t)d + SEL_CHUNK_MAX + 32 + 128 + 128;  // q, sc, red, sel_s, sel_m
+  n += 2;                                                 // theta (8 bytes)
+  n += (nchunk + 3) & ~3;                                 // len
+  n += 2 * (size_t)nchunk * topk;                         // ls, li
+  return n * 4;
+}
+
+cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                  int Hkv, int N, int d, int topk, float scale, int32_t* idx,
+                                  int32_t* cnt, float* logg, void* ws, cudaStream_t st) {
+  const int T_ = (N + SAS_BLOCK - 1) / SAS_BLOCK;
+  if (B == 0 || T_ == 0) return cudaSuccess;
+  float* qbar = static_cast<float*>(ws);
+  dim3 grid(T_, Hkv, B);
+#define SAS_QBAR(T, D) \
+  k_qbar_prefill<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(q), Hq, Hkv, N, qbar)
+  if (bf16) {
+    if (d == 128) SAS_QBAR(__nv_bfloat16, 128); else SAS_QBAR(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) SAS_QBAR(float, 128); else SAS_QBAR(float, 64);
+  }
+#undef SAS_QBAR
+  const int nblk = N / SAS_BLOCK;
+  const int nchunk_max = (T_ - 1 + SEL_CHUNK_MAX - 1) / SEL_CHUNK_MAX;
+  const size_t smem = prefill_select_smem(d, nchunk_max > 0 ? nchunk_max : 1, topk);
+  if (d == 128) {
+    ensure_smem(k_select_prefill<128>, smem);
+    k_select_prefill<128><<<grid, SEL_THREADS, smem, st>>>(qbar, ksum, Hkv, nblk, topk, scale,
+                                                           idx, cnt, logg);
+  } else {
+    ensure_smem(k_select_prefill<64>, smem);
+    k_select_prefill<64><<<grid, SEL_THREADS, smem, st>>>(qbar, ksum, Hkv, nblk, topk, scale,
+                                                          idx, cnt, logg);
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ decode
+// Scratch layout per plan (rows = B*Hkv, nchunk chunks per row):
+//   counters [rows] int | len [rows][nchunk] int | cmax, csum [rows][nchunk]
+//   float | ls [rows][nchunk][k] float | li [rows][nchunk][k] int
+struct DecodeSelectWs {
+  int* counter;
+  int* len;
+  float* cmax;
+  float* csum;
+  float* ls;
+  int* li;
+};
+
+static size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+static DecodeSelectWs carve_decode_select(int* counters, void* ws, const SelectPlan& p) {
+  DecodeSelectWs w;
+  char* c = static_cast<char*>(ws);
+  const size_t rc = (size_t)p.rows * p.nchunk;
+  w.counter = counters;
+  w.len = reinterpret_cast<int*>(c); c += align16(sizeof(int) * rc);
+  w.cmax = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc);
+  w.csum = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc);
+  w.ls = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc * p.topk);
+  w.li = reinterpret_cast<int*>(c);
+  return w;
+}
+
+size_t decode_select_ws_bytes(const SelectPlan& p) {
+  const size_t rc = (size_t)p.rows * p.nchunk;
+  return align16(sizeof(int) * rc) + 2 * align16(sizeof(float) * rc) +
+         align16(sizeof(float) * rc * p.topk) + align16(sizeof(int) * rc * p.topk);
+}
+
+SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk) {
+  SelectPlan p;
+  p.rows = B * Hkv;
+  p.topk = topk;
+  const int nblk = Lmax / SAS_BLOCK;
+  // Aim for about two CTAs per SM over all rows, chunks of 64..256 blocks.
+  const long long target = 2LL * 148;
+  int chunk = 64;
+  while (chunk < DEC_CHUNK_MAX &&
+         ((long long)p.rows * ((nblk + chunk - 1) / chunk) > target ||
+          (nblk + chunk - 1) / chunk > DEC_NCHUNK_MAX))
+    chunk *= 2;
+  p.chunk = chunk;
+  p.nchunk = nblk > 0 ? (nblk + chunk - 1) / chunk : 1;
+  return p;
+}
+
+static size_t decode_merge_smem(int nchunk, int topk) {
+  return sizeof(float) * (2 * (size_t)nchunk + ((nchunk + 3) & ~3) + 2 * (size_t)nchunk * topk);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
+    const T* __restrict__ q, const float* __restrict__ ksum, int Hq, int Hkv, int nblk,
+    const int32_t* __restrict__ lens, int topk, float scale, int chunk, DecodeSelectWs w,
+    int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg) {
+  __shared__ __align__(16) float q_s[D];
+  __shared__ float sc[DEC_CHUNK_MAX];
+  __shared__ float red[32];
+  __shared__ float sel_s[128];
+  __shared__ int sel_m[128];
+  __shared__ unsigned long long theta_s;
+  __shared__ int is_last;
+  // merge staging (last CTA of a row): the row's chunk partials and lists
+  extern __shared__ __align__(16) unsigned char dsm[];
+  const int c = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
+  const int nchunk = gridDim.x;
+  const int G = Hq / Hkv;
+  const int row = b * Hkv + r;
+  const int n_tok = min(max(lens[b], 1), nblk * SAS_BLOCK);  // 1 <= n <= Lmax
+  const int C = (n_tok - 1) / SAS_BLOCK;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    float s = 0.f;
+    for (int g = 0; g < G; ++g) s += to_f(q[((size_t)b * Hq + r * G + g) * D + i]);
+    q_s[i] = s / (float)G;
+  }
+  __syncthreads();
+  const int m0 = c * chunk, n = max(0, min(chunk, C - m0));
+  const float* ks_row = ksum + (size_t)row * nblk * D;
+  score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
+  __syncthreads();
+  const size_t rc = (size_t)row * nchunk + c;
+  if (topk > 0) chunk_topk<true>(sc, m0, n, topk, w.ls + rc * topk, w.li + rc * topk);
+  float lm = -FLT_MAX;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) lm = fmaxf(lm, sc[i]);
+  lm = block_reduce_max(lm, red);
+  float le = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) le += __expf(sc[i] - lm);
+  le = block_reduce_sum(le, red);
+  if (threadIdx.x == 0) {
+    w.len[rc] = min(topk, n);
+    w.cmax[rc] = lm;
+    w.csum[rc] = le;
+  }
+  // Publish this chunk, then count it; the last chunk of the row merges.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(w.counter + row, 1) == nchunk - 1);
+  __syncthreads();
+  // No explicit launch trigger: a programmatic dependent (the decode attention)
+  // is only guaranteed to see writes made before the trigger, and the merge
+  // below writes the selection it consumes. The implicit trigger at grid exit
+  // comes after every write.
+  if (!is_last) return;
+  __threadfence();
+  // Stage the row's partials in shared memory with one parallel pass of L2
+  // loads, then merge there (a serial walk over L2 would be latency-bound).
+  float* cm_s = reinterpret_cast<float*>(dsm);
+  float* cs_s = cm_s + nchunk;
+  int* len_s = reinterpret_cast<int*>(cs_s + nchunk);
+  float* ls_s = reinterpret_cast<float*>(len_s + ((nchunk + 3) & ~3));
+  int* li_s = reinterpret_cast<int*>(ls_s + (size_t)nchunk * topk);
+  const size_t r0 = (size_t)row * nchunk;
+  for (int i = threadIdx.x; i < nchunk; i += blockDim.x) {
+    cm_s[i] = __ldcg(w.cmax + r0 + i);  // empty chunks: -FLT_MAX and 0
+    cs_s[i] = __ldcg(w.csum + r0 + i);
+    len_s[i] = __ldcg(w.len + r0 + i);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < nchunk * topk; e += blockDim.x) {
+    const int cc = e / topk, p = e - cc * topk;
+    if (p < len_s[cc]) {
+      ls_s[e] = __ldcg(w.ls + r0 * topk + e);
+      li_s[e] = __ldcg(w.li + r0 * topk + e);
+    }
+  }
+  float mx = -FLT_MAX;
+  for (int i = threadIdx.x; i < nchunk; i += blockDim.x) mx = fmaxf(mx, cm_s[i]);
+  const float M = block_reduce_max(mx, red);
+  float lsum = 0.f;
+  for (int i = threadIdx.x; i < nchunk; i += blockDim.x)
+    if (cs_s[i] > 0.f) lsum += cs_s[i] * __expf(cm_s[i] - M);
+  const float S = block_reduce_sum(lsum, red);
+  const float lse = (C > 0) ? M + __logf(S) : 0.f;
+  const int kk = min(topk, C);
+  if (topk > 0)
+    merge_lists<false>(ls_s, li_s, len_s, nchunk, topk, kk, lse, sel_s, sel_m, &theta_s,
+                       idx + (size_t)row * topk, logg + (size_t)row * topk);
+  if (threadIdx.x == 0) {
+    cnt[row] = kk;
+    w.counter[row] = 0;  // ready for the next call
+  }
+}
+
+cudaError_t launch_select_decode(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                 int Hkv, int Lmax, int d, int topk, const int32_t* lens,
+                                 float scale, int32_t* idx, int32_t* cnt, float* logg,
+                                 const SelectPlan& plan, int* counters, void* ws,
+                                 cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  DecodeSelectWs w = carve_decode_select(counters, ws, plan);
+  const int nblk = Lmax / SAS_BLOCK;
+  dim3 grid(plan.nchunk, Hkv, B);
+const size_t smem = decode_merge_smem(plan.nchunk, topk);
+#define SAS_SELD(T, D)                                                                       \
+  do {                                                                                       \
+    ensure_smem(k_select_decode<T, D>, smem);                                                \
+    k_select_decode<T, D><<<grid, SEL_THREADS, smem, st>>>(static_cast<const T*>(q), ksum,   \
+                                                           Hq, Hkv, nblk, lens, topk, scale, \
+                                                           plan.chunk, w, idx, cnt, logg);   \
+  } while (0)
+  if (bf16) {
+    if (d == 128) SAS_SELD(__nv_bfloat16, 128); else SAS_SELD(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) SAS_SELD(float, 128); else SAS_SELD(float, 64);
+  }
+#undef SAS_SELD
+  return cudaGetLastError();
+}
+
+}  // namespace sas

@@ -1,0 +1,67 @@
+// Block summaries: the mean of each complete 64-key block (SAS close reading,
+// liuzhao09.github.io, section 2.1: a block summary compresses the block's
+// adjacent keys and is what the selector reads).
+//
+// One CTA per (block m, head h, sequence b); 256 threads. Each thread loads
+// 16-byte vectors of one key row and accumulates fp32 column sums; the row
+// groups are reduced through shared memory. HBM-bound: every key is read
+// once, 4 bytes per column are written per block.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sas {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_block_summary(const T* __restrict__ k, int N, int nblk,
+                                                       const int32_t* __restrict__ lens,
+                                                       float* __restrict__ ksum) {
+  constexpr int VEC = Vec16<T>::N;
+  constexpr int TPR = D / VEC;   // threads per key row
+  constexpr int RP = 256 / TPR;  // key rows per pass
+  __shared__ float red[RP][D];
+  const int m = blockIdx.x, h = blockIdx.y, b = blockIdx.z, H = gridDim.y;
+  const int tid = threadIdx.x, c = tid % TPR, rg = tid / TPR;
+  int nvalid = nblk;
+  if (lens) nvalid = min(nblk, lens[b] / SAS_BLOCK);
+  const T* base = k + (((size_t)b * H + h) * N + (size_t)m * SAS_BLOCK) * D + c * VEC;
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+  if (m < nvalid) {
+#pragma unroll
+    for (int r = rg; r < SAS_BLOCK; r += RP) {
+      float x[VEC];
+      Vec16<T>::load_nc(base + (size_t)r * D, x);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] += x[i];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) red[rg][c * VEC + i] = acc[i];
+  __syncthreads();
+  float* out = ksum + (((size_t)b * H + h) * nblk + m) * D;
+  for (int col = tid; col < D; col += 256) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < RP; ++r) s += red[r][col];
+    out[col] = (m < nvalid) ? s * (1.0f / SAS_BLOCK) : 0.f;
+  }
+}
+
+cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
+                                 const int32_t* lens, float* ksum, cudaStream_t st) {
+  const int nblk = N / SAS_BLOCK;
+  if (nblk == 0 || B == 0 || H == 0) return cudaSuccess;
+  dim3 grid(nblk, H, B);
+#define SAS_SUM(T, D) \
+  k_block_summary<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(k), N, nblk, lens, ksum)
+  if (bf16) {
+    if (d == 128) SAS_SUM(__nv_bfloat16, 128); else SAS_SUM(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) SAS_SUM(float, 128); else SAS_SUM(float, 64);
+  }
+#undef SAS_SUM
+  return cudaGetLastError();
+}
+
+}  // namespace sas

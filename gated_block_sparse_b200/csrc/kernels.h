@@ -1,0 +1,60 @@
+// Host-side launchers of the SAS kernels (internal; the public ABI is sas.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sas {
+
+// Block summaries: ksum[b,h,m] = mean of keys 64m..64m+63.
+cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
+                                 const int32_t* lens, float* ksum, cudaStream_t st);
+
+// ---- selection
+// Shared layout of one row's per-chunk partial results (decode scratch).
+struct SelectPlan {
+  int rows;       // number of selection rows
+  int chunk;      // history blocks per chunk
+  int nchunk;     // chunks per row
+  int topk;
+};
+SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk);
+size_t decode_select_ws_bytes(const SelectPlan& p);
+
+cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                  int Hkv, int N, int d, int topk, float scale, int32_t* idx,
+                                  int32_t* cnt, float* logg, void* ws, cudaStream_t st);
+size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d);
+
+// Decode selection. `counters` holds one int per row and must be zero on
+// entry (the kernel leaves it zero); `ws` holds the plan's partials.
+cudaError_t launch_select_decode(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                 int Hkv, int Lmax, int d, int topk, const int32_t* lens,
+                                 float scale, int32_t* idx, int32_t* cnt, float* logg,
+                                 const SelectPlan& plan, int* counters, void* ws,
+                                 cudaStream_t st);
+
+// ---- decode attention
+size_t decode_attend_ws_bytes(int B, int Hq, int Hkv, int topk, int d);
+cudaError_t launch_decode_attend(const void* q, const void* kc, const void* vc, int bf16, int B,
+                                 int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                                 const int32_t* idx, const int32_t* cnt, const float* logg,
+                                 int topk, int gated, float scale, void* o, int* counters,
+                                 void* ws, cudaStream_t st, bool pdl);
+uint32_t* decode_error_word();
+uint32_t* attn_simt_error_word();
+
+// ---- prefill attention (SIMT path: fp32 or bf16 inputs, any GPU of sm_100a)
+cudaError_t launch_attn_fwd_simt(const void* q, const void* k, const void* v, int bf16, int B,
+                                 int Hq, int Hkv, int N, int d, const int32_t* idx,
+                                 const int32_t* cnt, const float* logg, int topk, float scale,
+                                 void* o, float* lse, cudaStream_t st);
+size_t attn_bwd_simt_ws_bytes(int B, int Hkv, int N, int d);
+cudaError_t launch_attn_bwd_simt(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, int bf16, int B, int Hq, int Hkv, int N, int d,
+                                 const float* lse, const int32_t* idx, const int32_t* cnt,
+                                 const float* logg, int topk, float scale, void* dq, void* dk,
+                                 void* dv, float* dlogg, void* ws, cudaStream_t st);
+
+}  // namespace sas

@@ -1,0 +1,227 @@
+"""Python binding of libsas (include/sas.h): argument marshalling only.
+
+Each function has the name of the C entry point it calls. Tensors are torch
+CUDA tensors (torch provides device memory and the current stream); every step
+of the computation runs in the library's CUDA kernels. There is no CPU
+fallback: if libsas.so is missing or no GPU is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libsas.so")
+
+SAS_F32, SAS_BF16 = 0, 1
+SAS_PREFILL, SAS_DECODE = 0, 1
+STATUS = {0: "SAS_OK", 1: "SAS_ERR_INVALID_ARG", 2: "SAS_ERR_UNSUPPORTED", 3: "SAS_ERR_CUDA",
+          4: "SAS_ERR_TIMEOUT", 5: "SAS_ERR_INTERNAL"}
+
+# exported symbol -> (restype, argtypes)
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "sas_strerror": (ctypes.c_char_p, [_I]),
+    "sas_last_error_message": (ctypes.c_char_p, []),
+    "sas_version": (_I, []),
+    "sas_block_summary": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sas_select_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "sas_select": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F, _P, _P, _P, _P, _Z, _P]),
+    "sas_attn_fwd_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "sas_attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I, _F, _P, _P, _P, _Z,
+                          _P]),
+    "sas_attn_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
+    "sas_attn_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _F, _P,
+                          _P, _P, _P, _P, _Z, _P]),
+    "sas_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sas_decode_attend_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sas_decode_attend": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _F,
+                               _P, _P, _Z, _P]),
+    "sas_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P, _P, _Z,
+                        _P]),
+}
+
+_lib = None
+
+
+class SasError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsas.so (built in-tree by gated_block_sparse_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: run `python -m gated_block_sparse_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        msg = load_library().sas_last_error_message().decode()
+        raise SasError(fn, status, msg)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SAS_BF16
+    if t.dtype == torch.float32:
+        return SAS_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ws(nbytes: int, device, ws: torch.Tensor | None) -> torch.Tensor:
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def sas_block_summary(k: torch.Tensor, lens: torch.Tensor | None = None,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Mean of each complete 64-key block: k [B][H][N][d] -> [B][H][N//64][d] fp32."""
+    B, H, N, d = k.shape
+    if out is None:
+        out = torch.empty((B, H, N // 64, d), dtype=torch.float32, device=k.device)
+    _check("sas_block_summary", load_library().sas_block_summary(
+        _ptr(k), _dt(k), B, H, N, d, _ptr(lens), _ptr(out), _stream(stream)))
+    return out
+
+
+def sas_select(q: torch.Tensor, ksum: torch.Tensor, Hkv: int, topk: int, mode: str = "prefill",
+               lens: torch.Tensor | None = None, scale: float = 0.0, out=None, ws=None,
+               stream=None):
+    """Scores, gate and Top-K. Returns (idx int32, cnt int32, logg fp32).
+
+    prefill: q [B][Hq][N][d] -> idx/logg [B][Hkv][T][topk], cnt [B][Hkv][T].
+    decode:  q [B][Hq][d], N = Lmax = 64 * ksum.shape[2] -> idx/logg
+             [B][Hkv][topk], cnt [B][Hkv].
+    """
+    lib = load_library()
+    if mode == "prefill":
+        B, Hq, N, d = q.shape
+        T = -(-N // 64)
+        shape = (B, Hkv, T)
+        m = SAS_PREFILL
+    elif mode == "decode":
+        B, Hq, d = q.shape
+        N = ksum.shape[2] * 64
+        shape = (B, Hkv)
+        m = SAS_DECODE
+    else:
+        raise ValueError(mode)
+    if out is None:
+        out = (torch.empty(shape + (topk,), dtype=torch.int32, device=q.device),
+               torch.empty(shape, dtype=torch.int32, device=q.device),
+               torch.empty(shape + (topk,), dtype=torch.float32, device=q.device))
+    idx, cnt, logg = out
+    need = lib.sas_select_workspace_size(B, Hq, Hkv, N, d, topk, m)
+    w = _ws(need, q.device, ws)
+    _check("sas_select", lib.sas_select(
+        _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, m, _ptr(lens), float(scale),
+        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, _ptr(w),
+        w.numel(), _stream(stream)))
+    return idx, cnt, logg
+
+
+def sas_attn_fwd(q, k, v, idx, cnt, logg, scale: float = 0.0, out=None, ws=None, stream=None):
+    """Gated sparse prefill forward. Returns (o [B][Hq][N][d], lse [B][Hq][N] fp32)."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    topk = idx.shape[-1]
+    if out is None:
+        out = (torch.empty_like(q), torch.empty((B, Hq, N), dtype=torch.float32, device=q.device))
+    o, lse = out
+    need = lib.sas_attn_fwd_workspace_size(B, Hq, Hkv, N, d, topk, _dt(q))
+    w = _ws(need, q.device, ws)
+    _check("sas_attn_fwd", lib.sas_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(idx) if topk else None,
+        _ptr(cnt), _ptr(logg) if topk else None, topk, float(scale), _ptr(o), _ptr(lse),
+        _ptr(w), w.numel(), _stream(stream)))
+    return o, lse
+
+
+def sas_attn_bwd(q, k, v, o, dout, lse, idx, cnt, logg, scale: float = 0.0, out=None, ws=None,
+                 stream=None):
+    """Backward of sas_attn_fwd. Returns (dq, dk, dv, dlogg)."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    topk = idx.shape[-1]
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+               torch.empty(idx.shape, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dlogg = out
+    need = lib.sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, _dt(q))
+    w = _ws(need, q.device, ws)
+    _check("sas_attn_bwd", lib.sas_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _dt(q), B, Hq, Hkv, N, d, _ptr(lse),
+        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk,
+        float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlogg) if topk else None, _ptr(w),
+        w.numel(), _stream(stream)))
+    return dq, dk, dv, dlogg
+
+
+def sas_decode_workspace_size(B: int, Hq: int, Hkv: int, Lmax: int, d: int, topk: int) -> int:
+    return load_library().sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, topk)
+
+
+def sas_decode(q, kc, vc, lens, ksum, topk: int, gated: int = 1, scale: float = 0.0, out=None,
+               idx_out=None, ws=None, stream=None):
+    """One decode step: q [B][Hq][d], caches [B][Hkv][Lmax][d] -> o [B][Hq][d]."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Hkv, Lmax = kc.shape[1], kc.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    need = lib.sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, topk)
+    w = _ws(need, q.device, ws)
+    _check("sas_decode", lib.sas_decode(
+        _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens), _ptr(ksum), topk,
+        int(gated), float(scale), _ptr(out), _ptr(idx_out), _ptr(w), w.numel(), _stream(stream)))
+    return out
+
+
+def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: float = 0.0,
+                      out=None, ws=None, stream=None):
+    """Decode attention for a given selection (idx/cnt/logg as sas_select's
+    decode outputs): q [B][Hq][d] -> o [B][Hq][d]."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Hkv, Lmax = kc.shape[1], kc.shape[2]
+    topk = idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = lib.sas_decode_attend_workspace_size(B, Hq, Hkv, Lmax, d, topk)
+    w = _ws(need, q.device, ws)
+    _check("sas_decode_attend", lib.sas_decode_attend(
+        _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens),
+        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
+        float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
+    return out

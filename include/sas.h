@@ -1,0 +1,193 @@
+/*
+ * sas.h -- C ABI of the SAS gated block-sparse causal attention library
+ * (libsas.so, CUDA kernels for sm_100a).
+ *
+ * The method (SAS close reading, liuzhao09.github.io, sections 2.1, 2.2 and
+ * 2.4; SAS reproduction note, daiwk.github.io, core formula):
+ *   - the sequence is cut into contiguous blocks of b = 64 tokens;
+ *   - each history block m has a summary kbar_m (the mean of its 64 keys);
+ *   - a selector scores the C causally visible history blocks,
+ *     s_m = scale * qbar . kbar_m, scale = 1/sqrt(d) by default;
+ *   - the gate is g = softmax(s) over those C blocks, g0 = 1 for the current
+ *     block, log g_m = s_m - LSE(s);
+ *   - I = TopK(s, k) (ties go to the lower block index), S = B0 + I, with B0
+ *     the current block, always kept and causally masked;
+ *   - o = softmax(q K_S^T * scale + log g_S) V_S;
+ *   - the backward pass returns dQ, dK, dV and, per selected block, d(log g):
+ *     the sum of the logit gradients inside that block.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer, allocated and owned by the
+ *     caller. The library never allocates, frees or synchronises; all work is
+ *     enqueued on `stream` (NULL = the legacy default stream) and the call
+ *     returns as soon as it is enqueued.
+ *   - Layouts are dense row-major ("HND"): q, o, dO, dq [B][Hq][N][d];
+ *     k, v, dk, dv [B][Hkv][N][d]; decode q/o [B][Hq][d]; caches
+ *     [B][Hkv][Lmax][d]; block summaries [B][Hkv][N/64][d] fp32.
+ *     Selection rows: prefill idx/logg/dlogg [B][Hkv][T][topk] and cnt
+ *     [B][Hkv][T] with T = ceil(N/64); decode idx [B][Hkv][topk].
+ *     idx lists the kept history blocks in ascending order, padded with -1;
+ *     cnt = min(topk, C).
+ *   - Element type of q/k/v/o/dO/dq/dk/dv/caches: SAS_BF16 or SAS_F32, the
+ *     same for all of them in one call. Scores, gates, lse and summaries are
+ *     fp32; accumulation is fp32.
+ *   - Supported: d in {64, 128}; block size 64 (fixed); Hq % Hkv == 0;
+ *     Hq/Hkv <= 8; 1 <= topk <= 128 (topk = 0 is accepted where stated);
+ *     every pointer 16-byte aligned. Other shapes return SAS_ERR_UNSUPPORTED.
+ *   - scale <= 0 selects the default 1/sqrt(d).
+ *   - Invalid arguments are rejected on the host before any launch, with
+ *     SAS_ERR_INVALID_ARG and a message in sas_last_error_message().
+ *   - Workspace: each call that needs scratch memory states its size through
+ *     a *_workspace_size() function; pass a caller-owned device buffer of at
+ *     least that many bytes (16-byte aligned) as ws/ws_bytes. Contents need
+ *     not be initialised. Calls that share a workspace must not overlap.
+ *   - Calls are stateless apart from the workspace and may be captured in a
+ *     CUDA graph.
+ */
+#ifndef SAS_H
+#define SAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* sas_stream_t;
+
+typedef enum sas_status {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or argument      */
+  SAS_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, group, topk)    */
+  SAS_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed          */
+  SAS_ERR_TIMEOUT = 4,      /* reserved: a bounded device wait gave up       */
+  SAS_ERR_INTERNAL = 5      /* an internal consistency check failed          */
+} sas_status;
+
+typedef enum sas_dtype { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
+typedef enum sas_mode { SAS_PREFILL = 0, SAS_DECODE = 1 } sas_mode;
+
+/* Static text for a status code. */
+const char* sas_strerror(sas_status status);
+/* Detail of the last failing call on this host thread ("" if none). */
+const char* sas_last_error_message(void);
+/* Library version, major*10000 + minor*100 + patch. */
+int sas_version(void);
+
+/*
+ * Block summaries (SAS close reading, section 2.1: a block summary compresses
+ * the block's adjacent keys; here the mean of the 64 keys).
+ *   k     [B][H][N][d] (dt)              input
+ *   lens  [B] int32 or NULL              valid length per sequence; blocks
+ *                                        not complete within lens[b] get 0
+ *   ksum  [B][H][N/64][d] fp32           output, ksum[b,h,m] = mean of keys
+ *                                        64m .. 64m+63
+ * No workspace. N/64 == 0 is a no-op.
+ */
+sas_status sas_block_summary(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                             const int32_t* lens, float* ksum, sas_stream_t stream);
+
+/*
+ * Selector scores, normalised gate and Top-K (SAS close reading, sections 2.1
+ * and 2.2: s = R(q, {K_Bm}), I = TopK(s, k), g = softmax(s), log g = s - LSE).
+ * The selector is parameter-free: s_m = scale * qbar . ksum_m.
+ *   mode SAS_PREFILL: q [B][Hq][N][d]; one row per (b, kv group r, query
+ *     block t), qbar = mean of q over the group's Hq/Hkv heads and the query
+ *     block's tokens, C = t. Outputs idx/logg [B][Hkv][T][topk], cnt
+ *     [B][Hkv][T]. lens must be NULL.
+ *   mode SAS_DECODE: q [B][Hq][d] (one token per sequence at position
+ *     lens[b]-1); one row per (b, r), qbar = mean over the group's heads,
+ *     C = (lens[b]-1)/64. N is Lmax. Outputs idx/logg [B][Hkv][topk], cnt
+ *     [B][Hkv]. lens [B] int32 device, 1 <= lens[b] <= N.
+ *   ksum  [B][Hkv][N/64][d] fp32 (from sas_block_summary)
+ *   logg  log g of each kept block (padding slots 0)
+ *   topk >= 0; topk = 0 gives cnt = 0.
+ * Workspace: sas_select_workspace_size().
+ */
+size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_mode mode);
+sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
+                      int N, int d, int topk, sas_mode mode, const int32_t* lens, float scale,
+                      int32_t* idx, int32_t* cnt, float* logg, void* ws, size_t ws_bytes,
+                      sas_stream_t stream);
+
+/*
+ * Gated sparse attention forward for prefill/training (SAS close reading,
+ * sections 2.2 and 2.4; reproduction note, core formula):
+ *   o_i = sum_j softmax_j(z_ij) v_j,  lse_i = log sum_j exp(z_ij),
+ *   z_ij = scale * q_i . k_j + logg[slot(j)] for keys of kept history blocks,
+ *   z_ij = scale * q_i . k_j for keys j <= i of the current block.
+ * Unselected blocks are skipped, never masked.
+ *   q [B][Hq][N][d], k, v [B][Hkv][N][d]     inputs (dt)
+ *   idx, cnt, logg                           prefill selection rows (any
+ *     selection is accepted: ascending distinct indices < t, -1 padded)
+ *   o [B][Hq][N][d] (dt), lse [B][Hq][N] fp32 outputs
+ * Workspace: sas_attn_fwd_workspace_size() (may be 0).
+ */
+size_t sas_attn_fwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_dtype dt);
+sas_status sas_attn_fwd(const void* q, const void* k, const void* v, sas_dtype dt, int B, int Hq,
+                        int Hkv, int N, int d, const int32_t* idx, const int32_t* cnt,
+                        const float* logg, int topk, float scale, void* o, float* lse, void* ws,
+                        size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Backward of the forward above for L with dL/do = dO (SAS close reading,
+ * section 2.4 and eq. 5): with p recomputed from lse,
+ *   D_i = dO_i . o_i, dp_ij = dO_i . v_j, dz_ij = p_ij (dp_ij - D_i),
+ *   dq_i = scale sum_j dz_ij k_j, dk_j = scale sum_i dz_ij q_i,
+ *   dv_j = sum_i p_ij dO_i,
+ *   dlogg[b,r,t,slot] = sum over the group's heads, the rows of query block t
+ *     and the slot's 64 keys of dz.
+ *   o, lse: the forward's outputs for the same inputs.
+ *   dq [B][Hq][N][d], dk, dv [B][Hkv][N][d] (dt), dlogg [B][Hkv][T][topk]
+ *   fp32 outputs; padding slots of dlogg are 0. Outputs are overwritten.
+ * Workspace: sas_attn_bwd_workspace_size().
+ */
+size_t sas_attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_dtype dt);
+sas_status sas_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, sas_dtype dt, int B, int Hq, int Hkv, int N, int d,
+                        const float* lse, const int32_t* idx, const int32_t* cnt,
+                        const float* logg, int topk, float scale, void* dq, void* dk, void* dv,
+                        float* dlogg, void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * One decode step (SAS close reading, section 2.4 serving path: GQA groups
+ * share one block set; section 2.1: the current block is always kept):
+ * selection as sas_select(SAS_DECODE), then for every head h of group r
+ *   o_h = softmax(scale * q_h K_S^T + bias) V_S over the kept blocks and the
+ *   lens[b]-64t tokens of the current block t = (lens[b]-1)/64, with
+ *   bias = logg of the key's block when gated = 1 and 0 when gated = 0
+ *   (the inference-time "Algorithm 2" reading, section 2.1).
+ *   q [B][Hq][d], kc, vc [B][Hkv][Lmax][d] (dt), lens [B] int32 device
+ *   ksum [B][Hkv][Lmax/64][d] fp32 summaries of the cache
+ *   o [B][Hq][d] (dt) output; idx_out [B][Hkv][topk] int32 or NULL
+ * Workspace: sas_decode_workspace_size().
+ */
+size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk);
+sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype dt, int B, int Hq,
+                      int Hkv, int Lmax, int d, const int32_t* lens, const float* ksum, int topk,
+                      int gated, float scale, void* o, int32_t* idx_out, void* ws,
+                      size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Decode attention for a given selection: the attention half of sas_decode,
+ * with idx/cnt/logg as inputs (layouts of sas_select(SAS_DECODE)), so that any
+ * selection and any gate can be applied. Same definition as sas_decode
+ * (SAS close reading, sections 2.1, 2.2 and 2.4).
+ *   idx [B][Hkv][topk] int32 (ascending, < (lens[b]-1)/64), cnt [B][Hkv],
+ *   logg [B][Hkv][topk] fp32; o [B][Hq][d] (dt) output.
+ * Workspace: sas_decode_attend_workspace_size().
+ */
+size_t sas_decode_attend_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk);
+sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_dtype dt, int B,
+                             int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                             const int32_t* idx, const int32_t* cnt, const float* logg, int topk,
+                             int gated, float scale, void* o, void* ws, size_t ws_bytes,
+                             sas_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAS_H */

@@ -181,7 +181,7 @@ def _token_set(t, N, sel, sel_logg):
     return np.concatenate(pos), np.concatenate(bias), cur
 
 
-def _block_rows(qt, kS, vS, bias, cur, dot=None, scale=1.0):
+def _block_rows(qt, kS, vS, bias, cur, dot=None, scale=1.0, o_for_D=None):
     """Forward (and, with dot, backward) for the rows of one query block.
 
     qt [nr][d] are the rows i = cur[0..nr-1]; kS, vS [ns][d] the token set
@@ -190,6 +190,10 @@ def _block_rows(qt, kS, vS, bias, cur, dot=None, scale=1.0):
     z = scale * q k^T + bias; p = softmax(z); o = p V; lse = log sum e^z.
     Backward of L = sum(dO * o): D_i = dO_i . o_i, dp = dO V^T,
     dz = p (dp - D), dq = scale dz K, dK = scale dz^T Q, dV = p^T dO.
+    o_for_D, when given, is the output as the forward stored it (rounded to
+    the storage dtype), or a function mapping the exact rows of o to their
+    stored form; D then uses it, as the backward's interface defines D from
+    the forward's output.
     """
     nr = qt.shape[0]
     nhist = kS.shape[0] - cur.shape[0]
@@ -204,7 +208,9 @@ def _block_rows(qt, kS, vS, bias, cur, dot=None, scale=1.0):
     lse = (mx + np.log(ssum))[:, 0]
     if dot is None:
         return o, lse
-    D = (dot * o).sum(axis=1, keepdims=True)
+    if callable(o_for_D):
+        o_for_D = o_for_D(o)
+    D = (dot * (o if o_for_D is None else o_for_D)).sum(axis=1, keepdims=True)
     dp = dot @ vS.T
     dz = p * (dp - D)
     dq = scale * (dz @ kS)
@@ -241,13 +247,16 @@ def attn_fwd(q, k, v, idx, cnt, logg, scale: float | None = None):
     return o, lse
 
 
-def attn_bwd(q, k, v, do, idx, cnt, logg, scale: float | None = None):
+def attn_bwd(q, k, v, do, idx, cnt, logg, scale: float | None = None, o_stored=None):
     """Gradients of L = sum(dO * o) with o from attn_fwd.
 
     dlogg[b, r, t, slot] = sum over the group's heads, the rows of query
     block t and the slot's 64 keys of the logit gradient dz (section 2.4).
-    Returns dq, dk, dv, dlogg.
+    o_stored: optional forward output as stored (see _block_rows); the row
+    term D_i = dO_i . o_i then uses it. Returns dq, dk, dv, dlogg.
     """
+    if o_stored is not None and not callable(o_stored):
+        o_stored = _f64(o_stored)
     q, k, v, do, logg = _f64(q), _f64(k), _f64(v), _f64(do), _f64(logg)
     idx, cnt = np.asarray(idx), np.asarray(cnt)
     B, Hq, N, d = q.shape
@@ -267,7 +276,9 @@ def attn_bwd(q, k, v, do, idx, cnt, logg, scale: float | None = None):
                 pos, bias, cur = _token_set(t, N, idx[b, r, t, :kk], logg[b, r, t, :kk])
                 _, _, dqt, dkS, dvS, dz = _block_rows(
                     q[b, h, cur], k[b, r, pos], v[b, r, pos], bias, cur,
-                    dot=do[b, h, cur], scale=scale)
+                    dot=do[b, h, cur], scale=scale,
+                    o_for_D=o_stored if (o_stored is None or callable(o_stored))
+                    else o_stored[b, h, cur])
                 dq[b, h, cur] = dqt
                 np.add.at(dk[b, r], pos, dkS)
                 np.add.at(dv[b, r], pos, dvS)
@@ -277,13 +288,15 @@ def attn_bwd(q, k, v, do, idx, cnt, logg, scale: float | None = None):
 
 
 def query_block(q, k, v, do, idx, cnt, logg, b: int, r: int, t: int,
-                scale: float | None = None):
+                scale: float | None = None, o_stored=None):
     """Forward and backward restricted to query block t of kv group r.
 
     The same definitions as attn_fwd / attn_bwd, for sampled checks of
     full-size workloads. Returns per head of the group: o, lse, dq (rows of
     block t), and dlogg[slot] summed over the group's heads, plus this
     block's dk/dv contributions {position array, dk rows, dv rows}.
+    o_stored: optional function mapping exact output rows to their stored
+    form, used for the row term D as in attn_bwd.
     """
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
@@ -297,7 +310,8 @@ def query_block(q, k, v, do, idx, cnt, logg, b: int, r: int, t: int,
                dk=np.zeros_like(kS), dv=np.zeros_like(vS))
     for h in range(r * G, (r + 1) * G):
         o, lse, dq, dkS, dvS, dz = _block_rows(
-            _f64(q[b, h, cur]), kS, vS, bias, cur, dot=_f64(do[b, h, cur]), scale=scale)
+            _f64(q[b, h, cur]), kS, vS, bias, cur, dot=_f64(do[b, h, cur]), scale=scale,
+            o_for_D=o_stored)
         out["o"].append(o)
         out["lse"].append(lse)
         out["dq"].append(dq)
@@ -309,7 +323,7 @@ def query_block(q, k, v, do, idx, cnt, logg, b: int, r: int, t: int,
 
 
 def key_block_grads(q, k, v, do, idx, cnt, logg, b: int, r: int, j: int,
-                    scale: float | None = None):
+                    scale: float | None = None, o_stored=None):
     """dk, dv of key block j of kv group r: the sum of the contributions of
     every query block that selected j, and of query block j itself (for
     which j is the current block)."""
@@ -322,7 +336,7 @@ def key_block_grads(q, k, v, do, idx, cnt, logg, b: int, r: int, j: int,
         kk = int(cnt[b, r, t])
         if t != j and j not in set(int(x) for x in idx[b, r, t, :kk]):
             continue
-        res = query_block(q, k, v, do, idx, cnt, logg, b, r, t, scale)
+        res = query_block(q, k, v, do, idx, cnt, logg, b, r, t, scale, o_stored)
         hit = (res["pos"] >= lo) & (res["pos"] < lo + BLOCK)
         np.add.at(dk, res["pos"][hit] - lo, res["dk"][hit])
         np.add.at(dv, res["pos"][hit] - lo, res["dv"][hit])
@@ -346,6 +360,23 @@ def decode(q, kc, vc, lens, ksum, Hkv: int, topk: int, gated: int = 1,
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     idx, cnt, logg, _ = select_decode(q, ksum, lens, Hkv, topk, scale)
+    o, lse = decode_attend(q, kc, vc, lens, idx, cnt, logg, Hkv, gated, scale)
+    return o, idx, cnt, lse
+
+
+def decode_attend(q, kc, vc, lens, idx, cnt, logg, Hkv: int, gated: int = 1,
+                  scale: float | None = None):
+    """Decode attention for a given selection: every head of kv group r
+    attends over the kept blocks idx[b, r, :cnt] (bias log g when gated=1,
+    none when gated=0) and the n-64t tokens of the current block.
+    Returns o [B][Hq][d], lse [B][Hq]."""
+    q = _f64(q)
+    logg = _f64(logg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, d = q.shape
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
     o = np.zeros((B, Hq, d))
     lse = np.zeros((B, Hq))
     for b in range(B):
@@ -371,4 +402,4 @@ def decode(q, kc, vc, lens, ksum, Hkv: int, topk: int, gated: int = 1,
                 e = np.exp(z - mx)
                 o[b, h] = (e / e.sum()) @ vr
                 lse[b, h] = mx + np.log(e.sum())
-    return o, idx, cnt, lse
+    return o, lse

@@ -1,0 +1,103 @@
+"""The C ABI loads, exports every entry point include/sas.h declares, and
+rejects bad arguments on the host before any launch (CPU only: no call here
+reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_block_sparse_b200 import sas
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sas.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sas_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_block_sparse_b200 import build
+    build.build()
+    return sas.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) == 14
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in sas.SIGNATURES, n
+
+
+def test_strerror_and_version(lib):
+    assert lib.sas_version() == 100
+    for code, text in [(0, b"ok"), (1, b"invalid argument"), (2, b"unsupported configuration"),
+                       (3, b"CUDA error"), (4, b"device wait timed out"), (5, b"internal error")]:
+        assert lib.sas_strerror(code) == text
+
+
+def test_workspace_sizes_are_consistent(lib):
+    # decode workspace grows with batch and top-k and is 16-byte granular
+    a = lib.sas_decode_workspace_size(1, 32, 8, 65536, 128, 15)
+    b = lib.sas_decode_workspace_size(8, 32, 8, 131072, 128, 31)
+    assert a > 0 and b > a and a % 16 == 0 and b % 16 == 0
+    # prefill selection needs one fp32 query summary per (b, group, block)
+    assert lib.sas_select_workspace_size(1, 32, 8, 16384, 128, 31, 0) == 8 * 256 * 128 * 4
+    assert lib.sas_attn_bwd_workspace_size(1, 32, 8, 16384, 128, 31, 1) == 2 * 8 * 16384 * 128 * 4
+    assert lib.sas_decode_workspace_size(0, 32, 8, 65536, 128, 15) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_rejects_bad_head_dim(lib):
+    st = lib.sas_block_summary(FAKE, 1, 1, 2, 128, 96, None, FAKE, None)
+    assert st == 2 and b"head dim" in lib.sas_last_error_message()
+
+
+def test_rejects_group_mismatch(lib):
+    st = lib.sas_attn_fwd(FAKE, FAKE, FAKE, 1, 1, 6, 4, 128, 64, FAKE, FAKE, FAKE, 2, 0.0, FAKE,
+                          FAKE, None, 0, None)
+    assert st == 1 and b"multiple" in lib.sas_last_error_message()
+
+
+def test_rejects_null_and_misaligned_pointers(lib):
+    st = lib.sas_attn_fwd(None, FAKE, FAKE, 1, 1, 4, 4, 128, 64, FAKE, FAKE, FAKE, 2, 0.0, FAKE,
+                          FAKE, None, 0, None)
+    assert st == 1 and b"q must not be NULL" in lib.sas_last_error_message()
+    st = lib.sas_attn_fwd(FAKE + 4, FAKE, FAKE, 1, 1, 4, 4, 128, 64, FAKE, FAKE, FAKE, 2, 0.0,
+                          FAKE, FAKE, None, 0, None)
+    assert st == 1 and b"aligned" in lib.sas_last_error_message()
+
+
+def test_rejects_topk_and_workspace(lib):
+    st = lib.sas_select(FAKE, 1, FAKE, 1, 4, 4, 128, 64, 129, 0, None, 0.0, FAKE, FAKE, FAKE,
+                        FAKE, 1 << 20, None)
+    assert st == 2
+    st = lib.sas_select(FAKE, 1, FAKE, 1, 4, 4, 128, 64, 2, 0, None, 0.0, FAKE, FAKE, FAKE,
+                        FAKE, 16, None)
+    assert st == 1 and b"workspace too small" in lib.sas_last_error_message()
+
+
+def test_rejects_bad_decode_shapes(lib):
+    ws = lib.sas_decode_workspace_size(1, 32, 8, 65536, 128, 15)
+    st = lib.sas_decode(FAKE, FAKE, FAKE, 1, 1, 24, 8, 65536, 128, FAKE, FAKE, 15, 1, 0.0, FAKE,
+                        None, FAKE, ws, None)
+    assert st == 2  # 3 query heads per kv head is not a supported group size
+    st = lib.sas_decode(FAKE, FAKE, FAKE, 1, 1, 32, 8, 65000, 128, FAKE, FAKE, 15, 1, 0.0, FAKE,
+                        None, FAKE, ws, None)
+    assert st == 1 and b"multiple of 64" in lib.sas_last_error_message()
+    st = lib.sas_decode(FAKE, FAKE, FAKE, 1, 1, 32, 8, 65536, 128, FAKE, FAKE, 15, 2, 0.0, FAKE,
+                        None, FAKE, ws, None)
+    assert st == 1 and b"gated" in lib.sas_last_error_message()
+
+
+def test_empty_inputs_are_noops(lib):
+    # B = 0 or N = 0: nothing to do, no pointer needed, no launch
+    assert lib.sas_attn_fwd(None, None, None, 1, 0, 4, 4, 128, 64, None, None, None, 2, 0.0, None,
+                            None, None, 0, None) == 0
+    assert lib.sas_block_summary(None, 1, 1, 2, 63, 64, None, None, None) == 0

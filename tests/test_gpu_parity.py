@@ -1,0 +1,326 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Bars: block indices and counts bit-exact; floating-point outputs within
+max-abs 2e-2 for bf16 data and 1e-4 for fp32 data (o, lse, dq, dk, dv, dlogg,
+log g). An output stored in bf16 cannot be nearer the fp64 value than its own
+rounding, so for those outputs the bound is 2e-2 + 2^-8 |ref| (the bf16 unit
+roundoff); fp32-stored outputs (lse, dlogg, log g) get the plain bound.
+Summaries are fp32 sums of 64 values: 1e-5.
+
+The backward's row term is D_i = dO_i . o_i with o as the forward stored it
+(the interface passes the stored output in); the oracle's backward is given
+its own forward output rounded to the same storage dtype.
+
+Both sides consume the same stored bytes: the seeded generators produce
+bf16/fp32 tensors, the oracle upcasts them to fp64. Where a test feeds a
+selection to the attention kernels it is the oracle's (idx, cnt, and log g
+rounded to fp32), so the attention parity does not depend on the selection
+parity, which is tested on its own.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_block_sparse_b200 import inputs, sas
+from oracle import sas_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+
+
+def dev(t):
+    return t.to(DEV).contiguous()
+
+
+def np64(t):
+    return t.detach().cpu().double().numpy()
+
+
+def maxerr(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    return 0.0 if a.size == 0 else float(np.abs(a - b).max())
+
+
+def excess(got, ref, base, stored_bf16):
+    """Largest |got - ref| beyond the bound (<= 0 passes)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    if got.size == 0:
+        return -base
+    bound = base + (2.0 ** -8) * np.abs(ref) if stored_bf16 else base
+    return float((np.abs(got - ref) - bound).max())
+
+
+def stored(dtype):
+    return lambda rows: inputs.to_storage(rows, dtype).double().numpy()
+
+
+def boundary_gap(scores: dict, topk: int) -> float:
+    g = np.inf
+    for s in scores.values():
+        if len(s) > topk:
+            ss = np.sort(s)[::-1]
+            g = min(g, ss[topk - 1] - ss[topk])
+    return g
+
+
+def oracle_selection(q, k, Hkv, topk):
+    ks = O.block_summary(k)
+    idx, cnt, logg, scores = O.select_prefill(q, ks, Hkv, topk)
+    return idx, cnt, logg.astype(np.float32), scores
+
+
+# ------------------------------------------------------------------ summaries
+@pytest.mark.parametrize("dtype,d,N", [("bf16", 128, 1000), ("f32", 64, 640), ("bf16", 64, 64),
+                                       ("f32", 128, 130)])
+def test_block_summary(dtype, d, N):
+    k = inputs.gen_prefill(2, 2, 2, N, d, dtype, seed=11)["k"]
+    got = sas.sas_block_summary(dev(k))
+    torch.cuda.synchronize()
+    assert maxerr(np64(got), O.block_summary(k)) < 1e-5
+
+
+def test_block_summary_lens():
+    k = inputs.gen_prefill(3, 2, 2, 512, 128, "bf16", seed=12)["k"]
+    lens = torch.tensor([512, 200, 1], dtype=torch.int32)
+    got = sas.sas_block_summary(dev(k), lens=dev(lens))
+    torch.cuda.synchronize()
+    assert maxerr(np64(got), O.block_summary(k, lens=lens.numpy())) < 1e-5
+
+
+# ------------------------------------------------------------------ selection
+def _check_select(q, k, Hkv, topk, tol):
+    ks = sas.sas_block_summary(dev(k))
+    idx, cnt, logg = sas.sas_select(dev(q), ks, Hkv, topk, "prefill")
+    torch.cuda.synchronize()
+    oi, oc, ol, scores = oracle_selection(q, k, Hkv, topk)
+    assert np.array_equal(cnt.cpu().numpy(), oc)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    assert maxerr(np64(logg), ol) < tol
+    return scores
+
+
+def test_select_prefill_c1():
+    x = inputs.gen_config("c1")
+    c = inputs.CONFIGS["c1"]
+    scores = _check_select(x["q"], x["k"], c["Hkv"], c["topk"], 1e-5)
+    assert boundary_gap(scores, c["topk"]) >= 1.5e-3
+
+
+@pytest.mark.parametrize("N,d,topk", [(2048, 128, 7), (1000, 64, 3), (4096, 128, 31)])
+def test_select_prefill_planted_bf16(N, d, topk):
+    x = inputs.gen_prefill(2, 8, 2, N, d, "bf16", seed=20 + N, plant="ramp")
+    scores = _check_select(x["q"], x["k"], 2, topk, 1e-4)
+    assert boundary_gap(scores, topk) >= 1.5e-3
+
+
+def test_select_prefill_many_chunks():
+    # C up to 319 history blocks: two score chunks and a list merge per row
+    x = inputs.gen_prefill(1, 2, 1, 20480, 64, "bf16", seed=33, plant="ramp")
+    scores = _check_select(x["q"], x["k"], 1, 40, 1e-4)
+    assert boundary_gap(scores, 40) >= 1.5e-3
+
+
+def test_select_prefill_exact_ties():
+    x = inputs.gen_prefill(1, 4, 2, 1024, 128, "bf16", seed=34)
+    k = torch.zeros_like(x["k"])
+    _check_select(x["q"], k, 2, 5, 1e-5)  # all scores 0: lowest indices, log g = -log C
+
+
+def test_select_prefill_topk_zero():
+    x = inputs.gen_prefill(1, 4, 2, 512, 64, "f32", seed=35)
+    ks = sas.sas_block_summary(dev(x["k"]))
+    idx, cnt, logg = sas.sas_select(dev(x["q"]), ks, 2, 0, "prefill")
+    torch.cuda.synchronize()
+    assert int(cnt.abs().sum()) == 0
+
+
+# ------------------------------------------------------------------ attention
+def _fwd_bwd_check(x, Hkv, topk, dtype, sel=None):
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    if sel is None:
+        sel = oracle_selection(q, k, Hkv, topk)
+    idx, cnt, logg = sel[:3]
+    dq_, dk_, dv_, do_ = dev(q), dev(k), dev(v), dev(do)
+    ti, tc, tl = dev(torch.from_numpy(idx)), dev(torch.from_numpy(cnt)), dev(torch.from_numpy(logg))
+    o, lse = sas.sas_attn_fwd(dq_, dk_, dv_, ti, tc, tl)
+    gq, gk, gv, gl = sas.sas_attn_bwd(dq_, dk_, dv_, o, do_, lse, ti, tc, tl)
+    torch.cuda.synchronize()
+    oo, olse = O.attn_fwd(q, k, v, idx, cnt, logg)
+    oq, okk, ov, ol = O.attn_bwd(q, k, v, do, idx, cnt, logg, o_stored=stored(dtype))
+    tol = TOL[dtype]
+    bf = dtype == "bf16"
+    errs = dict(o=excess(np64(o), oo, tol, bf), lse=excess(np64(lse), olse, tol, False),
+                dq=excess(np64(gq), oq, tol, bf), dk=excess(np64(gk), okk, tol, bf),
+                dv=excess(np64(gv), ov, tol, bf), dlogg=excess(np64(gl), ol, tol, False))
+    for name, e in errs.items():
+        assert e <= 0, (name, e, errs)
+    return errs
+
+
+def test_attn_c1_fp32():
+    c = inputs.CONFIGS["c1"]
+    _fwd_bwd_check(inputs.gen_config("c1"), c["Hkv"], c["topk"], "f32")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,topk", [(1, 8, 2, 1000, 128, 3), (2, 4, 4, 576, 64, 2),
+                                               (1, 8, 1, 768, 128, 5)])
+def test_attn_bf16_ragged(B, Hq, Hkv, N, d, topk):
+    x = inputs.gen_prefill(B, Hq, Hkv, N, d, "bf16", seed=40 + N)
+    _fwd_bwd_check(x, Hkv, topk, "bf16")
+
+
+def test_attn_dense_equivalence_bf16():
+    # every history block selected and log g = 0: plain causal attention
+    x = inputs.gen_prefill(1, 4, 2, 512, 128, "bf16", seed=50)
+    T = 8
+    idx = np.full((1, 2, T, T), -1, dtype=np.int32)
+    cnt = np.zeros((1, 2, T), dtype=np.int32)
+    for t in range(T):
+        idx[:, :, t, :t] = np.arange(t)
+        cnt[:, :, t] = t
+    _fwd_bwd_check(x, 2, T, "bf16", sel=(idx, cnt, np.zeros((1, 2, T, T), np.float32)))
+
+
+def test_attn_topk_zero_current_block_only():
+    x = inputs.gen_prefill(1, 2, 2, 256, 64, "f32", seed=51)
+    sel = (np.zeros((1, 2, 4, 0), np.int32), np.zeros((1, 2, 4), np.int32),
+           np.zeros((1, 2, 4, 0), np.float32))
+    q, k, v = (dev(x[n]) for n in ("q", "k", "v"))
+    o, lse = sas.sas_attn_fwd(q, k, v, dev(torch.zeros(1, 2, 4, 1, dtype=torch.int32))[..., :0],
+                              dev(torch.from_numpy(sel[1])),
+                              dev(torch.zeros(1, 2, 4, 1))[..., :0])
+    torch.cuda.synchronize()
+    oo, olse = O.attn_fwd(x["q"], x["k"], x["v"], *sel)
+    assert maxerr(np64(o), oo) < 1e-4 and maxerr(np64(lse), olse) < 1e-4
+
+
+def test_attn_c3_shape_sampled():
+    """Full c3 workload (N = 16384, GQA 32/8, d = 128, top-k 31) in the
+    launch configuration the bench times; selection exact on every row, the
+    attention checked on sampled query blocks and key blocks."""
+    c = inputs.CONFIGS["c3"]
+    x = inputs.gen_config("c3")
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    ks = sas.sas_block_summary(dev(k))
+    ti, tc, tl = sas.sas_select(dev(q), ks, c["Hkv"], c["topk"], "prefill")
+    o, lse = sas.sas_attn_fwd(dev(q), dev(k), dev(v), ti, tc, tl)
+    gq, gk, gv, gl = sas.sas_attn_bwd(dev(q), dev(k), dev(v), o, dev(do), lse, ti, tc, tl)
+    torch.cuda.synchronize()
+    oi, oc, ol, scores = oracle_selection(q, k, c["Hkv"], c["topk"])
+    assert boundary_gap(scores, c["topk"]) >= 1.5e-3
+    assert np.array_equal(tc.cpu().numpy(), oc) and np.array_equal(ti.cpu().numpy(), oi)
+    assert maxerr(np64(tl), ol) < 1e-4
+    o, lse, gq, gk, gv, gl = (t.cpu() for t in (o, lse, gq, gk, gv, gl))
+    tol = TOL["bf16"]
+    ol32 = ol.astype(np.float32)
+    st = stored("bf16")
+    for (r, t) in [(0, 0), (3, 1), (7, 31), (2, 32), (5, 200), (1, 255)]:
+        res = O.query_block(q, k, v, do, oi, oc, ol32, 0, r, t, o_stored=st)
+        for j, h in enumerate(range(r * 4, r * 4 + 4)):
+            rows = slice(t * 64, (t + 1) * 64)
+            assert excess(np64(o[0, h, rows]), res["o"][j], tol, True) <= 0
+            assert excess(np64(lse[0, h, rows]), res["lse"][j], tol, False) <= 0
+            assert excess(np64(gq[0, h, rows]), res["dq"][j], tol, True) <= 0
+        assert excess(np64(gl[0, r, t, :oc[0, r, t]]), res["dlogg"], tol, False) <= 0
+    popular = int(np.bincount(oi[0, 6][oi[0, 6] >= 0].ravel()).argmax())
+    for (r, j) in [(0, 255), (4, 17), (6, popular)]:
+        gk_ref, gv_ref = O.key_block_grads(q, k, v, do, oi, oc, ol32, 0, r, j, o_stored=st)
+        assert excess(np64(gk[0, r, j * 64:(j + 1) * 64]), gk_ref, tol, True) <= 0
+        assert excess(np64(gv[0, r, j * 64:(j + 1) * 64]), gv_ref, tol, True) <= 0
+
+
+# ------------------------------------------------------------------ decode
+def _decode_check(x, Hkv, topk, gated, tol=2e-2):
+    q, kc, vc, lens = x["q"], x["kc"], x["vc"], x["lens"]
+    ks = sas.sas_block_summary(dev(kc))
+    idx_out = torch.empty((q.shape[0], Hkv, topk), dtype=torch.int32, device=DEV)
+    o = sas.sas_decode(dev(q), dev(kc), dev(vc), dev(lens), ks, topk, gated=gated,
+                       idx_out=idx_out if topk else None)
+    torch.cuda.synchronize()
+    oks = O.block_summary(kc)
+    assert maxerr(np64(ks), oks) < 1e-5
+    oo, oi, oc, _ = O.decode(q, kc, vc, lens.numpy(), oks, Hkv, topk, gated=gated)
+    if topk:
+        assert np.array_equal(idx_out.cpu().numpy(), oi)
+    err = excess(np64(o), oo, tol, q.dtype == torch.bfloat16)
+    assert err <= 0, err
+    _, _, _, scores = O.select_decode(q, oks, lens.numpy(), Hkv, topk)
+    return scores
+
+
+@pytest.mark.parametrize("gated", [1, 0])
+def test_decode_c2(gated):
+    c = inputs.CONFIGS["c2"]
+    scores = _decode_check(inputs.gen_config("c2"), c["Hkv"], c["topk"], gated)
+    assert boundary_gap(scores, c["topk"]) >= 1.5e-3
+
+
+@pytest.mark.parametrize("lens", [[1, 64, 65, 1024], [700, 128, 1000, 63]])
+def test_decode_ragged_small(lens):
+    x = inputs.gen_decode(4, 8, 2, 1024, 128, lens, "bf16", seed=60, planted=8)
+    scores = _decode_check(x, 2, 4, 1)
+    assert boundary_gap(scores, 4) >= 1.5e-3
+
+
+@pytest.mark.parametrize("G,d,dtype", [(1, 64, "f32"), (2, 128, "f32"), (8, 64, "bf16")])
+def test_decode_group_sizes(G, d, dtype):
+    x = inputs.gen_decode(2, 2 * G, 2, 2048, d, [2048, 1500], dtype, seed=61, planted=6)
+    _decode_check(x, 2, 5, 1, tol=TOL[dtype])
+
+
+def test_decode_exact_ties():
+    x = inputs.gen_decode(1, 32, 8, 4096, 128, [4000], "bf16", seed=62)
+    x["kc"] = torch.zeros_like(x["kc"])
+    _decode_check(x, 8, 15, 1)
+
+
+def test_decode_topk_zero():
+    x = inputs.gen_decode(2, 8, 2, 512, 64, [300, 512], "bf16", seed=63)
+    _decode_check(x, 2, 0, 1)
+
+
+@pytest.mark.parametrize("name", ["c4", "c5"])
+def test_decode_full_configs(name):
+    c = inputs.CONFIGS[name]
+    scores = _decode_check(inputs.gen_config(name), c["Hkv"], c["topk"], c["gated"])
+    assert boundary_gap(scores, c["topk"]) >= 1.5e-3
+
+
+def test_decode_repeat_is_bitwise_stable():
+    x = inputs.gen_decode(1, 32, 8, 8192, 128, [8100], "bf16", seed=64, planted=16)
+    ks = sas.sas_block_summary(dev(x["kc"]))
+    args = (dev(x["q"]), dev(x["kc"]), dev(x["vc"]), dev(x["lens"]), ks, 15)
+    a = sas.sas_decode(*args).clone()
+    b = sas.sas_decode(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_decode_attend_forced_selection():
+    """Decode attention with an arbitrary selection and arbitrary gates."""
+    B, Hq, Hkv, L, d, topk = 2, 8, 2, 2048, 128, 6
+    x = inputs.gen_decode(B, Hq, Hkv, L, d, [2048, 1111], "bf16", seed=66)
+    rng = np.random.Generator(np.random.PCG64(67))
+    idx = np.full((B, Hkv, topk), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    logg = np.zeros((B, Hkv, topk), np.float32)
+    for b, n in enumerate([2048, 1111]):
+        C = (n - 1) // 64
+        for r in range(Hkv):
+            kk = int(rng.integers(0, topk + 1))
+            idx[b, r, :kk] = np.sort(rng.choice(C, kk, replace=False))
+            cnt[b, r] = kk
+            logg[b, r, :kk] = rng.uniform(-6, 0, kk)
+    for gated in (1, 0):
+        o = sas.sas_decode_attend(dev(x["q"]), dev(x["kc"]), dev(x["vc"]), dev(x["lens"]),
+                                  dev(torch.from_numpy(idx)), dev(torch.from_numpy(cnt)),
+                                  dev(torch.from_numpy(logg)), gated=gated)
+        torch.cuda.synchronize()
+        ref, _ = O.decode_attend(x["q"], x["kc"], x["vc"], x["lens"].numpy(), idx, cnt, logg,
+                                 Hkv, gated=gated)
+        assert excess(np64(o), ref, 2e-2, True) <= 0

@@ -404,3 +404,22 @@ def test_decode_selection_enumeration():
     s = np.array([qbar @ kc[0, 0, m * 64:(m + 1) * 64].mean(axis=0) / np.sqrt(d) for m in range(7)])
     assert idx[0, 0].tolist() == brute.topk_enumerate(s, 3).tolist()
     assert np.allclose(logg[0, 0], s[idx[0, 0]] - np.log(np.exp(s).sum()), atol=1e-13)
+
+
+def test_stored_output_form_of_D():
+    """attn_bwd with the exact output passed as the stored one is unchanged;
+    a rounded stored output moves only the row term D (dv does not use D)."""
+    q, k, v, do, idx, cnt, logg = _sparse_case(120, N=256, d=16, topk=2)
+    o, _ = O.attn_fwd(q, k, v, idx, cnt, logg)
+    ref = O.attn_bwd(q, k, v, do, idx, cnt, logg)
+    same = O.attn_bwd(q, k, v, do, idx, cnt, logg, o_stored=o)
+    for a, b in zip(ref, same):
+        assert np.abs(a - b).max() < 1e-13
+    rounded = inputs.to_storage(o, "bf16").double().numpy()
+    moved = O.attn_bwd(q, k, v, do, idx, cnt, logg, o_stored=rounded)
+    assert np.abs(moved[2] - ref[2]).max() < 1e-13          # dv
+    assert 0 < np.abs(moved[3] - ref[3]).max() < 0.05        # dlogg shifts a little
+    as_fn = O.attn_bwd(q, k, v, do, idx, cnt, logg,
+                       o_stored=lambda rows: inputs.to_storage(rows, "bf16").double().numpy())
+    for a, b in zip(moved, as_fn):
+        assert np.abs(a - b).max() < 1e-13

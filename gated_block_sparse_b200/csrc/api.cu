@@ -159,6 +159,38 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
                      "sas_select launch");
 }
 
+size_t sas_select_prefill_noalloc_capacity(void) {
+  return sas::select_prefill_static_capacity() * sizeof(float);
+}
+
+sas_status sas_select_prefill_noalloc(const void* q, sas_dtype dt, const float* ksum, int B,
+                                      int Hq, int Hkv, int N, int d, int topk, float scale,
+                                      int32_t* idx, int32_t* cnt, float* logg,
+                                      sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(cnt);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  if (N / 64 > 0) REQUIRE_PTR(ksum);
+  REQUIRE((N + 63) / 64 - 1 <= 256 * 64, SAS_ERR_UNSUPPORTED, "prefill N too long for selection");
+  const size_t need = sas::select_prefill_ws_bytes(B, Hkv, N, d);
+  const size_t cap = sas_select_prefill_noalloc_capacity();
+  REQUIRE(need <= cap, SAS_ERR_UNSUPPORTED,
+          "sas_select_prefill_noalloc: B*Hkv*ceil(N/64)*d*4 = %zu bytes of query summaries exceed "
+          "the fixed %zu-byte device array; use sas_select with a workspace",
+          need, cap);
+  return cuda_status(sas::launch_select_prefill_static(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d,
+                                                       topk, resolve_scale(scale, d), idx, cnt,
+                                                       logg, (cudaStream_t)stream),
+                     "sas_select_prefill_noalloc launch");
+}
+
 size_t sas_attn_fwd_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_dtype dt) {
   (void)B; (void)Hq; (void)Hkv; (void)N; (void)d; (void)topk; (void)dt;
   return 0;

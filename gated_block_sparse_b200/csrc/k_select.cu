@@ -312,6 +312,51 @@ cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, in
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ prefill, no allocation
+// For callers that cannot allocate device memory at call time, the prefill
+// selection can keep its query summaries in a fixed array that is part of
+// the library image instead of a caller-provided workspace. The array is
+// statically sized (kStaticQbarFloats fp32 values, 4 MiB); every GPU that
+// loads the library holds it until the process exits. All calls share it:
+// each call overwrites the part it uses before reading it (nothing needs
+// to start at zero), and calls that overlap on the GPU race on it.
+constexpr size_t kStaticQbarFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_qbar_static[kStaticQbarFloats];
+
+size_t select_prefill_static_capacity() { return kStaticQbarFloats; }
+
+// Device address of the array for the current device: looked up with
+// cudaGetSymbolAddress on the first call per device (the host-side name is
+// only a stand-in and must never be passed to a kernel), then cached.
+static cudaError_t static_qbar_address(float** out) {
+  static std::mutex mu;
+  static std::map<int, float*> addr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_qbar_static);
+    if (e != cudaSuccess) return e;
+    it = addr.emplace(dev, static_cast<float*>(p)).first;
+  }
+  *out = it->second;
+  return cudaSuccess;
+}
+
+cudaError_t launch_select_prefill_static(const void* q, int bf16, const float* ksum, int B,
+                                         int Hq, int Hkv, int N, int d, int topk, float scale,
+                                         int32_t* idx, int32_t* cnt, float* logg,
+                                         cudaStream_t st) {
+  float* qbar = nullptr;
+  cudaError_t e = static_qbar_address(&qbar);
+  if (e != cudaSuccess) return e;
+  return launch_select_prefill(q, bf16, ksum, B, Hq, Hkv, N, d, topk, scale, idx, cnt, logg, qbar,
+                               st);
+}
+
 // ------------------------------------------------------------------ decode
 // Scratch layout per plan (rows = B*Hkv, nchunk chunks per row):
 //   counters [rows] int | len [rows][nchunk] int | cmax, csum [rows][nchunk]

@@ -26,6 +26,13 @@ cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, in
                                   int Hkv, int N, int d, int topk, float scale, int32_t* idx,
                                   int32_t* cnt, float* logg, void* ws, cudaStream_t st);
 size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d);
+// Prefill selection with its query-summary scratch in a fixed device array
+// of the library (no workspace argument); capacity in fp32 values.
+size_t select_prefill_static_capacity();
+cudaError_t launch_select_prefill_static(const void* q, int bf16, const float* ksum, int B,
+                                         int Hq, int Hkv, int N, int d, int topk, float scale,
+                                         int32_t* idx, int32_t* cnt, float* logg,
+                                         cudaStream_t st);
 
 // Decode selection. `counters` holds one int per row and must be zero on
 // entry (the kernel leaves it zero); `ws` holds the plan's partials.

@@ -29,6 +29,8 @@ SIGNATURES = {
     "sas_block_summary": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sas_select_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "sas_select": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F, _P, _P, _P, _P, _Z, _P]),
+    "sas_select_prefill_noalloc_capacity": (_Z, []),
+    "sas_select_prefill_noalloc": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "sas_attn_fwd_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "sas_attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I, _F, _P, _P, _P, _Z,
                           _P]),
@@ -146,6 +148,25 @@ def sas_select(q: torch.Tensor, ksum: torch.Tensor, Hkv: int, topk: int, mode: s
         _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, m, _ptr(lens), float(scale),
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, _ptr(w),
         w.numel(), _stream(stream)))
+    return idx, cnt, logg
+
+
+def sas_select_prefill_noalloc(q: torch.Tensor, ksum: torch.Tensor, Hkv: int, topk: int,
+                               scale: float = 0.0, out=None, stream=None):
+    """Prefill selection whose scratch is the library's fixed device array:
+    the call itself allocates no device memory (pass `out` to supply the
+    output buffers too). Returns (idx, cnt, logg) like sas_select."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    T = -(-N // 64)
+    if out is None:
+        out = (torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=q.device),
+               torch.empty((B, Hkv, T), dtype=torch.int32, device=q.device),
+               torch.empty((B, Hkv, T, topk), dtype=torch.float32, device=q.device))
+    idx, cnt, logg = out
+    _check("sas_select_prefill_noalloc", lib.sas_select_prefill_noalloc(
+        _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, float(scale),
+        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, _stream(stream)))
     return idx, cnt, logg
 
 

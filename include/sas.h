@@ -113,6 +113,31 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
                       sas_stream_t stream);
 
 /*
+ * Prefill selection that allocates nothing and takes no workspace. The paper
+ * has no counterpart: this is an interface variant of sas_select(SAS_PREFILL)
+ * for callers that cannot allocate device memory when they call, such as a
+ * host runtime that hands a kernel library only its input and output
+ * buffers and forbids device allocation after start-up (cudaMalloc can
+ * synchronise the device and has no latency bound).
+ *   Same arguments, layouts and results as sas_select in SAS_PREFILL mode.
+ *   Its scratch (the fp32 query summary of every (b, kv group, query block),
+ *   B*Hkv*ceil(N/64)*d*4 bytes) lives in a fixed device array inside the
+ *   library of sas_select_prefill_noalloc_capacity() bytes (4 MiB), which
+ *   every GPU that loads the library keeps until the process exits. Larger
+ *   problems are rejected with SAS_ERR_UNSUPPORTED and a message.
+ *   The first call on each device looks up the array's device address once
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls share the array; each call overwrites what it reads, and calls
+ *   that overlap on the GPU (other streams, other threads) race on it.
+ *   Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+size_t sas_select_prefill_noalloc_capacity(void);
+sas_status sas_select_prefill_noalloc(const void* q, sas_dtype dt, const float* ksum, int B,
+                                      int Hq, int Hkv, int N, int d, int topk, float scale,
+                                      int32_t* idx, int32_t* cnt, float* logg,
+                                      sas_stream_t stream);
+
+/*
  * Gated sparse attention forward for prefill/training (SAS close reading,
  * sections 2.2 and 2.4; reproduction note, core formula):
  *   o_i = sum_j softmax_j(z_ij) v_j,  lse_i = log sum_j exp(z_ij),

@@ -27,7 +27,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 14
+    assert len(names) == 16
     for n in names:
         assert hasattr(lib, n), n
         assert n in sas.SIGNATURES, n
@@ -101,3 +101,11 @@ def test_empty_inputs_are_noops(lib):
     assert lib.sas_attn_fwd(None, None, None, 1, 0, 4, 4, 128, 64, None, None, None, 2, 0.0, None,
                             None, None, 0, None) == 0
     assert lib.sas_block_summary(None, 1, 1, 2, 63, 64, None, None, None) == 0
+
+
+def test_noalloc_selection_capacity_and_rejection(lib):
+    assert lib.sas_select_prefill_noalloc_capacity() == 4 << 20
+    # 8 groups x 2048 query blocks x 128 x 4 B = 8 MiB of query summaries: rejected before launch
+    st = lib.sas_select_prefill_noalloc(FAKE, 1, FAKE, 1, 8, 8, 131072, 128, 4, 0.0, FAKE, FAKE,
+                                        FAKE, None)
+    assert st == 2 and b"exceed" in lib.sas_last_error_message()

@@ -57,26 +57,6 @@ float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sq
 
 size_t a16(size_t x) { return (x + 15) & ~(size_t)15; }
 
-// Decode workspace: counters [2 * rows] | select partials | attend partials |
-// idx [rows][topk] | cnt [rows] | logg [rows][topk].
-struct DecodeLayout {
-  size_t counters, sel, att, idx, cnt, logg, total;
-};
-DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int d, int topk) {
-  DecodeLayout L;
-  const int rows = B * Hkv;
-  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, Lmax, topk);
-  size_t off = 0;
-  L.counters = off; off += a16(sizeof(int) * 2 * (size_t)rows);
-  L.sel = off; off += a16(sas::decode_select_ws_bytes(p));
-  L.att = off; off += a16(sas::decode_attend_ws_bytes(B, Hq, Hkv, topk, d));
-  L.idx = off; off += a16(sizeof(int32_t) * (size_t)rows * topk);
-  L.cnt = off; off += a16(sizeof(int32_t) * (size_t)rows);
-  L.logg = off; off += a16(sizeof(float) * (size_t)rows * topk);
-  L.total = off;
-  return L;
-}
-
 }  // namespace
 
 extern "C" {
@@ -312,8 +292,8 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
 }
 
 size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk) {
-  if (B <= 0 || Hkv <= 0 || Lmax <= 0 || d <= 0 || topk < 0) return 0;
-  return decode_layout(B, Hq, Hkv, Lmax, d, topk).total;
+  (void)B; (void)Hq; (void)Hkv; (void)Lmax; (void)d; (void)topk;
+  return 0;  // the one-launch cluster kernel keeps everything in shared memory
 }
 
 sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype dt, int B, int Hq,
@@ -321,6 +301,7 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                       int gated, float scale, void* o, int32_t* idx_out, void* ws,
                       size_t ws_bytes, sas_stream_t stream) {
   g_last_error.clear();
+  (void)ws; (void)ws_bytes;
   sas_status s = check_decode(dt, B, Hq, Hkv, Lmax, d, topk, gated);
   if (s != SAS_OK) return s;
   if (B == 0) return SAS_OK;
@@ -331,26 +312,10 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
   REQUIRE_PTR(ksum);
   REQUIRE_PTR(o);
   if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
-  const DecodeLayout L = decode_layout(B, Hq, Hkv, Lmax, d, topk);
-  REQUIRE(ws_bytes >= L.total, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, L.total);
-  REQUIRE_PTR(ws);
-  char* w = static_cast<char*>(ws);
-  cudaStream_t st = (cudaStream_t)stream;
-  const int rows = B * Hkv;
-  int* counters = reinterpret_cast<int*>(w + L.counters);
-  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.idx);
-  int32_t* cnt = reinterpret_cast<int32_t*>(w + L.cnt);
-  float* logg = reinterpret_cast<float*>(w + L.logg);
-  const float sc = resolve_scale(scale, d);
-  cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * 2 * (size_t)rows, st);
-  if (e != cudaSuccess) return cuda_status(e, "sas_decode memset");
-  const sas::SelectPlan p = sas::plan_decode_select(B, Hkv, Lmax, topk);
-  e = sas::launch_select_decode(q, dt == SAS_BF16, ksum, B, Hq, Hkv, Lmax, d, topk, lens, sc, idx,
-                                cnt, logg, p, counters, w + L.sel, st);
-  if (e != cudaSuccess) return cuda_status(e, "sas_decode select launch");
-  e = sas::launch_decode_attend(q, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, idx, cnt,
-                                logg, topk, gated, sc, o, counters + rows, w + L.att, st, true);
-  return cuda_status(e, "sas_decode attend launch");
+  return cuda_status(sas::launch_decode_fused(q, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens,
+                                              ksum, topk, gated, resolve_scale(scale, d), o,
+                                              idx_out, (cudaStream_t)stream),
+                     "sas_decode launch");
 }
 
 }  // extern "C"

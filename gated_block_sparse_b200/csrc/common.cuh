@@ -85,6 +85,69 @@ __device__ __forceinline__ bool beats(float sa, int ia, float sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
 }
 
+// ---------------------------------------------------------------- Top-K lists
+// Order key of a candidate block: larger score first, then lower block index,
+// packed into one unsigned 64-bit integer (larger key = better candidate).
+// A -0 score must be stored as +0 beforehand so that exact ties are equal.
+__device__ __forceinline__ unsigned long long cand_key(float s, int m) {
+  uint32_t u = __float_as_uint(s);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving map
+  return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)m);
+}
+
+// Pairwise tree merge of nl best-first candidate lists held in shared memory
+// (list l: len[l] entries at s/m + l*stride, stride >= k) into one best-first
+// list of the min(k, total) best candidates, left in list 0 of whichever
+// buffer the function returns (0 = A, 1 = B). Each level merges lists 2i and
+// 2i+1: an entry at position p of one list has rank p plus the number of
+// entries of the other list with a larger key (one binary search); ranks
+// below k are kept. Keys are unique, so ranks never collide. All threads of
+// the block must call it.
+__device__ inline int tree_merge(float* As, int* Am, int* Alen, float* Bs, int* Bm, int* Blen,
+                                 int nl, int stride, int k) {
+  int which = 0;
+  while (nl > 1) {
+    float* ss = which ? Bs : As;
+    int* sm_ = which ? Bm : Am;
+    int* sl = which ? Blen : Alen;
+    float* ds = which ? As : Bs;
+    int* dm = which ? Am : Bm;
+    int* dl = which ? Alen : Blen;
+    const int npairs = (nl + 1) >> 1;
+    for (int e = threadIdx.x; e < nl * stride; e += blockDim.x) {
+      const int l = e / stride, p = e - l * stride;
+      if (p >= sl[l]) continue;
+      const float sv = ss[e];
+      const int mv = sm_[e];
+      const int partner = l ^ 1;
+      int rank = p;
+      if (partner < nl) {
+        const unsigned long long key = cand_key(sv, mv);
+        const float* ps = ss + partner * stride;
+        const int* pm = sm_ + partner * stride;
+        int lo = 0, hi = sl[partner];
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (cand_key(ps[mid], pm[mid]) > key) lo = mid + 1; else hi = mid;
+        }
+        rank += lo;
+      }
+      if (rank < k) {
+        ds[(l >> 1) * stride + rank] = sv;
+        dm[(l >> 1) * stride + rank] = mv;
+      }
+    }
+    for (int o = threadIdx.x; o < npairs; o += blockDim.x) {
+      const int a = sl[2 * o], b2 = (2 * o + 1 < nl) ? sl[2 * o + 1] : 0;
+      dl[o] = min(k, a + b2);
+    }
+    __syncthreads();
+    which ^= 1;
+    nl = npairs;
+  }
+  return which;
+}
+
 // ---------------------------------------------------------------- PDL
 // Programmatic dependent launch: a kernel launched with the programmatic
 // stream serialization attribute may start before its predecessor ends.

@@ -7,13 +7,11 @@
 // key is (score descending, block index ascending), packed into one 64-bit
 // integer. Each chunk of up to 256 history blocks is scored into shared
 // memory and reduced to its own best-first list of min(k, n) candidates by
-// rank counting. The merge takes theta = the best k-th entry among the full
-// lists; every global Top-K member is at or above theta (the list that gives
-// theta alone holds k keys >= theta), so only entries >= theta are ranked,
-// each by binary searches in the sorted lists. The kept blocks are then
-// written in ascending block order. (The MSA notes, papercache, Top-K kernel
-// section, use per-lane heaps and a shuffle merge on H800; chunk lists plus a
-// threshold merge suit wide CTAs and need no heap.)
+// rank counting. The lists are then merged pairwise in a tree (each entry
+// ranked in its partner list by one binary search, the best k kept per
+// level), and the kept blocks are written in ascending block order. (The MSA
+// notes, papercache, Top-K kernel section, use per-lane heaps and a shuffle
+// merge on H800; chunk lists plus a parallel tree merge suit wide CTAs.)
 //
 // Prefill: one CTA per (b, kv group, query block). Decode: one CTA per
 // (b, kv group, chunk); the last CTA to finish a row (atomic counter, no
@@ -29,12 +27,6 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_CHUNK_MAX = 256;      // prefill chunk
 constexpr int DEC_CHUNK_MAX = 512;      // decode chunk upper bound
 constexpr int DEC_NCHUNK_MAX = 128;     // decode chunks per row upper bound
-
-__device__ __forceinline__ unsigned long long cand_key(float s, int m) {
-  uint32_t u = __float_as_uint(s);
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // order-preserving map
-  return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)m);
-}
 
 __device__ __forceinline__ float block_reduce_max(float v, float* red) {
   v = warp_max(v);
@@ -117,67 +109,18 @@ __device__ void chunk_topk(const float* sc, int m0, int n, int k, float* ls, int
   }
 }
 
-// Merge nchunk best-first lists (list c: len[c] entries at ls/li + c*k) into
-// the kk best entries, written to out_idx/out_logg in ascending block order
-// (log g = s - lse), padded to k with -1 / 0. sel_s/sel_m: kk-entry scratch
-// in shared memory. Loads go through L2 (.cg) because the lists may have
-// been written by other CTAs of the grid.
-template <typename X>
-__device__ __forceinline__ X ld_list(const X* p, bool global) {
-  return global ? __ldcg(p) : *p;
-}
-
-template <bool kGlobal>
-__device__ void merge_lists(const float* ls, const int* li, const int* len, int nchunk, int k,
-                            int kk, float lse, float* sel_s, int* sel_m,
-                            unsigned long long* theta_s, int32_t* out_idx, float* out_logg) {
-  const int tid = threadIdx.x;
-  if (tid == 0) *theta_s = 0ull;
-  __syncthreads();
-  for (int c = tid; c < nchunk; c += blockDim.x) {
-    const int L = ld_list(len + c, kGlobal);
-    if (L == k && k > 0) {
-      const unsigned long long key = cand_key(ld_list(ls + (size_t)c * k + k - 1, kGlobal),
-                                              ld_list(li + (size_t)c * k + k - 1, kGlobal));
-      atomicMax(theta_s, key);
-    }
-  }
-  __syncthreads();
-  const unsigned long long theta = *theta_s;
-  const int total = nchunk * k;
-  for (int e = tid; e < total; e += blockDim.x) {
-    const int c = e / k, p = e - c * k;
-    if (p >= ld_list(len + c, kGlobal)) continue;
-    const float s = ld_list(ls + e, kGlobal);
-    const int m = ld_list(li + e, kGlobal);
-    const unsigned long long key = cand_key(s, m);
-    if (key < theta) continue;
-    int rank = 0;
-    for (int c2 = 0; c2 < nchunk && rank < kk; ++c2) {
-      int lo = 0, hi = ld_list(len + c2, kGlobal);  // count entries of list c2 with a larger key
-      const float* s2 = ls + (size_t)c2 * k;
-      const int* m2 = li + (size_t)c2 * k;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        const unsigned long long km = cand_key(ld_list(s2 + mid, kGlobal), ld_list(m2 + mid, kGlobal));
-        if (km > key) lo = mid + 1; else hi = mid;
-      }
-      rank += lo;
-    }
-    if (rank < kk) {
-      sel_s[rank] = s;
-      sel_m[rank] = m;
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < kk; i += blockDim.x) {
-    const int mi = sel_m[i];
+// Writes the kk best entries of a best-first list (s/m) to out_idx/out_logg
+// in ascending block order (log g = s - lse), padded to k with -1 / 0.
+__device__ void write_selection(const float* s, const int* m, int kk, int k, float lse,
+                                int32_t* out_idx, float* out_logg) {
+  for (int i = threadIdx.x; i < kk; i += blockDim.x) {
+    const int mi = m[i];
     int pos = 0;
-    for (int j = 0; j < kk; ++j) pos += sel_m[j] < mi;
+    for (int j = 0; j < kk; ++j) pos += m[j] < mi;
     out_idx[pos] = mi;
-    out_logg[pos] = sel_s[i] - lse;
+    out_logg[pos] = s[i] - lse;
   }
-  for (int i = kk + tid; i < k; i += blockDim.x) {
+  for (int i = kk + threadIdx.x; i < k; i += blockDim.x) {
     out_idx[i] = -1;
     out_logg[i] = 0.f;
   }
@@ -228,15 +171,16 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
   const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z, T_ = gridDim.x;
   const int C = t;
   const int nchunk = (C + SEL_CHUNK_MAX - 1) / SEL_CHUNK_MAX;
+  const int nck = (nchunk + 3) & ~3;
   float* q_s = reinterpret_cast<float*>(smem_raw);
   float* sc = q_s + D;
   float* red = sc + SEL_CHUNK_MAX;
-  float* sel_s = red + 32;
-  int* sel_m = reinterpret_cast<int*>(sel_s + 128);
-  unsigned long long* theta_s = reinterpret_cast<unsigned long long*>(sel_m + 128);
-  int* len = reinterpret_cast<int*>(theta_s + 1);
-  float* ls = reinterpret_cast<float*>(len + ((nchunk + 3) & ~3));
+  int* len = reinterpret_cast<int*>(red + 32);
+  int* len_b = len + nck;
+  float* ls = reinterpret_cast<float*>(len_b + nck);
   int* li = reinterpret_cast<int*>(ls + (size_t)nchunk * topk);
+  float* ls_b = reinterpret_cast<float*>(li + (size_t)nchunk * topk);
+  int* li_b = reinterpret_cast<int*>(ls_b + (size_t)nchunk * topk);
 
   const size_t row = ((size_t)b * Hkv + r) * T_ + t;
   const float* qrow = qbar + row * D;
@@ -263,9 +207,11 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
   }
   const int kk = min(topk, C);
   const float lse = (C > 0) ? run_m + __logf(run_s) : 0.f;
-  if (topk > 0)
-    merge_lists<false>(ls, li, len, nchunk, topk, kk, lse, sel_s, sel_m, theta_s, idx + row * topk,
-                logg + row * topk);
+  if (topk > 0) {
+    const int wb = tree_merge(ls, li, len, ls_b, li_b, len_b, nchunk, topk, topk);
+    write_selection(wb ? ls_b : ls, wb ? li_b : li, kk, topk, lse, idx + row * topk,
+                    logg + row * topk);
+  }
   if (threadIdx.x == 0) cnt[row] = kk;
 }
 
@@ -275,10 +221,9 @@ size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d) {
 }
 
 static size_t prefill_select_smem(int d, int nchunk, int topk) {
-  size_t n = (size_t)d + SEL_CHUNK_MAX + 32 + 128 + 128;  // q, sc, red, sel_s, sel_m
-  n += 2;                                                 // theta (8 bytes)
-  n += (nchunk + 3) & ~3;                                 // len
-  n += 2 * (size_t)nchunk * topk;                         // ls, li
+  size_t n = (size_t)d + SEL_CHUNK_MAX + 32;  // q, sc, red
+  n += 2 * (size_t)((nchunk + 3) & ~3);       // len, len_b
+  n += 4 * (size_t)nchunk * topk;             // ls, li, ls_b, li_b
   return n * 4;
 }
 
@@ -409,7 +354,8 @@ SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk) {
 }
 
 static size_t decode_merge_smem(int nchunk, int topk) {
-  return sizeof(float) * (2 * (size_t)nchunk + ((nchunk + 3) & ~3) + 2 * (size_t)nchunk * topk);
+  const size_t nck = (nchunk + 3) & ~3;
+  return sizeof(float) * (4 * nck + 4 * (size_t)nchunk * topk);
 }
 
 template <typename T, int D>
@@ -420,9 +366,6 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   __shared__ __align__(16) float q_s[D];
   __shared__ float sc[DEC_CHUNK_MAX];
   __shared__ float red[32];
-  __shared__ float sel_s[128];
-  __shared__ int sel_m[128];
-  __shared__ unsigned long long theta_s;
   __shared__ int is_last;
   // merge staging (last CTA of a row): the row's chunk partials and lists
   extern __shared__ __align__(16) unsigned char dsm[];
@@ -468,11 +411,15 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   __threadfence();
   // Stage the row's partials in shared memory with one parallel pass of L2
   // loads, then merge there (a serial walk over L2 would be latency-bound).
+  const int nck = (nchunk + 3) & ~3;
   float* cm_s = reinterpret_cast<float*>(dsm);
-  float* cs_s = cm_s + nchunk;
-  int* len_s = reinterpret_cast<int*>(cs_s + nchunk);
-  float* ls_s = reinterpret_cast<float*>(len_s + ((nchunk + 3) & ~3));
+  float* cs_s = cm_s + nck;
+  int* len_s = reinterpret_cast<int*>(cs_s + nck);
+  int* len_b = len_s + nck;
+  float* ls_s = reinterpret_cast<float*>(len_b + nck);
   int* li_s = reinterpret_cast<int*>(ls_s + (size_t)nchunk * topk);
+  float* ls_b = reinterpret_cast<float*>(li_s + (size_t)nchunk * topk);
+  int* li_b = reinterpret_cast<int*>(ls_b + (size_t)nchunk * topk);
   const size_t r0 = (size_t)row * nchunk;
   for (int i = threadIdx.x; i < nchunk; i += blockDim.x) {
     cm_s[i] = __ldcg(w.cmax + r0 + i);  // empty chunks: -FLT_MAX and 0
@@ -496,9 +443,12 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   const float S = block_reduce_sum(lsum, red);
   const float lse = (C > 0) ? M + __logf(S) : 0.f;
   const int kk = min(topk, C);
-  if (topk > 0)
-    merge_lists<false>(ls_s, li_s, len_s, nchunk, topk, kk, lse, sel_s, sel_m, &theta_s,
-                       idx + (size_t)row * topk, logg + (size_t)row * topk);
+  if (topk > 0) {
+    __syncthreads();
+    const int wb = tree_merge(ls_s, li_s, len_s, ls_b, li_b, len_b, nchunk, topk, topk);
+    write_selection(wb ? ls_b : ls_s, wb ? li_b : li_s, kk, topk, lse, idx + (size_t)row * topk,
+                    logg + (size_t)row * topk);
+  }
   if (threadIdx.x == 0) {
     cnt[row] = kk;
     w.counter[row] = 0;  // ready for the next call

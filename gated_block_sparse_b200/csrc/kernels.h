@@ -50,6 +50,14 @@ cudaError_t launch_decode_attend(const void* q, const void* kc, const void* vc, 
                                  int topk, int gated, float scale, void* o, int* counters,
                                  void* ws, cudaStream_t st, bool pdl);
 uint32_t* decode_error_word();
+
+// One-launch decode step: selection + attention + combine, one thread-block
+// cluster per (sequence, kv group); needs no workspace.
+cudaError_t launch_decode_fused(const void* q, const void* kc, const void* vc, int bf16, int B,
+                                int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                                const float* ksum, int topk, int gated, float scale, void* o,
+                                int32_t* idx_out, cudaStream_t st);
+uint32_t* decode_fused_error_word();
 uint32_t* attn_simt_error_word();
 
 // ---- prefill attention (SIMT path: fp32 or bf16 inputs, any GPU of sm_100a)

@@ -187,7 +187,9 @@ sas_status sas_attn_bwd(const void* q, const void* k, const void* v, const void*
  *   q [B][Hq][d], kc, vc [B][Hkv][Lmax][d] (dt), lens [B] int32 device
  *   ksum [B][Hkv][Lmax/64][d] fp32 summaries of the cache
  *   o [B][Hq][d] (dt) output; idx_out [B][Hkv][topk] int32 or NULL
- * Workspace: sas_decode_workspace_size().
+ * One launch: a thread-block cluster per (b, kv group) selects, attends and
+ * combines through distributed shared memory. Workspace:
+ * sas_decode_workspace_size() returns 0; ws may be NULL.
  */
 size_t sas_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int d, int topk);
 sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype dt, int B, int Hq,

@@ -41,14 +41,15 @@ def test_strerror_and_version(lib):
 
 
 def test_workspace_sizes_are_consistent(lib):
-    # decode workspace grows with batch and top-k and is 16-byte granular
-    a = lib.sas_decode_workspace_size(1, 32, 8, 65536, 128, 15)
-    b = lib.sas_decode_workspace_size(8, 32, 8, 131072, 128, 31)
+    # the one-launch decode needs no workspace; the split decode attention does
+    assert lib.sas_decode_workspace_size(8, 32, 8, 131072, 128, 31) == 0
+    a = lib.sas_decode_attend_workspace_size(1, 32, 8, 65536, 128, 15)
+    b = lib.sas_decode_attend_workspace_size(8, 32, 8, 131072, 128, 31)
     assert a > 0 and b > a and a % 16 == 0 and b % 16 == 0
     # prefill selection needs one fp32 query summary per (b, group, block)
     assert lib.sas_select_workspace_size(1, 32, 8, 16384, 128, 31, 0) == 8 * 256 * 128 * 4
     assert lib.sas_attn_bwd_workspace_size(1, 32, 8, 16384, 128, 31, 1) == 2 * 8 * 16384 * 128 * 4
-    assert lib.sas_decode_workspace_size(0, 32, 8, 65536, 128, 15) == 0
+    assert lib.sas_decode_attend_workspace_size(0, 32, 8, 65536, 128, 15) == 0
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
@@ -84,7 +85,7 @@ def test_rejects_topk_and_workspace(lib):
 
 
 def test_rejects_bad_decode_shapes(lib):
-    ws = lib.sas_decode_workspace_size(1, 32, 8, 65536, 128, 15)
+    ws = 1 << 20
     st = lib.sas_decode(FAKE, FAKE, FAKE, 1, 1, 24, 8, 65536, 128, FAKE, FAKE, 15, 1, 0.0, FAKE,
                         None, FAKE, ws, None)
     assert st == 2  # 3 query heads per kv head is not a supported group size

@@ -95,47 +95,48 @@ __device__ __forceinline__ unsigned long long cand_key(float s, int m) {
   return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)m);
 }
 
-// Pairwise tree merge of nl best-first candidate lists held in shared memory
-// (list l: len[l] entries at s/m + l*stride, stride >= k) into one best-first
-// list of the min(k, total) best candidates, left in list 0 of whichever
-// buffer the function returns (0 = A, 1 = B). Each level merges lists 2i and
-// 2i+1: an entry at position p of one list has rank p plus the number of
-// entries of the other list with a larger key (one binary search); ranks
-// below k are kept. Keys are unique, so ranks never collide. All threads of
-// the block must call it.
-__device__ inline int tree_merge(float* As, int* Am, int* Alen, float* Bs, int* Bm, int* Blen,
-                                 int nl, int stride, int k) {
+__device__ __forceinline__ float key_score(unsigned long long key) {
+  const uint32_t u = (uint32_t)(key >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ int key_block(unsigned long long key) {
+  return (int)(0xffffffffu - (uint32_t)key);
+}
+
+// Pairwise tree merge of nl best-first candidate lists of keys in shared
+// memory (list l: len[l] keys at A + (l << lg), i.e. a power-of-two stride
+// 2^lg >= k) into one best-first list of the min(k, total) best keys, left
+// in list 0 of the buffer it returns (0 = A, 1 = B). Each level merges lists
+// 2i and 2i+1: a key at position p of one list has rank p plus the number of
+// keys of the other list that are larger (one binary search); ranks below k
+// are kept. Keys are unique, so ranks never collide. All threads of the
+// block must call it.
+__device__ inline int tree_merge(unsigned long long* A, int* Alen, unsigned long long* B, int* Blen,
+                                 int nl, int lg, int k) {
   int which = 0;
+  const int stride = 1 << lg;
   while (nl > 1) {
-    float* ss = which ? Bs : As;
-    int* sm_ = which ? Bm : Am;
-    int* sl = which ? Blen : Alen;
-    float* ds = which ? As : Bs;
-    int* dm = which ? Am : Bm;
+    const unsigned long long* src = which ? B : A;
+    const int* sl = which ? Blen : Alen;
+    unsigned long long* dst = which ? A : B;
     int* dl = which ? Alen : Blen;
     const int npairs = (nl + 1) >> 1;
-    for (int e = threadIdx.x; e < nl * stride; e += blockDim.x) {
-      const int l = e / stride, p = e - l * stride;
+    for (int e = threadIdx.x; e < (nl << lg); e += blockDim.x) {
+      const int l = e >> lg, p = e & (stride - 1);
       if (p >= sl[l]) continue;
-      const float sv = ss[e];
-      const int mv = sm_[e];
+      const unsigned long long key = src[e];
       const int partner = l ^ 1;
       int rank = p;
       if (partner < nl) {
-        const unsigned long long key = cand_key(sv, mv);
-        const float* ps = ss + partner * stride;
-        const int* pm = sm_ + partner * stride;
+        const unsigned long long* ps = src + (partner << lg);
         int lo = 0, hi = sl[partner];
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (cand_key(ps[mid], pm[mid]) > key) lo = mid + 1; else hi = mid;
+          if (ps[mid] > key) lo = mid + 1; else hi = mid;
         }
         rank += lo;
       }
-      if (rank < k) {
-        ds[(l >> 1) * stride + rank] = sv;
-        dm[(l >> 1) * stride + rank] = mv;
-      }
+      if (rank < k) dst[((l >> 1) << lg) + rank] = key;
     }
     for (int o = threadIdx.x; o < npairs; o += blockDim.x) {
       const int a = sl[2 * o], b2 = (2 * o + 1 < nl) ? sl[2 * o + 1] : 0;
@@ -146,6 +147,13 @@ __device__ inline int tree_merge(float* As, int* Am, int* Alen, float* Bs, int* 
     nl = npairs;
   }
   return which;
+}
+
+// log2 of the smallest power of two >= max(k, 1).
+__host__ __device__ inline int ceil_log2(int k) {
+  int lg = 0;
+  while ((1 << lg) < k) ++lg;
+  return lg;
 }
 
 // ---------------------------------------------------------------- PDL

@@ -45,6 +45,14 @@ __device__ uint32_t g_decode_fused_err = 0;
 constexpr int FD_THREADS = 256;
 constexpr int FD_WARPS = FD_THREADS / 32;
 
+// Two adjacent elements as fp32.
+__device__ __forceinline__ void load2(const float* p, float2& v) {
+  v = *reinterpret_cast<const float2*>(p);
+}
+__device__ __forceinline__ void load2(const __nv_bfloat16* p, float2& v) {
+  v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
@@ -56,8 +64,8 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 }
 
 struct FdSmem {  // byte offsets into dynamic shared memory
-  size_t kv0, u1, q, qbar, sc, zs, wa_s, wa_m, wb_s, wb_m, wlen_a, wlen_b, sa_s, sa_m, sb_s, sb_m,
-      slen_a, slen_b, smx, sse, kidx, klogg, cm, cl, cacc, bars, total;
+  size_t kv0, u1, q, qbar, sc, zs, wa, wb, wlen_a, wlen_b, sa, sb, slen_a, slen_b, smx, sse, kidx,
+      klogg, cm, cl, cacc, bars, total;
 };
 
 __host__ __device__ inline size_t fd_al(size_t x) { return (x + 127) & ~(size_t)127; }
@@ -68,7 +76,7 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int subc, int 
   FdSmem L;
   const size_t kvslot = (size_t)2 * SAS_BLOCK * D * es;
   const size_t ring = (size_t)2 * subc * D * 4;
-  const size_t kq = (size_t)(k > 0 ? k : 1);
+  const size_t kq = (size_t)1 << ceil_log2(k > 0 ? k : 1);  // list stride (power of two)
   size_t o = 0;
   L.kv0 = o; o += fd_al(kvslot);
   L.u1 = o; o += fd_al(kvslot > ring ? kvslot : ring);
@@ -76,16 +84,12 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int subc, int 
   L.qbar = o; o += fd_al((size_t)D * 4);
   L.sc = o; o += fd_al((size_t)(per > 0 ? per : 1) * 4);
   L.zs = o; o += fd_al((size_t)G * SAS_BLOCK * 4);
-  L.wa_s = o; o += fd_al(FD_WARPS * kq * 4);
-  L.wa_m = o; o += fd_al(FD_WARPS * kq * 4);
-  L.wb_s = o; o += fd_al(FD_WARPS * kq * 4);
-  L.wb_m = o; o += fd_al(FD_WARPS * kq * 4);
+  L.wa = o; o += fd_al(FD_WARPS * kq * 8);
+  L.wb = o; o += fd_al(FD_WARPS * kq * 8);
   L.wlen_a = o; o += fd_al(FD_WARPS * 4);
   L.wlen_b = o; o += fd_al(FD_WARPS * 4);
-  L.sa_s = o; o += fd_al((size_t)CS * kq * 4);
-  L.sa_m = o; o += fd_al((size_t)CS * kq * 4);
-  L.sb_s = o; o += fd_al((size_t)CS * kq * 4);
-  L.sb_m = o; o += fd_al((size_t)CS * kq * 4);
+  L.sa = o; o += fd_al((size_t)CS * kq * 8);
+  L.sb = o; o += fd_al((size_t)CS * kq * 8);
   L.slen_a = o; o += fd_al((size_t)CS * 4);
   L.slen_b = o; o += fd_al((size_t)CS * 4);
   L.smx = o; o += fd_al((size_t)CS * 4);
@@ -118,7 +122,8 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int CS = (int)cluster.num_blocks();
   const int crank = (int)cluster.block_rank();
   const FdSmem L = fd_layout(D, G, (int)sizeof(T), subc, per_max, topk, CS);
-  const int kq = topk > 0 ? topk : 1;
+  const int lg = ceil_log2(topk > 0 ? topk : 1);
+  const int kq = 1 << lg;  // list stride
   T* kv0 = reinterpret_cast<T*>(sm + L.kv0);
   T* kv1 = reinterpret_cast<T*>(sm + L.u1);
   float* sumbuf = reinterpret_cast<float*>(sm + L.u1);
@@ -126,16 +131,12 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   float* qbar = reinterpret_cast<float*>(sm + L.qbar);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
   float* zs = reinterpret_cast<float*>(sm + L.zs);
-  float* wa_s = reinterpret_cast<float*>(sm + L.wa_s);
-  int* wa_m = reinterpret_cast<int*>(sm + L.wa_m);
-  float* wb_s = reinterpret_cast<float*>(sm + L.wb_s);
-  int* wb_m = reinterpret_cast<int*>(sm + L.wb_m);
+  unsigned long long* wa = reinterpret_cast<unsigned long long*>(sm + L.wa);
+  unsigned long long* wb = reinterpret_cast<unsigned long long*>(sm + L.wb);
   int* wlen_a = reinterpret_cast<int*>(sm + L.wlen_a);
   int* wlen_b = reinterpret_cast<int*>(sm + L.wlen_b);
-  float* sa_s = reinterpret_cast<float*>(sm + L.sa_s);
-  int* sa_m = reinterpret_cast<int*>(sm + L.sa_m);
-  float* sb_s = reinterpret_cast<float*>(sm + L.sb_s);
-  int* sb_m = reinterpret_cast<int*>(sm + L.sb_m);
+  unsigned long long* sa = reinterpret_cast<unsigned long long*>(sm + L.sa);
+  unsigned long long* sb = reinterpret_cast<unsigned long long*>(sm + L.sb);
   int* slen_a = reinterpret_cast<int*>(sm + L.slen_a);
   int* slen_b = reinterpret_cast<int*>(sm + L.slen_b);
   float* smx = reinterpret_cast<float*>(sm + L.smx);
@@ -270,7 +271,20 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
   }
   int wsel = 0;  // which warp-list buffer holds this CTA's merged list (list 0)
-  if (topk > 0) {
+  if (topk > 0 && nmine <= FD_THREADS) {
+    // small range: one rank-counting pass over the whole range, one item per
+    // thread (broadcast shared-memory reads), straight into list 0 of A
+    if (tid < nmine) {
+      const float sj = sc[tid];
+      int rk = 0;
+      for (int x = 0; x < nmine; ++x) {
+        const float sx = sc[x];
+        rk += (sx > sj) || (sx == sj && x < tid);
+      }
+      if (rk < topk) wa[rk] = cand_key(sj, m0 + tid);
+    }
+    if (tid == 0) wlen_a[0] = min(topk, nmine);
+  } else if (topk > 0) {
     // each warp ranks its contiguous share of the range
     const int pw = (nmine + FD_WARPS - 1) / FD_WARPS;
     const int a0 = min(nmine, wid * pw), a1 = min(nmine, a0 + pw);
@@ -281,27 +295,22 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         const float sx = sc[x];
         rk += (sx > sj) || (sx == sj && x < j);
       }
-      if (rk < topk) {
-        wa_s[wid * kq + rk] = sj;
-        wa_m[wid * kq + rk] = m0 + j;
-      }
+      if (rk < topk) wa[wid * kq + rk] = cand_key(sj, m0 + j);
     }
     if (lane == 0) wlen_a[wid] = min(topk, a1 - a0);
     __syncthreads();
-    wsel = tree_merge(wa_s, wa_m, wlen_a, wb_s, wb_m, wlen_b, FD_WARPS, kq, topk);
+    wsel = tree_merge(wa, wlen_a, wb, wlen_b, FD_WARPS, lg, topk);
   }
   __syncthreads();
   // ---- push this CTA's list and partial sums into every CTA's stage slot
   cluster_wait_acquire();  // every CTA of the cluster is running
   {
-    const float* my_s = wsel ? wb_s : wa_s;
-    const int* my_m = wsel ? wb_m : wa_m;
+    const unsigned long long* mine = wsel ? wb : wa;
     const int my_len = topk > 0 ? (wsel ? wlen_b[0] : wlen_a[0]) : 0;
     for (int e = tid; e < CS * (my_len + 1); e += FD_THREADS) {
       const int c = e / (my_len + 1), p = e - c * (my_len + 1);
       if (p < my_len) {
-        *cluster.map_shared_rank(sa_s + crank * kq + p, c) = my_s[p];
-        *cluster.map_shared_rank(sa_m + crank * kq + p, c) = my_m[p];
+        *cluster.map_shared_rank(sa + crank * kq + p, c) = mine[p];
       } else {
         *cluster.map_shared_rank(slen_a + crank, c) = my_len;
         *cluster.map_shared_rank(smx + crank, c) = loc_mx;
@@ -323,15 +332,14 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     lse = (C > 0) ? M + __logf(S) : 0.f;
   }
   if (topk > 0) {
-    const int ssel = tree_merge(sa_s, sa_m, slen_a, sb_s, sb_m, slen_b, CS, kq, topk);
-    const float* fs = ssel ? sb_s : sa_s;
-    const int* fm = ssel ? sb_m : sa_m;
+    const int ssel = tree_merge(sa, slen_a, sb, slen_b, CS, lg, topk);
+    const unsigned long long* fk = ssel ? sb : sa;
     for (int i = tid; i < kk; i += FD_THREADS) {  // ascending block order
-      const int mi = fm[i];
+      const int mi = key_block(fk[i]);
       int pos = 0;
-      for (int j = 0; j < kk; ++j) pos += fm[j] < mi;
+      for (int j = 0; j < kk; ++j) pos += key_block(fk[j]) < mi;
       kidx[pos] = mi;
-      klogg[pos] = fs[i] - lse;
+      klogg[pos] = key_score(fk[i]) - lse;
     }
     __syncthreads();
     if (crank == 0 && idx_out != nullptr)
@@ -432,14 +440,19 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         const float* z = zs + h * SAS_BLOCK;
         const float al = alpha_s[h];
         float a0 = acc[it][0] * al, a1 = acc[it][1] * al;
+        float b0 = 0.f, b1 = 0.f;  // two independent chains per column
 #pragma unroll 8
-        for (int j = 0; j < SAS_BLOCK; ++j) {
-          const float pj = z[j];
-          a0 += pj * to_f(vt[(size_t)j * D + c]);
-          a1 += pj * to_f(vt[(size_t)j * D + c + 1]);
+        for (int j = 0; j < SAS_BLOCK; j += 2) {
+          float2 v0, v1;
+          load2(vt + (size_t)j * D + c, v0);
+          load2(vt + (size_t)(j + 1) * D + c, v1);
+          a0 += z[j] * v0.x;
+          a1 += z[j] * v0.y;
+          b0 += z[j + 1] * v1.x;
+          b1 += z[j + 1] * v1.y;
         }
-        acc[it][0] = a0;
-        acc[it][1] = a1;
+        acc[it][0] = a0 + b0;
+        acc[it][1] = a1 + b1;
       }
     }
     __syncthreads();  // slot and zs consumed

@@ -92,9 +92,9 @@ __device__ void score_chunk(const float* __restrict__ ks_row, int m0, int n,
   }
 }
 
-// Best-first list of the min(k, n) best entries of sc[0..n) (blocks m0..).
-template <bool kGlobalOut>
-__device__ void chunk_topk(const float* sc, int m0, int n, int k, float* ls, int* li) {
+// Best-first list of the keys of the min(k, n) best entries of sc[0..n)
+// (blocks m0 + j), by rank counting.
+__device__ void chunk_topk(const float* sc, int m0, int n, int k, unsigned long long* out) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const float si = sc[i];
     int r = 0;
@@ -102,23 +102,20 @@ __device__ void chunk_topk(const float* sc, int m0, int n, int k, float* ls, int
       const float sj = sc[j];
       r += (sj > si) || (sj == si && j < i);
     }
-    if (r < k) {
-      ls[r] = si;
-      li[r] = m0 + i;
-    }
+    if (r < k) out[r] = cand_key(si, m0 + i);
   }
 }
 
-// Writes the kk best entries of a best-first list (s/m) to out_idx/out_logg
-// in ascending block order (log g = s - lse), padded to k with -1 / 0.
-__device__ void write_selection(const float* s, const int* m, int kk, int k, float lse,
+// Writes the kk best entries of a best-first key list to out_idx/out_logg in
+// ascending block order (log g = s - lse), padded to k with -1 / 0.
+__device__ void write_selection(const unsigned long long* keys, int kk, int k, float lse,
                                 int32_t* out_idx, float* out_logg) {
   for (int i = threadIdx.x; i < kk; i += blockDim.x) {
-    const int mi = m[i];
+    const int mi = key_block(keys[i]);
     int pos = 0;
-    for (int j = 0; j < kk; ++j) pos += m[j] < mi;
+    for (int j = 0; j < kk; ++j) pos += key_block(keys[j]) < mi;
     out_idx[pos] = mi;
-    out_logg[pos] = s[i] - lse;
+    out_logg[pos] = key_score(keys[i]) - lse;
   }
   for (int i = kk + threadIdx.x; i < k; i += blockDim.x) {
     out_idx[i] = -1;
@@ -177,10 +174,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
   float* red = sc + SEL_CHUNK_MAX;
   int* len = reinterpret_cast<int*>(red + 32);
   int* len_b = len + nck;
-  float* ls = reinterpret_cast<float*>(len_b + nck);
-  int* li = reinterpret_cast<int*>(ls + (size_t)nchunk * topk);
-  float* ls_b = reinterpret_cast<float*>(li + (size_t)nchunk * topk);
-  int* li_b = reinterpret_cast<int*>(ls_b + (size_t)nchunk * topk);
+  const int lg = ceil_log2(topk);
+  unsigned long long* la = reinterpret_cast<unsigned long long*>(len_b + nck);  // 8-byte aligned
+  unsigned long long* lb = la + ((size_t)nchunk << lg);
 
   const size_t row = ((size_t)b * Hkv + r) * T_ + t;
   const float* qrow = qbar + row * D;
@@ -192,7 +188,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
     const int m0 = c * SEL_CHUNK_MAX, n = min(SEL_CHUNK_MAX, C - m0);
     score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
     __syncthreads();
-    if (topk > 0) chunk_topk<false>(sc, m0, n, topk, ls + (size_t)c * topk, li + (size_t)c * topk);
+    if (topk > 0) chunk_topk(sc, m0, n, topk, la + ((size_t)c << lg));
     float lm = -FLT_MAX;
     for (int i = threadIdx.x; i < n; i += blockDim.x) lm = fmaxf(lm, sc[i]);
     lm = block_reduce_max(lm, red);
@@ -208,8 +204,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
   const int kk = min(topk, C);
   const float lse = (C > 0) ? run_m + __logf(run_s) : 0.f;
   if (topk > 0) {
-    const int wb = tree_merge(ls, li, len, ls_b, li_b, len_b, nchunk, topk, topk);
-    write_selection(wb ? ls_b : ls, wb ? li_b : li, kk, topk, lse, idx + row * topk,
+    const int wb = tree_merge(la, len, lb, len_b, nchunk, lg, topk);
+    write_selection(wb ? lb : la, kk, topk, lse, idx + row * topk,
                     logg + row * topk);
   }
   if (threadIdx.x == 0) cnt[row] = kk;
@@ -223,8 +219,8 @@ size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d) {
 static size_t prefill_select_smem(int d, int nchunk, int topk) {
   size_t n = (size_t)d + SEL_CHUNK_MAX + 32;  // q, sc, red
   n += 2 * (size_t)((nchunk + 3) & ~3);       // len, len_b
-  n += 4 * (size_t)nchunk * topk;             // ls, li, ls_b, li_b
-  return n * 4;
+  n += 4 * ((size_t)nchunk << ceil_log2(topk));  // two key buffers (8 bytes each)
+  return n * 4 + 8;
 }
 
 cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
@@ -305,14 +301,13 @@ cudaError_t launch_select_prefill_static(const void* q, int bf16, const float* k
 // ------------------------------------------------------------------ decode
 // Scratch layout per plan (rows = B*Hkv, nchunk chunks per row):
 //   counters [rows] int | len [rows][nchunk] int | cmax, csum [rows][nchunk]
-//   float | ls [rows][nchunk][k] float | li [rows][nchunk][k] int
+//   float | keys [rows][nchunk][k] u64
 struct DecodeSelectWs {
   int* counter;
   int* len;
   float* cmax;
   float* csum;
-  float* ls;
-  int* li;
+  unsigned long long* lk;
 };
 
 static size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -325,15 +320,14 @@ static DecodeSelectWs carve_decode_select(int* counters, void* ws, const SelectP
   w.len = reinterpret_cast<int*>(c); c += align16(sizeof(int) * rc);
   w.cmax = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc);
   w.csum = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc);
-  w.ls = reinterpret_cast<float*>(c); c += align16(sizeof(float) * rc * p.topk);
-  w.li = reinterpret_cast<int*>(c);
+  w.lk = reinterpret_cast<unsigned long long*>(c);
   return w;
 }
 
 size_t decode_select_ws_bytes(const SelectPlan& p) {
   const size_t rc = (size_t)p.rows * p.nchunk;
   return align16(sizeof(int) * rc) + 2 * align16(sizeof(float) * rc) +
-         align16(sizeof(float) * rc * p.topk) + align16(sizeof(int) * rc * p.topk);
+         align16(sizeof(unsigned long long) * rc * p.topk);
 }
 
 SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk) {
@@ -355,7 +349,7 @@ SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk) {
 
 static size_t decode_merge_smem(int nchunk, int topk) {
   const size_t nck = (nchunk + 3) & ~3;
-  return sizeof(float) * (4 * nck + 4 * (size_t)nchunk * topk);
+  return sizeof(float) * 4 * nck + 2 * 8 * ((size_t)nchunk << ceil_log2(topk));
 }
 
 template <typename T, int D>
@@ -386,7 +380,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
   __syncthreads();
   const size_t rc = (size_t)row * nchunk + c;
-  if (topk > 0) chunk_topk<true>(sc, m0, n, topk, w.ls + rc * topk, w.li + rc * topk);
+  if (topk > 0) chunk_topk(sc, m0, n, topk, w.lk + rc * topk);
   float lm = -FLT_MAX;
   for (int i = threadIdx.x; i < n; i += blockDim.x) lm = fmaxf(lm, sc[i]);
   lm = block_reduce_max(lm, red);
@@ -416,10 +410,9 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   float* cs_s = cm_s + nck;
   int* len_s = reinterpret_cast<int*>(cs_s + nck);
   int* len_b = len_s + nck;
-  float* ls_s = reinterpret_cast<float*>(len_b + nck);
-  int* li_s = reinterpret_cast<int*>(ls_s + (size_t)nchunk * topk);
-  float* ls_b = reinterpret_cast<float*>(li_s + (size_t)nchunk * topk);
-  int* li_b = reinterpret_cast<int*>(ls_b + (size_t)nchunk * topk);
+  const int lg = ceil_log2(topk);
+  unsigned long long* la = reinterpret_cast<unsigned long long*>(len_b + nck);
+  unsigned long long* lb = la + ((size_t)nchunk << lg);
   const size_t r0 = (size_t)row * nchunk;
   for (int i = threadIdx.x; i < nchunk; i += blockDim.x) {
     cm_s[i] = __ldcg(w.cmax + r0 + i);  // empty chunks: -FLT_MAX and 0
@@ -429,10 +422,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   __syncthreads();
   for (int e = threadIdx.x; e < nchunk * topk; e += blockDim.x) {
     const int cc = e / topk, p = e - cc * topk;
-    if (p < len_s[cc]) {
-      ls_s[e] = __ldcg(w.ls + r0 * topk + e);
-      li_s[e] = __ldcg(w.li + r0 * topk + e);
-    }
+    if (p < len_s[cc]) la[((size_t)cc << lg) + p] = __ldcg(w.lk + r0 * topk + e);
   }
   float mx = -FLT_MAX;
   for (int i = threadIdx.x; i < nchunk; i += blockDim.x) mx = fmaxf(mx, cm_s[i]);
@@ -445,8 +435,8 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   const int kk = min(topk, C);
   if (topk > 0) {
     __syncthreads();
-    const int wb = tree_merge(ls_s, li_s, len_s, ls_b, li_b, len_b, nchunk, topk, topk);
-    write_selection(wb ? ls_b : ls_s, wb ? li_b : li_s, kk, topk, lse, idx + (size_t)row * topk,
+    const int wb = tree_merge(la, len_s, lb, len_b, nchunk, lg, topk);
+    write_selection(wb ? lb : la, kk, topk, lse, idx + (size_t)row * topk,
                     logg + (size_t)row * topk);
   }
   if (threadIdx.x == 0) {

@@ -58,8 +58,11 @@ def measured_peaks() -> dict:
 
 
 def source_sha(name: str) -> str:
-    p = os.path.join(ROOT, "gated_block_sparse_b200", "csrc", name)
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    """Hash of a kernel's source file and the shared device headers."""
+    h = hashlib.sha256()
+    for f in (name, "common.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "gated_block_sparse_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, source: str):

@@ -202,6 +202,11 @@ sas_status sas_attn_fwd(const void* q, const void* k, const void* v, sas_dtype d
   if (s != SAS_OK) return s;
   REQUIRE_PTR(o);
   REQUIRE_PTR(lse);
+  if (sas::attn_fwd_tc_supported(dt == SAS_BF16, d, Hq, Hkv) && topk > 0)
+    return cuda_status(sas::launch_attn_fwd_tc(q, k, v, B, Hq, Hkv, N, idx, cnt, logg, topk,
+                                               resolve_scale(scale, d), o, lse,
+                                               (cudaStream_t)stream),
+                       "sas_attn_fwd launch");
   return cuda_status(sas::launch_attn_fwd_simt(q, k, v, dt == SAS_BF16, B, Hq, Hkv, N, d, idx, cnt,
                                                logg, topk, resolve_scale(scale, d), o, lse,
                                                (cudaStream_t)stream),

@@ -1,0 +1,328 @@
+// Gated sparse attention forward on the 5th-generation tensor cores (bf16,
+// d = 128): TMA-fed tcgen05 MMAs with TMEM accumulators.
+//
+// Definition (SAS close reading, liuzhao09.github.io, sections 2.1, 2.2 and
+// 2.4; SAS reproduction note, daiwk.github.io, core formula): for query row i
+// of block t, z_ij = scale * q_i . k_j + log g of j's block over the kept
+// history blocks, and z_ij = scale * q_i . k_j over keys j <= i of the
+// current block; o_i = softmax(z) V, lse_i = log sum exp z. The gate is added
+// to the QK^T tile before the online-softmax update; unselected blocks are
+// never loaded; the score matrix is never materialised.
+//
+// One CTA per (query block t, kv group r, pair of query heads of the group):
+// an M = 128 tile (2 heads x 64 rows) that shares every K/V block it loads.
+//   warp 4     TMA producer: Q once (4 boxes of 64 rows x 64 columns, 128-byte
+//              swizzle), then K and V of each unit into a 2-stage ring;
+//   warp 5     one elected thread issues tcgen05.mma: S_j = Q K_j^T
+//              (M128 N64 K128, two TMEM buffers of 64 columns) and
+//              O += P_j V_j (M128 N128 K64, 128 TMEM columns);
+//   warps 0-3  softmax: thread i owns row i = TMEM lane i; loads S_j,
+//              applies scale, bias and the causal mask in the log2 domain,
+//              updates the running max lazily (O in TMEM is rescaled only when
+//              the max grows by more than 2^8), writes P_j as bf16 into shared
+//              memory in the 128-byte-swizzled K-major layout the MMA reads;
+//              at the end divides O by the row sum and writes o and lse.
+// About 113 KB of shared memory and 256 TMEM columns per CTA, so two CTAs
+// share an SM and overlap one's softmax with the other's MMAs. Every wait is
+// bounded.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "tc.cuh"
+
+namespace sas {
+
+__device__ uint32_t g_attn_fwd_tc_err = 0;
+
+namespace {
+
+constexpr int FT_THREADS = 192;
+constexpr int D = 128;
+constexpr uint32_t Q_BYTES = 128 * D * 2;           // 32 KB
+constexpr uint32_t KV_STAGE_BYTES = 2 * 64 * D * 2;  // K + V block, 32 KB
+constexpr uint32_t P_BYTES = 128 * 64 * 2;          // 16 KB
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = OFF_Q + Q_BYTES;
+constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RESCALE_LOG2 = 8.0f;  // lazy rescale threshold (log2 units)
+
+enum Bar { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 10, NBAR = 11 };
+
+}  // namespace
+
+__global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+    const __grid_constant__ CUtensorMap vmap, int Hq, int Hkv, int N,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
+    const float* __restrict__ logg, int topk, float scale, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ lse) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
+  uint32_t* err = &g_attn_fwd_tc_err;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = Hq / Hkv, pairs = G / 2;
+  const int T_ = gridDim.x;
+  const int t = T_ - 1 - (int)blockIdx.x;  // longest rows first
+  const int r = blockIdx.y / pairs, hp = blockIdx.y % pairs, b = blockIdx.z;
+  const int h0 = r * G + 2 * hp;
+  const size_t srow = ((size_t)b * Hkv + r) * T_ + t;
+  const int kk = min(max(cnt[srow], 0), topk);
+  const int nunits = kk + 1;  // kept history blocks, then the current block
+  const int32_t* idx_row = idx + srow * topk;
+  const float* logg_row = logg + srow * topk;
+  if ((smem_u32(sm) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
+    if (tid == 0) atomicOr(err, kErrBadIndex);
+    return;
+  }
+  if (tid == 0) {
+    // S-empty (both buffers) and P-full take one arrival per softmax warp
+    for (int i = 0; i < NBAR; ++i)
+      mbar_init(&bars[i], (i == B_SE || i == B_SE + 1 || i == B_PF) ? 4 : 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) tc::tmem_alloc(tmem_slot, 256);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_s[2] = {tmem, tmem + 64};
+  const uint32_t tm_o = tmem + 128;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tc::prefetch_map(&qmap);
+      tc::prefetch_map(&kmap);
+      tc::prefetch_map(&vmap);
+      mbar_arrive_expect_tx(&bars[B_Q], Q_BYTES);
+      for (int c = 0; c < 2; ++c)
+        for (int h = 0; h < 2; ++h)
+          tc::tma_load_3d(sm + OFF_Q + c * 16384 + h * 8192, &qmap, 64 * c, 64 * t,
+                          b * Hq + h0 + h, &bars[B_Q]);
+      for (int j = 0; j < nunits; ++j) {
+        const int s = j & 1;
+        if (j >= 2) mbar_wait(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
+        int blk = (j < kk) ? idx_row[j] : t;
+        if (blk < 0 || blk >= t) {
+          if (j < kk) atomicOr(err, kErrBadIndex);
+          blk = t;
+        }
+        unsigned char* st = sm + OFF_KV + s * KV_STAGE_BYTES;
+        mbar_arrive_expect_tx(&bars[B_KVF + s], KV_STAGE_BYTES);
+        const int plane = b * Hkv + r;
+        tc::tma_load_3d(st, &kmap, 0, 64 * blk, plane, &bars[B_KVF + s]);
+        tc::tma_load_3d(st + 8192, &kmap, 64, 64 * blk, plane, &bars[B_KVF + s]);
+        tc::tma_load_3d(st + 16384, &vmap, 0, 64 * blk, plane, &bars[B_KVF + s]);
+        tc::tma_load_3d(st + 24576, &vmap, 64, 64 * blk, plane, &bars[B_KVF + s]);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_QK = tc::idesc_bf16(128, 64, 0, 0);
+      constexpr uint32_t ID_PV = tc::idesc_bf16(128, 128, 0, 1);
+      const uint32_t q_addr = smem_u32(sm + OFF_Q);
+      const uint32_t p_addr = smem_u32(sm + OFF_P);
+      mbar_wait(&bars[B_Q], 0, err);
+      auto pv = [&](int j) {  // O += P_j V_j
+        mbar_wait(&bars[B_PF], j & 1, err);
+        tc::fence_after_sync();
+        const uint32_t v_addr = smem_u32(sm + OFF_KV + (j & 1) * KV_STAGE_BYTES + 16384);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t a = tc::sw128_desc(p_addr + ks * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(v_addr + ks * 2048, 8192, 1024);
+          tc::mma_bf16(tm_o, a, bd, ID_PV, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc::commit(&bars[B_OD]);
+        tc::commit(&bars[B_KVE + (j & 1)]);
+      };
+      for (int j = 0; j < nunits; ++j) {
+        const int s = j & 1;
+        mbar_wait(&bars[B_KVF + s], (j >> 1) & 1, err);
+        if (j >= 2) mbar_wait(&bars[B_SE + s], ((j >> 1) - 1) & 1, err);
+        tc::fence_after_sync();
+        const uint32_t k_addr = smem_u32(sm + OFF_KV + s * KV_STAGE_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {  // K = 128 in steps of 16 (32 bytes)
+          const uint32_t c = ks >> 2, off = (ks & 3) * 32;
+          const uint64_t a = tc::sw128_desc(q_addr + c * 16384 + off, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(k_addr + c * 8192 + off, 16, 1024);
+          tc::mma_bf16(tm_s[s], a, bd, ID_QK, ks > 0 ? 1u : 0u);
+        }
+        tc::commit(&bars[B_SF + s]);
+        if (j >= 1) pv(j - 1);
+      }
+      pv(nunits - 1);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int row = tid;  // 0..127 = TMEM lane
+    const int hh = row >> 6, qr = row & 63;
+    const int pos = 64 * t + qr;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float c1 = scale * LOG2E;
+    float m = -1e30f, l = 0.f;
+    unsigned char* prow = sm + OFF_P + row * 128;
+    for (int j = 0; j < nunits; ++j) {
+      const int s = j & 1;
+      const bool cur = (j == kk);
+      const float bias = cur ? 0.f : logg_row[j] * LOG2E;
+      mbar_wait(&bars[B_SF + s], (j >> 1) & 1, err);
+      tc::fence_after_sync();
+      float z[64];
+      {
+        float a[32], bb[32];
+        tc::tmem_ld32(tm_s[s] + lane_off, a);
+        tc::tmem_ld32(tm_s[s] + lane_off + 32, bb);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          z[i] = a[i];
+          z[32 + i] = bb[i];
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_SE + s]);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        float v = z[i] * c1 + bias;
+        if (cur && i > qr) v = -INFINITY;
+        z[i] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float mnew = fmaxf(m, mx);
+      const bool grow = (j == 0) || (mnew > m + RESCALE_LOG2);
+      const float muse = grow ? mnew : m;
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = exp2f(z[2 * i] - muse), p1 = exp2f(z[2 * i + 1] - muse);
+        rs += p0 + p1;
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      if (j > 0) {
+        // PV_{j-1} must be done: O is stable and the P buffer is free
+        mbar_wait(&bars[B_OD], (j - 1) & 1, err);
+        tc::fence_after_sync();
+        const float alpha = grow ? exp2f(m - muse) : 1.f;
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float ov[32];
+            tc::tmem_ld32(tm_o + lane_off + 32 * c, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tc::tmem_st32(tm_o + lane_off + 32 * c, ov);
+          }
+          tc::tmem_wait_st();
+        }
+        l = l * alpha + rs;
+      } else {
+        l = rs;
+      }
+      m = muse;
+      // P row (64 bf16 = 8 chunks of 16 bytes), 128-byte swizzle: chunk c of
+      // row i sits at chunk position c ^ (i & 7)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_PF]);
+    }
+    // epilogue
+    mbar_wait(&bars[B_OD], (nunits - 1) & 1, err);
+    tc::fence_after_sync();
+    const float inv = 1.f / l;
+    const bool valid = pos < N;
+    __nv_bfloat16* orow = o + (((size_t)b * Hq + h0 + hh) * N + (valid ? pos : 0)) * D;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float ov[32];
+      tc::tmem_ld32(tm_o + lane_off + 32 * c, ov);
+      tc::tmem_wait_ld();
+      if (valid) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * g + 2 * e] * inv,
+                                                      ov[8 * g + 2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(orow + 32 * c + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    if (valid) lse[((size_t)b * Hq + h0 + hh) * N + pos] = (m + log2f(l)) / LOG2E;
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ------------------------------------------------------------------ host
+static bool make_map(CUtensorMap* map, const void* base, int rows_per_plane, int planes) {
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows_per_plane, (cuuint64_t)planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows_per_plane * D * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = cuTensorMapEncodeTiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                                      const_cast<void*>(base), dims, strides, box, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool attn_fwd_tc_supported(int bf16, int d, int Hq, int Hkv) {
+  const int G = Hq / Hkv;
+  return bf16 && d == 128 && G >= 2 && (G % 2) == 0;
+}
+
+cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq,
+                               int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* o, float* lse,
+                               cudaStream_t st) {
+  const int T_ = (N + 63) / 64;
+  if (B == 0 || T_ == 0) return cudaSuccess;
+  CUtensorMap qm, km, vm;
+  if (!make_map(&qm, q, N, B * Hq) || !make_map(&km, k, N, B * Hkv) ||
+      !make_map(&vm, v, N, B * Hkv))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem(k_attn_fwd_tc, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(T_, Hkv * (Hq / Hkv / 2), B);
+  k_attn_fwd_tc<<<grid, FT_THREADS, SMEM_BYTES, st>>>(qm, km, vm, Hq, Hkv, N, idx, cnt, logg,
+                                                       topk, scale,
+                                                       static_cast<__nv_bfloat16*>(o), lse);
+  return cudaGetLastError();
+}
+
+uint32_t* attn_fwd_tc_error_word() {
+  void* p = nullptr;
+  cudaGetSymbolAddress(&p, g_attn_fwd_tc_err);
+  return static_cast<uint32_t*>(p);
+}
+
+}  // namespace sas

@@ -65,6 +65,13 @@ cudaError_t launch_attn_fwd_simt(const void* q, const void* k, const void* v, in
                                  int Hq, int Hkv, int N, int d, const int32_t* idx,
                                  const int32_t* cnt, const float* logg, int topk, float scale,
                                  void* o, float* lse, cudaStream_t st);
+// Tensor-core forward (tcgen05 + TMEM + TMA): bf16, d = 128, even group size.
+bool attn_fwd_tc_supported(int bf16, int d, int Hq, int Hkv);
+cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq,
+                               int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* o, float* lse,
+                               cudaStream_t st);
+uint32_t* attn_fwd_tc_error_word();
 size_t attn_bwd_simt_ws_bytes(int B, int Hkv, int N, int d);
 cudaError_t launch_attn_bwd_simt(const void* q, const void* k, const void* v, const void* o,
                                  const void* dout, int bf16, int B, int Hq, int Hkv, int N, int d,

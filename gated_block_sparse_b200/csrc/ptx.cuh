@@ -1,6 +1,6 @@
 // Inline-PTX wrappers for sm_100a: mbarriers, bulk (TMA) copies, fences.
-// Every wait is bounded: after kSpinLimit polls it records an error code in
-// a device flag and returns false, so a lost arrival cannot hang the GPU.
+// Every wait is bounded in time: it records an error code in a device flag
+// and returns false, so a lost arrival cannot hang the GPU.
 #pragma once
 
 #include <stdint.h>
@@ -10,8 +10,6 @@ namespace sas {
 // Device-side error word, read back by the host API after a kernel (0 = ok).
 // Kernels OR in one of these bits when a bounded wait gives up.
 enum : uint32_t { kErrWaitTimeout = 1u, kErrBadIndex = 2u };
-
-constexpr uint32_t kSpinLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -53,11 +51,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wall-clock bound of one wait. A try_wait may suspend the thread for a
+// hardware-chosen time, so the bound is on time, not on the poll count.
+constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;  // 200 ms
+
 // Bounded wait for the phase with the given parity to complete. Returns false
-// (and sets kErrWaitTimeout in *err when err is non-null) if it gives up.
+// if it gives up: after kWaitLimitNs, or at once when *err already carries
+// kErrWaitTimeout (a wait elsewhere timed out: the launch is aborting, so no
+// further wait may stall). A timeout sets kErrWaitTimeout in *err.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0) {
+      if (err && (*reinterpret_cast<volatile uint32_t*>(err) & kErrWaitTimeout)) return false;
+      if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
   if (err) atomicOr(err, kErrWaitTimeout);
   return false;
 }

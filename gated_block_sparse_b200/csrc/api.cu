@@ -240,6 +240,11 @@ sas_status sas_attn_bwd(const void* q, const void* k, const void* v, const void*
   const size_t need = sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt);
   REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
   REQUIRE_PTR(ws);
+  if (sas::attn_fwd_tc_supported(dt == SAS_BF16, d, Hq, Hkv) && topk > 0)
+    return cuda_status(sas::launch_attn_bwd_tc(q, k, v, o, dout, B, Hq, Hkv, N, lse, idx, cnt,
+                                               logg, topk, resolve_scale(scale, d), dq, dk, dv,
+                                               dlogg, ws, (cudaStream_t)stream),
+                       "sas_attn_bwd launch");
   return cuda_status(sas::launch_attn_bwd_simt(q, k, v, o, dout, dt == SAS_BF16, B, Hq, Hkv, N, d,
                                                lse, idx, cnt, logg, topk, resolve_scale(scale, d),
                                                dq, dk, dv, dlogg, ws, (cudaStream_t)stream),

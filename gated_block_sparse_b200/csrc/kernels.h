@@ -72,6 +72,13 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int 
                                const float* logg, int topk, float scale, void* o, float* lse,
                                cudaStream_t st);
 uint32_t* attn_fwd_tc_error_word();
+// Tensor-core backward (same support as the forward); ws as attn_bwd_simt.
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, int B, int Hq, int Hkv, int N,
+                               const float* lse, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* dq, void* dk,
+                               void* dv, float* dlogg, void* ws, cudaStream_t st);
+uint32_t* attn_bwd_tc_error_word();
 size_t attn_bwd_simt_ws_bytes(int B, int Hkv, int N, int d);
 cudaError_t launch_attn_bwd_simt(const void* q, const void* k, const void* v, const void* o,
                                  const void* dout, int bf16, int B, int Hq, int Hkv, int N, int d,

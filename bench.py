@@ -437,20 +437,26 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
     ms_b, _ = timed_graphs(bwd_step, max(3, K), 2, world, stream, chunk=8)
     tf, tb = ms_f / max(3, K) * 1e-3, ms_b / max(3, K) * 1e-3
     peaks = measured_peaks()
-    simt_peak = 148 * 128 * 2 * peaks["sm_max"] * 1e6 / 1e12  # fp32 FMA lanes x 2 x clock
-    if tb >= tf:
-        kern, kf, kt = "k_attn_bwd_simt", f_bwd, tb
-    else:
-        kern, kf, kt = "k_attn_fwd_simt", f_fwd, tf
+    tensor = c["dtype"] == "bf16" and d == 128 and (Hq // Hkv) % 2 == 0
+    if tensor:  # tcgen05 kernels, timed alone: the burst bf16 peak
+        names = ("k_attn_fwd_tc", "k_attn_bwd_tc")
+        srcs = ("k_attn_fwd_tc.cu", "k_attn_bwd_tc.cu")
+        peak, bound = peaks["bf16"], "tensor"
+        psrc = f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, cuBLAS bf16 burst)"
+    else:  # fp32 CUDA-core kernels
+        names = ("k_attn_fwd_simt", "k_attn_bwd_simt")
+        srcs = ("k_attn_simt.cu", "k_attn_simt.cu")
+        peak, bound = 148 * 128 * 2 * peaks["sm_max"] * 1e6 / 1e12, "alu"
+        psrc = "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock"
+    i = 1 if tb >= tf else 0
+    kern, kf, kt = names[i], (f_fwd, f_bwd)[i], (tf, tb)[i]
     ach = kf / kt / 1e12
-    roof = {"bound": "alu", "kernel": kern, "achieved": round(ach, 3), "peak": round(simt_peak, 1),
-            "unit": "TFLOP/s", "frac": round(ach / simt_peak, 4),
-            "traffic": recorded_traffic(kern, "k_attn_simt.cu"),
-            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x max SM clock "
-                           "(fp32 CUDA-core path)",
+    roof = {"bound": bound, "kernel": kern, "achieved": round(ach, 2), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+            "traffic": recorded_traffic(kern, srcs[i]), "peak_source": psrc,
             "algorithmic_flops_per_launch": kf, "launch_ms": round(kt * 1e3, 4),
             "fwd_ms": round(tf * 1e3, 4), "bwd_ms": round(tb * 1e3, 4),
-            "bf16_tensor_peak_for_reference": peaks["bf16"]}
+            "fwd_tflops": round(f_fwd / tf / 1e12, 2), "bwd_tflops": round(f_bwd / tb / 1e12, 2)}
 
     # end to end: pinned host inputs in, gradients out
     pin = {n: torch.empty(h[n].shape, dtype=h[n].dtype, pin_memory=True) for n in ("q", "k", "v", "do")}
@@ -488,7 +494,7 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
         "roofline": roof,
         "e2e": {"value": round(total * E * world / (ms_e2e * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 7 * K,
+        "gpu_launches": 7 * K,  # summary, query means, selection, forward, backward, 2 conversions
         "clocks": clk,
     }
 

@@ -17,13 +17,18 @@
 // 128-byte-swizzled layout; the same buffer is the K-major A operand of dQ
 // and the MN-major B operand of dK^T (P likewise for dV^T). dK^T / dV^T are
 // double-buffered in TMEM; the softmax warps, which own TMEM lanes = d,
-// read them and add them into fp32 accumulators of dk and dv (coalesced
-// reductions; a conversion pass writes the output dtype). dlogg is summed
-// in-CTA in a fixed order and added once per CTA.
-//   warp 4: TMA (Q and dO once; K and V of each unit into a 2-stage ring)
-//   warp 5: one thread issues all MMAs
-//   warps 0-3: softmax / gradient rows and the reductions
-// 512 TMEM columns and about 161 KB of shared memory: one CTA per SM.
+// read them and add them into fp32 accumulators of dk and dv (a conversion
+// pass writes the output dtype). dlogg is summed in-CTA in a fixed order and
+// added once per CTA.
+//   warp 8: TMA (Q and dO once; K and V of each unit into a 2-stage ring)
+//   warp 9: one thread issues all MMAs; S/dP of unit j+1 are issued while
+//           the gradient warps form unit j's P and dS
+//   warps 0-7: gradient rows: warps w and w+4 share the TMEM lanes of rows
+//           32(w%4).. and split the 64 key columns, two warps per SM
+//           sub-partition to hide instruction latency
+// dK^T / dV^T are added to the fp32 accumulators through a shared-memory
+// transpose and 16-byte vector reductions.
+// 512 TMEM columns and about 193 KB of shared memory: one CTA per SM.
 #include <cuda.h>
 #include <math.h>
 
@@ -38,7 +43,8 @@ __device__ uint32_t g_attn_bwd_tc_err = 0;
 
 namespace {
 
-constexpr int BT_THREADS = 192;
+constexpr int BT_THREADS = 320;  // 8 gradient warps, TMA warp, MMA warp
+constexpr int NGW = 8;           // gradient warps
 constexpr int D = 128;
 constexpr uint32_t TILE128 = 128 * D * 2;            // Q or dO: 32 KB
 constexpr uint32_t KV_STAGE = 2 * 64 * D * 2;        // K + V: 32 KB
@@ -48,7 +54,8 @@ constexpr uint32_t OFF_DO = OFF_Q + TILE128;
 constexpr uint32_t OFF_KV = OFF_DO + TILE128;
 constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;
 constexpr uint32_t OFF_DS = OFF_P + PT_BYTES;
-constexpr uint32_t OFF_BAR = OFF_DS + PT_BYTES;
+constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [64 keys][128 d] transpose
+constexpr uint32_t OFF_BAR = OFF_T + 64 * D * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -68,12 +75,9 @@ enum Bar {
 constexpr uint32_t C_S = 0, C_DP = 64, C_DQ = 128, C_DKT = 256, C_DVT = 320, C_BUF = 128;
 
 __device__ __forceinline__ void named_bar_softmax() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-__device__ __forceinline__ void red_add(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
 
 }  // namespace
 
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   extern __shared__ __align__(1024) unsigned char sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
-  float* red_s = reinterpret_cast<float*>(sm + OFF_BAR + NBAR * 8 + 16);  // [4]
+  float* red_s = reinterpret_cast<float*>(sm + OFF_BAR + NBAR * 8 + 16);  // [NGW]
   uint32_t* err = &g_attn_bwd_tc_err;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = Hq / Hkv, pairs = G / 2;
@@ -112,18 +116,18 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   };
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool four = (i == B_SE || i == B_PF || i == B_TE || i == B_TE + 1);
-      mbar_init(&bars[i], four ? 4 : 1);
+      const bool per_warp = (i == B_SE || i == B_PF || i == B_TE || i == B_TE + 1);
+      mbar_init(&bars[i], per_warp ? NGW : 1);
     }
     fence_mbar_init();
   }
-  if (warp == 5) tc::tmem_alloc(tmem_slot, 512);
+  if (warp == 9) tc::tmem_alloc(tmem_slot, 512);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tc::prefetch_map(&qmap);
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         tc::tma_load_3d(st + 24576, &vmap, 64, 64 * blk, plane, &bars[B_KVF + s]);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ID_N64 = tc::idesc_bf16(128, 64, 0, 0);     // S, dP
@@ -161,7 +165,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
       const uint32_t q_a = smem_u32(sm + OFF_Q), do_a = smem_u32(sm + OFF_DO);
       const uint32_t p_a = smem_u32(sm + OFF_P), ds_a = smem_u32(sm + OFF_DS);
       mbar_wait(&bars[B_Q], 0, err);
-      for (int j = 0; j < nunits; ++j) {
+      // S/dP of unit j+1 are issued as soon as the gradient warps have copied
+      // S/dP of unit j into registers, so they run while unit j's P and dS are
+      // being formed; the dQ / dK^T / dV^T products of unit j follow.
+      auto issue_sdp = [&](int j) {
         const int s = j & 1;
         const uint32_t k_a = smem_u32(sm + OFF_KV + s * KV_STAGE);
         const uint32_t v_a = k_a + 16384;
@@ -177,6 +184,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
                        tc::sw128_desc(v_a + c * 8192 + off, 16, 1024), ID_N64, ks > 0);
         }
         tc::commit(&bars[B_SF]);
+      };
+      auto issue_grad = [&](int j) {
+        const int s = j & 1;
+        const uint32_t k_a = smem_u32(sm + OFF_KV + s * KV_STAGE);
         mbar_wait(&bars[B_PF], j & 1, err);
         if (j >= 2) mbar_wait(&bars[B_TE + s], ((j >> 1) - 1) & 1, err);
         tc::fence_after_sync();
@@ -194,15 +205,24 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         }
         tc::commit(&bars[B_MD]);
         tc::commit(&bars[B_KVE + s]);
+      };
+      issue_sdp(0);
+      for (int j = 0; j < nunits; ++j) {
+        if (j + 1 < nunits) issue_sdp(j + 1);
+        issue_grad(j);
       }
     }
   } else {
     // ---------------------------------------------------------------- gradient rows
-    const int row = tid;  // TMEM lane: query row for S/dP/dQ, head dim d for dK^T/dV^T
+    // Warps w and w + 4 share TMEM lanes 32(w%4)..+31 (query rows for S/dP/dQ,
+    // head dim for dK^T/dV^T) and split the columns: hc = w / 4 takes keys
+    // 32hc..32hc+31 of S/dP/dK^T/dV^T and columns 64hc..64hc+63 of dQ.
+    const int wq = warp & 3, hc = warp >> 2;
+    const int row = wq * 32 + lane;
     const int hh = row >> 6, qr = row & 63;
     const int pos = 64 * t + qr;
     const bool valid = pos < N;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float c1 = scale * LOG2E;
     const size_t qrow = ((size_t)b * Hq + h0 + hh) * N + (valid ? pos : 0);
     float Di = 0.f, lse2 = 0.f;
@@ -217,66 +237,65 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         for (int e = 0; e < 8; ++e) Di += a[e] * g[e];
       }
       lse2 = lse[qrow] * LOG2E;
+    } else {
+      lse2 = INFINITY;  // rows past N: every p is 2^-inf = 0
     }
     unsigned char* prow = sm + OFF_P + row * 128;
     unsigned char* dsrow = sm + OFF_DS + row * 128;
     const size_t kvbase = ((size_t)b * Hkv + r) * N * D;
-    auto flush_kv = [&](int jj) {  // add unit jj's dK^T / dV^T (lane = d) to the accumulators
+    float* tsm = reinterpret_cast<float*>(sm + OFF_T);
+    const int gtid = hc * 128 + row;  // 0..255 over the gradient warps
+    // Add unit jj's dK^T / dV^T (TMEM lanes = d, columns = keys) to the fp32
+    // accumulators: transpose through shared memory into [key][d], then one
+    // 16-byte vector reduction per four head-dim values.
+    auto flush_kv = [&](int jj) {
       const int blk = unit_block(jj);
+      const int nkeys = min(64, N - 64 * blk);
       const uint32_t cb = tmem + (jj & 1) * C_BUF + lane_off;
-      const int dcol = row;
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float kv[32], vv[32];
-        tc::tmem_ld32(cb + C_DKT + 32 * half, kv);
-        tc::tmem_ld32(cb + C_DVT + 32 * half, vv);
+      for (int m2 = 0; m2 < 2; ++m2) {
+        float* acc = m2 == 0 ? dk_acc : dv_acc;
+        float kv[32];
+        tc::tmem_ld32(cb + (m2 == 0 ? C_DKT : C_DVT) + 32 * hc, kv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = 64 * blk + 32 * half + i;
-          if (key < N) {
-            red_add(dk_acc + kvbase + (size_t)key * D + dcol, kv[i]);
-            red_add(dv_acc + kvbase + (size_t)key * D + dcol, vv[i]);
+        for (int i = 0; i < 32; ++i) tsm[(32 * hc + i) * D + row] = kv[i];
+        named_bar_softmax();
+        float* dst = acc + kvbase + (size_t)(64 * blk) * D;
+#pragma unroll 4
+        for (int e = gtid; e < 64 * (D / 4); e += 2 * 128) {
+          const int key = e >> 5, d4 = (e & 31) << 2;
+          if (key < nkeys) {
+            const float4 x = *reinterpret_cast<const float4*>(tsm + key * D + d4);
+            tc::red_add_v4(dst + (size_t)key * D + d4, x.x, x.y, x.z, x.w);
           }
         }
+        named_bar_softmax();
       }
     };
     for (int j = 0; j < nunits; ++j) {
-      const int s = j & 1;
       const bool cur = (j == kk);
       const float bias = cur ? 0.f : logg_row[j] * LOG2E;
       mbar_wait(&bars[B_SF], j & 1, err);
       tc::fence_after_sync();
-      float sv[64], dp[64];
-      {
-        float a0[32], a1[32];
-        tc::tmem_ld32(tmem + C_S + lane_off, a0);
-        tc::tmem_ld32(tmem + C_S + lane_off + 32, a1);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = a0[i];
-          sv[32 + i] = a1[i];
-        }
-        tc::tmem_ld32(tmem + C_DP + lane_off, a0);
-        tc::tmem_ld32(tmem + C_DP + lane_off + 32, a1);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          dp[i] = a0[i];
-          dp[32 + i] = a1[i];
-        }
-      }
+      float sv[32], dp[32];
+      tc::tmem_ld32(tmem + C_S + lane_off + 32 * hc, sv);
+      tc::tmem_ld32(tmem + C_DP + lane_off + 32 * hc, dp);
+      tc::tmem_wait_ld();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_SE]);
       float dsum = 0.f;
-      uint32_t pk[32], dk2[32];
+      uint32_t pk[16], dk2[16];
+      if (cur) {  // causal mask inside the current block
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        float p0 = exp2f(sv[i] * c1 + bias - lse2), p1 = exp2f(sv[i + 1] * c1 + bias - lse2);
-        if (!valid || (cur && i > qr)) p0 = 0.f;
-        if (!valid || (cur && i + 1 > qr)) p1 = 0.f;
+        for (int i = 0; i < 32; ++i)
+          if (32 * hc + i > qr) sv[i] = -INFINITY;
+      }
+      const float off = bias - lse2;
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float p0 = tc::ex2(fmaf(sv[i], c1, off)), p1 = tc::ex2(fmaf(sv[i + 1], c1, off));
         const float d0 = p0 * (dp[i] - Di), d1 = p1 * (dp[i + 1] - Di);
         dsum += d0 + d1;
         __nv_bfloat162 hp2 = __floats2bfloat162_rn(p0, p1);
@@ -289,8 +308,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         tc::fence_after_sync();
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int pc = (c ^ (row & 7)) << 4;
+      for (int c = 0; c < 4; ++c) {  // 16-byte chunks 4hc..4hc+3 of the row, swizzled
+        const int pc = ((4 * hc + c) ^ (row & 7)) << 4;
         *reinterpret_cast<uint4*>(prow + pc) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         *reinterpret_cast<uint4*>(dsrow + pc) =
@@ -310,16 +329,21 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         dsum = warp_sum(dsum);
         if (lane == 0) red_s[warp] = dsum;
         named_bar_softmax();
-        if (tid == 0) atomicAdd(dlogg + srow * topk + j, red_s[0] + red_s[1] + red_s[2] + red_s[3]);
+        if (gtid == 0) {
+          float a = 0.f;
+#pragma unroll
+          for (int w = 0; w < NGW; ++w) a += red_s[w];
+          atomicAdd(dlogg + srow * topk + j, a);
+        }
         named_bar_softmax();
       }
     }
     mbar_wait(&bars[B_MD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
     flush_kv(nunits - 1);
-    // dQ (already scaled through dS)
+    // dQ (already scaled through dS): columns 64hc..64hc+63 of this row
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 2 * hc; c < 2 * hc + 2; ++c) {
       float qv[32];
       tc::tmem_ld32(tmem + C_DQ + lane_off + 32 * c, qv);
       tc::tmem_wait_ld();
@@ -340,7 +364,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }

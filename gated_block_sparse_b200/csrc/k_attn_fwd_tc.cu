@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = exp2f(z[2 * i] - muse), p1 = exp2f(z[2 * i + 1] - muse);
+        const float p0 = tc::ex2(z[2 * i] - muse), p1 = tc::ex2(z[2 * i + 1] - muse);
         rs += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
         // PV_{j-1} must be done: O is stable and the P buffer is free
         mbar_wait(&bars[B_OD], (j - 1) & 1, err);
         tc::fence_after_sync();
-        const float alpha = grow ? exp2f(m - muse) : 1.f;
+        const float alpha = grow ? tc::ex2(m - muse) : 1.f;
         if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {

@@ -26,8 +26,9 @@
 //   warps 0-7: gradient rows: warps w and w+4 share the TMEM lanes of rows
 //           32(w%4).. and split the 64 key columns, two warps per SM
 //           sub-partition to hide instruction latency
-// dK^T / dV^T are added to the fp32 accumulators through a shared-memory
-// transpose and 16-byte vector reductions.
+// dK^T / dV^T are added to the fp32 accumulators through a per-warp
+// shared-memory transpose and 16-byte vector reductions; no CTA-wide barrier
+// runs inside the unit loop.
 // 512 TMEM columns and about 193 KB of shared memory: one CTA per SM.
 #include <cuda.h>
 #include <math.h>
@@ -55,7 +56,8 @@ constexpr uint32_t OFF_KV = OFF_DO + TILE128;
 constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;
 constexpr uint32_t OFF_DS = OFF_P + PT_BYTES;
 constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [64 keys][128 d] transpose
-constexpr uint32_t OFF_BAR = OFF_T + 64 * D * 4;
+constexpr uint32_t OFF_DL = OFF_T + 64 * D * 4;      // fp32 [unit][warp] d(log g) partials
+constexpr uint32_t OFF_BAR = OFF_DL + 129 * 8 * 4 + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -92,7 +94,6 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   extern __shared__ __align__(1024) unsigned char sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
-  float* red_s = reinterpret_cast<float*>(sm + OFF_BAR + NBAR * 8 + 16);  // [NGW]
   uint32_t* err = &g_attn_bwd_tc_err;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = Hq / Hkv, pairs = G / 2;
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
       const int blk = unit_block(jj);
       const int nkeys = min(64, N - 64 * blk);
       const uint32_t cb = tmem + (jj & 1) * C_BUF + lane_off;
+      float* tw = tsm + warp * 1024;  // this warp's [32 keys][32 d] slice
 #pragma unroll 1
       for (int m2 = 0; m2 < 2; ++m2) {
         float* acc = m2 == 0 ? dk_acc : dv_acc;
@@ -259,20 +261,22 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         tc::tmem_ld32(cb + (m2 == 0 ? C_DKT : C_DVT) + 32 * hc, kv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) tsm[(32 * hc + i) * D + row] = kv[i];
-        named_bar_softmax();
-        float* dst = acc + kvbase + (size_t)(64 * blk) * D;
-#pragma unroll 4
-        for (int e = gtid; e < 64 * (D / 4); e += 2 * 128) {
-          const int key = e >> 5, d4 = (e & 31) << 2;
-          if (key < nkeys) {
-            const float4 x = *reinterpret_cast<const float4*>(tsm + key * D + d4);
+        for (int i = 0; i < 32; ++i) tw[i * 32 + lane] = kv[i];
+        __syncwarp();
+        float* dst = acc + kvbase + (size_t)(64 * blk + 32 * hc) * D + 32 * wq;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int e = lane + 32 * it;
+          const int key = e >> 3, d4 = (e & 7) << 2;
+          if (32 * hc + key < nkeys) {
+            const float4 x = *reinterpret_cast<const float4*>(tw + key * 32 + d4);
             tc::red_add_v4(dst + (size_t)key * D + d4, x.x, x.y, x.z, x.w);
           }
         }
-        named_bar_softmax();
+        __syncwarp();
       }
     };
+    float* dl_s = reinterpret_cast<float*>(sm + OFF_DL);
     for (int j = 0; j < nunits; ++j) {
       const bool cur = (j == kk);
       const float bias = cur ? 0.f : logg_row[j] * LOG2E;
@@ -325,22 +329,21 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[B_TE + ((j - 1) & 1)]);
       }
-      if (!cur) {  // d(log g) of this slot, in a fixed order
+      if (!cur) {  // this warp's part of d(log g) of the slot, summed at the end
         dsum = warp_sum(dsum);
-        if (lane == 0) red_s[warp] = dsum;
-        named_bar_softmax();
-        if (gtid == 0) {
-          float a = 0.f;
-#pragma unroll
-          for (int w = 0; w < NGW; ++w) a += red_s[w];
-          atomicAdd(dlogg + srow * topk + j, a);
-        }
-        named_bar_softmax();
+        if (lane == 0) dl_s[j * NGW + warp] = dsum;
       }
     }
     mbar_wait(&bars[B_MD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
     flush_kv(nunits - 1);
+    named_bar_softmax();
+    for (int j = gtid; j < kk; j += 2 * 128) {  // d(log g): fixed-order sum over the warps
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < NGW; ++w) a += dl_s[j * NGW + w];
+      atomicAdd(dlogg + srow * topk + j, a);
+    }
     // dQ (already scaled through dS): columns 64hc..64hc+63 of this row
 #pragma unroll 1
     for (int c = 2 * hc; c < 2 * hc + 2; ++c) {

@@ -73,7 +73,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 if verbose and log:
                     print(f"== {os.path.basename(futs[f])}\n{log}", file=sys.stderr)
     if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcuda"]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")

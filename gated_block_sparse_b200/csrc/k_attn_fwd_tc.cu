@@ -283,16 +283,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
 
 // ------------------------------------------------------------------ host
 static bool make_map(CUtensorMap* map, const void* base, int rows_per_plane, int planes) {
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows_per_plane, (cuuint64_t)planes};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows_per_plane * D * 2};
-  const cuuint32_t box[3] = {64, 64, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = cuTensorMapEncodeTiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                                      const_cast<void*>(base), dims, strides, box, estr,
-                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_tma_map_bf16_3d(map, base, D, rows_per_plane, planes);
 }
 
 bool attn_fwd_tc_supported(int bf16, int d, int Hq, int Hkv) {

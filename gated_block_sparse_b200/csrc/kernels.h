@@ -1,11 +1,17 @@
 // Host-side launchers of the SAS kernels (internal; the public ABI is sas.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace sas {
+
+// 3-D bf16 TMA tensor map over a row-major [planes][rows_per_plane][d] tensor
+// ({64, 64, 1} box, 128-byte swizzle, zero fill); false when encoding fails.
+bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int rows_per_plane,
+                          int planes);
 
 // Block summaries: ksum[b,h,m] = mean of keys 64m..64m+63.
 cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,

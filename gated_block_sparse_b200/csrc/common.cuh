@@ -149,6 +149,83 @@ __device__ inline int tree_merge(unsigned long long* A, int* Alen, unsigned long
   return which;
 }
 
+// Top-k of nl <= 32 descending lists of unique 64-bit keys (list l at
+// A[l << lg], len[l] <= 2^lg entries) into out[0 .. min(k, sum len) - 1],
+// descending. The pruning threshold is the largest k-th key among the lists
+// that hold k keys: a key below it has at least k keys above it. Keys at or
+// above it are compacted into tmp; when at most 512 survive, each survivor
+// counts the survivors above it, which is its global rank (every key above a
+// survivor is a survivor). Otherwise the lists are merged pairwise
+// (tree_merge over A and B, whose length arrays it overwrites). *cnt is 0 on
+// entry. All threads of the block call it; it ends with a barrier.
+__device__ inline void topk_of_lists(unsigned long long* A, int* len, int nl, int lg, int k,
+                                     unsigned long long* out, unsigned long long* tmp,
+                                     unsigned long long* B, int* Blen, int* cnt) {
+  const int kq = 1 << lg;
+  const int lane = threadIdx.x & 31;
+  unsigned long long th = 0;
+  {
+    unsigned long long v = 0;
+    if (lane < nl && k > 0 && len[lane] >= k) v = A[(lane << lg) + k - 1];
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, off);
+      v = w > v ? w : v;
+    }
+    th = v;
+  }
+  // A tighter bound when k <= 32: the k-th largest of the 32 keys made of each
+  // list's first 32/nl' entries (nl' = nl rounded up to a power of two) is
+  // also at most the k-th largest of all keys. Each lane counts the keys of
+  // that sample above its own.
+  if (k <= 32) {
+    int nlp = 1;
+    while (nlp < nl) nlp <<= 1;
+    const int m = 32 / nlp, l = lane / m, p = lane % m;
+    const unsigned long long mine = (l < nl && p < len[l]) ? A[(l << lg) + p] : 0ull;
+    int above = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, mine, j) > mine;
+    const unsigned hit = __ballot_sync(0xffffffffu, mine != 0ull && above == k - 1);
+    if (hit) {
+      const unsigned long long kth = __shfl_sync(0xffffffffu, mine, __ffs(hit) - 1);
+      th = kth > th ? kth : th;
+    }
+  }
+  const int total = nl << lg;
+  for (int e0 = 0; e0 < total; e0 += blockDim.x) {
+    const int e = e0 + (int)threadIdx.x;
+    bool keep = false;
+    unsigned long long key = 0;
+    if (e < total && (e & (kq - 1)) < len[e >> lg]) {
+      key = A[e];
+      keep = key >= th;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    int base = 0;
+    if (lane == 0 && m) base = atomicAdd(cnt, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (keep) tmp[base + __popc(m & ((1u << lane) - 1u))] = key;
+  }
+  __syncthreads();
+  const int S = *cnt;
+  if (S <= 512) {
+    for (int i = threadIdx.x; i < S; i += blockDim.x) {
+      const unsigned long long key = tmp[i];
+      int rank = 0;
+      for (int j = 0; j < S; ++j) rank += tmp[j] > key;
+      if (rank < k) out[rank] = key;
+    }
+    __syncthreads();
+    return;
+  }
+  const int which = tree_merge(A, len, B, Blen, nl, lg, k);
+  const unsigned long long* res = which ? B : A;
+  const int n0 = which ? Blen[0] : len[0];
+  for (int i = threadIdx.x; i < n0; i += blockDim.x) out[i] = res[i];
+  __syncthreads();
+}
+
 // log2 of the smallest power of two >= max(k, 1).
 __host__ __device__ inline int ceil_log2(int k) {
   int lg = 0;

@@ -8,27 +8,32 @@
 // o = softmax(q K_S^T + log g_S) V_S), section 2.4 (serving: GQA groups share
 // one block set); the 1/sqrt(d) logit scale from the reproduction note.
 //
-// Cluster of CS CTAs (16, or 8 when the batch has many rows). CTA c of the
-// cluster:
+// Cluster of CS CTAs (16 when the rows fit the GPU that way, else fewer).
+// CTA c of the cluster:
 //   1. bulk-copies its contiguous range of the row's block summaries through
-//      a two-slot shared-memory ring and scores them against qbar (mean of
+//      a three-slot shared-memory ring and scores them against qbar (mean of
 //      the group's query heads); the current block's K/V, known before any
 //      selection, is prefetched at the same time by the CTA that owns it;
-//   2. reduces its range to a best-first list of min(k, n) candidates (rank
-//      counting per warp, then a pairwise tree merge of the 8 warp lists) and
-//      the range's (max, sum exp), and stores list and sums into the stage
-//      slot of every CTA of the cluster (remote shared-memory stores);
-//   3. after a cluster barrier every CTA merges the CS staged lists the same
-//      way and holds the row's kept blocks (ascending) and the gate's LSE;
-//   4. bulk-copies the K/V blocks of its share of the units (the current
-//      block first, then kept blocks) through a two-slot ring that reuses
-//      the summary ring, keeping an online softmax state (m, l, acc) for
-//      every head of the group, and stores head h's state into CTA h;
-//   5. after a second cluster barrier CTA h < G combines head h from the CS
-//      states (exact LSE rescaling) in its own shared memory and writes o.
-// Data moves between CTAs only by stores made before a barrier, so every
-// read after it is local. No global scratch, atomics or memsets; every wait
-// is bounded.
+//   2. reduces its range to (max, sum exp) and a best-first list of
+//      min(k, n) candidates, and stores both into its slot of every CTA of
+//      the cluster with asynchronous remote stores that complete on the
+//      receiver's mbarrier;
+//   3. once all lists have landed, every CTA merges them identically (one
+//      level: each candidate counts the keys above it in the other lists)
+//      and holds the row's kept blocks (ascending) and the gate's LSE;
+//   4. streams the K/V blocks of its share of the units (the current block
+//      first, then kept blocks) through a ring that reuses the summary ring.
+//      Each warp takes 8 keys of every unit and keeps its own online-softmax
+//      state (m, l, acc) for every head of the group, so no CTA-wide barrier
+//      runs per unit;
+//   5. folds the warp states into one per head and stores head h's state
+//      into CTA h (remote stores on CTA h's mbarrier); CTA h < G combines the
+//      CS states (exact LSE rescaling) and writes o.
+// Data moves between CTAs only by remote stores that complete on the
+// receiver's mbarrier, so every read is local. A cluster barrier after the
+// barrier initialisation orders the first remote store, and one at exit
+// keeps every CTA resident until all stores into it are done. No global
+// scratch, atomics or memsets; every wait is bounded.
 #include <cooperative_groups.h>
 #include <float.h>
 
@@ -42,120 +47,162 @@ namespace sas {
 
 __device__ uint32_t g_decode_fused_err = 0;
 
+namespace {
+
 constexpr int FD_THREADS = 256;
 constexpr int FD_WARPS = FD_THREADS / 32;
-
-// Two adjacent elements as fp32.
-__device__ __forceinline__ void load2(const float* p, float2& v) {
-  v = *reinterpret_cast<const float2*>(p);
-}
-__device__ __forceinline__ void load2(const __nv_bfloat16* p, float2& v) {
-  v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-}
-
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
+constexpr int FD_NS = 3;      // summary ring slots
+constexpr int FD_SUBC = 32;   // summaries per ring slot
+constexpr int FD_MAXKV = 4;   // K/V ring slots at most
+constexpr unsigned FULL = 0xffffffffu;
 
 struct FdSmem {  // byte offsets into dynamic shared memory
-  size_t kv0, u1, q, qbar, sc, zs, wa, wb, wlen_a, wlen_b, sa, sb, slen_a, slen_b, smx, sse, kidx,
-      klogg, cm, cl, cacc, bars, total;
+  size_t u, q, qbar, sc, mine, slen, stage, sstat, fin, kidx, klogg, cst, cml, bars, total;
+  size_t wl, wb, tmp, mb, mblen;  // list scratch inside region u, after K/V slot 0
+  int nkv;                        // K/V ring slots held by region u
 };
 
 __host__ __device__ inline size_t fd_al(size_t x) { return (x + 127) & ~(size_t)127; }
 
-// kv0: K/V slot 0 (the current block is prefetched into it). u1: the summary
-// ring (2 x subc summaries) during the scan, K/V slot 1 afterwards.
-__host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int subc, int per, int k, int CS) {
+// Region u: K/V slot 0 followed by the summary ring during the scan, then by
+// the list scratch (warp lists, survivors, merge buffer) during selection;
+// K/V slots 0 .. nkv-1 afterwards; the per-warp states at the end.
+__host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int kq, int CS) {
   FdSmem L;
   const size_t kvslot = (size_t)2 * SAS_BLOCK * D * es;
-  const size_t ring = (size_t)2 * subc * D * 4;
-  const size_t kq = (size_t)1 << ceil_log2(k > 0 ? k : 1);  // list stride (power of two)
+  L.wl = kvslot;
+  L.wb = L.wl + (size_t)FD_WARPS * kq * 8;
+  L.tmp = L.wb + (size_t)FD_WARPS * kq * 8;
+  L.mb = L.tmp + (size_t)CS * kq * 8;
+  L.mblen = L.mb + (size_t)CS * kq * 8;
+  size_t ub = kvslot + (size_t)FD_NS * FD_SUBC * D * 4;
+  if (ub < L.mblen + 128) ub = L.mblen + 128;
+  if (ub < 2 * kvslot) ub = 2 * kvslot;
+  const size_t comb = (size_t)FD_WARPS * G * (D + 2) * 4;
+  if (ub < comb) ub = comb;
+  L.nkv = (int)(ub / kvslot);
+  if (L.nkv > FD_MAXKV) L.nkv = FD_MAXKV;
   size_t o = 0;
-  L.kv0 = o; o += fd_al(kvslot);
-  L.u1 = o; o += fd_al(kvslot > ring ? kvslot : ring);
+  L.u = o; o += fd_al(ub);
   L.q = o; o += fd_al((size_t)G * D * 4);
   L.qbar = o; o += fd_al((size_t)D * 4);
   L.sc = o; o += fd_al((size_t)(per > 0 ? per : 1) * 4);
-  L.zs = o; o += fd_al((size_t)G * SAS_BLOCK * 4);
-  L.wa = o; o += fd_al(FD_WARPS * kq * 8);
-  L.wb = o; o += fd_al(FD_WARPS * kq * 8);
-  L.wlen_a = o; o += fd_al(FD_WARPS * 4);
-  L.wlen_b = o; o += fd_al(FD_WARPS * 4);
-  L.sa = o; o += fd_al((size_t)CS * kq * 8);
-  L.sb = o; o += fd_al((size_t)CS * kq * 8);
-  L.slen_a = o; o += fd_al((size_t)CS * 4);
-  L.slen_b = o; o += fd_al((size_t)CS * 4);
-  L.smx = o; o += fd_al((size_t)CS * 4);
-  L.sse = o; o += fd_al((size_t)CS * 4);
-  L.kidx = o; o += fd_al(128 * 4);
-  L.klogg = o; o += fd_al(128 * 4);
-  L.cm = o; o += fd_al((size_t)CS * 4);
-  L.cl = o; o += fd_al((size_t)CS * 4);
-  L.cacc = o; o += fd_al((size_t)CS * D * 4);
-  L.bars = o; o += fd_al(4 * 8);
+  L.mine = o; o += fd_al((size_t)kq * 8);
+  L.slen = o; o += fd_al((size_t)CS * 4);
+  L.stage = o; o += fd_al((size_t)CS * kq * 8);
+  L.sstat = o; o += fd_al((size_t)CS * 8);
+  L.fin = o; o += fd_al((size_t)kq * 8);
+  L.kidx = o; o += fd_al((size_t)kq * 4);
+  L.klogg = o; o += fd_al((size_t)kq * 4);
+  L.cst = o; o += fd_al((size_t)CS * D * 4);
+  L.cml = o; o += fd_al((size_t)CS * 8);
+  L.bars = o; o += fd_al((size_t)(FD_NS + 2 * FD_MAXKV + 2) * 8);
   L.total = o;
   return L;
 }
+
+// N consecutive elements (N = 2 or 4) as fp32.
+template <int N>
+__device__ __forceinline__ void loadn(const __nv_bfloat16* p, float (&v)[N]) {
+  if constexpr (N == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    v[0] = a.x; v[1] = a.y;
+  }
+}
+template <int N>
+__device__ __forceinline__ void loadn(const float* p, float (&v)[N]) {
+  if constexpr (N == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  } else {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    v[0] = a.x; v[1] = a.y;
+  }
+}
+
+// (a0, a1) += (x0, x1) * (y0, y1) as one packed fp32x2 FMA (sm_100).
+__device__ __forceinline__ void fma2(float& a0, float& a1, float x0, float x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 a, x, y;\n\t"
+      "mov.b64 a, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "fma.rn.f32x2 a, x, y, a;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
+
+// Combines two (max, sum exp) pairs; an empty pair is (-FLT_MAX, 0).
+__device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  s = s * __expf(m - M) + s2 * __expf(m2 - M);
+  m = M;
+}
+
+}  // namespace
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
     const float* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
-    int gated, float scale, int subc, int per_max, T* __restrict__ o,
-    int32_t* __restrict__ idx_out) {
+    int gated, float scale, int per_max, T* __restrict__ o, int32_t* __restrict__ idx_out) {
   constexpr int TILE = SAS_BLOCK * D;
-  constexpr int PER = D / 32;
-  constexpr int VEC = Vec16<T>::N;
-  constexpr int NCH = D / (8 * VEC);
+  constexpr int VEC = Vec16<T>::N;     // elements per 16-byte vector
+  constexpr int NCHK = D / (4 * VEC);  // 16-byte chunks of a key row per lane (4 lanes per key)
+  constexpr int CPL = D / 32;          // output columns per lane
+  constexpr int PER = D / 32;          // summary elements per lane
   extern __shared__ __align__(128) unsigned char sm[];
   cg::cluster_group cluster = cg::this_cluster();
-  // Every CTA of the cluster must be running before anyone stores into its
-  // shared memory: arrive now, wait just before the first remote store.
-  cluster_arrive_relaxed();
   const int CS = (int)cluster.num_blocks();
   const int crank = (int)cluster.block_rank();
-  const FdSmem L = fd_layout(D, G, (int)sizeof(T), subc, per_max, topk, CS);
   const int lg = ceil_log2(topk > 0 ? topk : 1);
-  const int kq = 1 << lg;  // list stride
-  T* kv0 = reinterpret_cast<T*>(sm + L.kv0);
-  T* kv1 = reinterpret_cast<T*>(sm + L.u1);
-  float* sumbuf = reinterpret_cast<float*>(sm + L.u1);
+  const int kq = 1 << lg;  // list stride (power of two)
+  const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS);
+  unsigned char* U = sm + L.u;
+  const size_t kvslot = (size_t)2 * TILE * sizeof(T);
+  float* ring = reinterpret_cast<float*>(U + kvslot);
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qbar = reinterpret_cast<float*>(sm + L.qbar);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
-  float* zs = reinterpret_cast<float*>(sm + L.zs);
-  unsigned long long* wa = reinterpret_cast<unsigned long long*>(sm + L.wa);
-  unsigned long long* wb = reinterpret_cast<unsigned long long*>(sm + L.wb);
-  int* wlen_a = reinterpret_cast<int*>(sm + L.wlen_a);
-  int* wlen_b = reinterpret_cast<int*>(sm + L.wlen_b);
-  unsigned long long* sa = reinterpret_cast<unsigned long long*>(sm + L.sa);
-  unsigned long long* sb = reinterpret_cast<unsigned long long*>(sm + L.sb);
-  int* slen_a = reinterpret_cast<int*>(sm + L.slen_a);
-  int* slen_b = reinterpret_cast<int*>(sm + L.slen_b);
-  float* smx = reinterpret_cast<float*>(sm + L.smx);
-  float* sse = reinterpret_cast<float*>(sm + L.sse);
+  unsigned long long* wl = reinterpret_cast<unsigned long long*>(U + L.wl);
+  unsigned long long* wb = reinterpret_cast<unsigned long long*>(U + L.wb);
+  unsigned long long* tmp = reinterpret_cast<unsigned long long*>(U + L.tmp);
+  unsigned long long* mb = reinterpret_cast<unsigned long long*>(U + L.mb);
+  int* mblen = reinterpret_cast<int*>(U + L.mblen);
+  unsigned long long* mine = reinterpret_cast<unsigned long long*>(sm + L.mine);
+  int* slen = reinterpret_cast<int*>(sm + L.slen);
+  unsigned long long* stage = reinterpret_cast<unsigned long long*>(sm + L.stage);
+  float* sstat = reinterpret_cast<float*>(sm + L.sstat);
+  unsigned long long* fin = reinterpret_cast<unsigned long long*>(sm + L.fin);
   int* kidx = reinterpret_cast<int*>(sm + L.kidx);
   float* klogg = reinterpret_cast<float*>(sm + L.klogg);
-  float* cm = reinterpret_cast<float*>(sm + L.cm);
-  float* cl = reinterpret_cast<float*>(sm + L.cl);
-  float* cacc = reinterpret_cast<float*>(sm + L.cacc);
+  float* cst = reinterpret_cast<float*>(sm + L.cst);
+  float* cml = reinterpret_cast<float*>(sm + L.cml);
   uint64_t* sum_bar = reinterpret_cast<uint64_t*>(sm + L.bars);
-  uint64_t* kv_bar = sum_bar + 2;
-  __shared__ float red[FD_WARPS];
-  __shared__ float alpha_s[G], m_run[G], l_run[G];
-  __shared__ float loc_mx, loc_se;
-  __shared__ int ok_s;
+  uint64_t* full = sum_bar + FD_NS;
+  uint64_t* empty = full + FD_MAXKV;
+  uint64_t* list_bar = empty + FD_MAXKV;
+  uint64_t* state_bar = list_bar + 1;
+  __shared__ float wred_m[FD_WARPS], wred_s[FD_WARPS];
+  __shared__ int wlen[FD_WARPS], wlen_b[FD_WARPS];
+  __shared__ int surv_cnt;
 
   const int r = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * G;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // the group's queries and the sequence length first: both loads in flight together
+  constexpr int QPT = (G * D + FD_THREADS - 1) / FD_THREADS;
+  float qreg[QPT];
+#pragma unroll
+  for (int j = 0; j < QPT; ++j) {
+    const int i = tid + j * FD_THREADS;
+    qreg[j] = i < G * D ? to_f(q[((size_t)b * Hq + r * G) * D + i]) : 0.f;
+  }
   const size_t row = (size_t)b * Hkv + r;
   const int nblk = Lmax / SAS_BLOCK;
   const int n = min(max(lens[b], 1), Lmax);
@@ -169,35 +216,53 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int upc = (units + CS - 1) / CS;  // units attended by each CTA
   const int u0 = min(units, crank * upc), u1 = min(units, u0 + upc), nu = u1 - u0;
   const bool own_cur = (kk >= u0 && kk < u1);
-  const int nsub = (nmine + subc - 1) / subc;
+  const int nsub = (nmine + FD_SUBC - 1) / FD_SUBC;
+  const int NKV = L.nkv;
   const size_t kvrow = row * (size_t)Lmax * D;
   const float* ks_row = ksum + row * (size_t)nblk * D;
   uint32_t* err = &g_decode_fused_err;
 
-  if (tid == 0) {
-    mbar_init(&sum_bar[0], 1);
-    mbar_init(&sum_bar[1], 1);
-    mbar_init(&kv_bar[0], 1);
-    mbar_init(&kv_bar[1], 1);
-    fence_mbar_init();
-    ok_s = 1;
+  // ---- 0. barriers, expected remote bytes, first copies, q and qbar
+  if (tid < CS) {
+    const int nm = min(C, (tid + 1) * per) - min(C, tid * per);
+    slen[tid] = topk > 0 ? min(topk, nm) : 0;
   }
-  __syncthreads();
   if (tid == 0) {
-    for (int i = 0; i < min(2, nsub); ++i) {
-      const int cnt_i = min(subc, nmine - i * subc);
+    for (int i = 0; i < FD_NS; ++i) mbar_init(&sum_bar[i], 1);
+    for (int i = 0; i < FD_MAXKV; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], FD_WARPS);
+    }
+    mbar_init(list_bar, 1);
+    mbar_init(state_bar, 1);
+    fence_mbar_init();
+    surv_cnt = 0;
+    uint32_t lb = 0;  // every CTA's list and (max, sum exp)
+    for (int c = 0; c < CS; ++c) {
+      const int nm = min(C, (c + 1) * per) - min(C, c * per);
+      lb += 8u * (uint32_t)(topk > 0 ? min(topk, nm) : 0) + 8u;
+    }
+    mbar_arrive_expect_tx(list_bar, lb);
+    if (crank < G) mbar_arrive_expect_tx(state_bar, (uint32_t)CS * (D * 4 + 8));
+    for (int i = 0; i < min(FD_NS, nsub); ++i) {
+      const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
       mbar_arrive_expect_tx(&sum_bar[i], (uint32_t)(cnt_i * D * 4));
-      bulk_g2s(sumbuf + (size_t)i * subc * D, ks_row + (size_t)(m0 + i * subc) * D,
+      bulk_g2s(ring + (size_t)i * FD_SUBC * D, ks_row + (size_t)(m0 + i * FD_SUBC) * D,
                (uint32_t)(cnt_i * D * 4), &sum_bar[i]);
     }
     if (own_cur) {  // the current block is unit 0 of this CTA's order, slot 0
-      mbar_arrive_expect_tx(&kv_bar[0], (uint32_t)(2 * TILE * sizeof(T)));
-      bulk_g2s(kv0, kc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &kv_bar[0]);
-      bulk_g2s(kv0 + TILE, vc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &kv_bar[0]);
+      mbar_arrive_expect_tx(&full[0], (uint32_t)(2 * TILE * sizeof(T)));
+      bulk_g2s(U, kc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &full[0]);
+      bulk_g2s(U + TILE * sizeof(T), vc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &full[0]);
     }
   }
-  for (int i = tid; i < G * D; i += FD_THREADS) q_s[i] = to_f(q[((size_t)b * Hq + r * G) * D + i]);
+#pragma unroll
+  for (int j = 0; j < QPT; ++j) {
+    const int i = tid + j * FD_THREADS;
+    if (i < G * D) q_s[i] = qreg[j];
+  }
   __syncthreads();
+  cluster_arrive_release();  // barriers are initialised: other CTAs may store into this one
   for (int i = tid; i < D; i += FD_THREADS) {
     float a = 0.f;
 #pragma unroll
@@ -212,10 +277,10 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
 #pragma unroll
     for (int i = 0; i < PER; ++i) qv[i] = qbar[lane * PER + i];
     for (int i = 0; i < nsub; ++i) {
-      const int slot = i & 1;
-      const int cnt_i = min(subc, nmine - i * subc);
-      if (!mbar_wait(&sum_bar[slot], (uint32_t)((i >> 1) & 1), err)) ok_s = 0;
-      const float* sb = sumbuf + (size_t)slot * subc * D;
+      const int slot = i % FD_NS;
+      const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
+      mbar_wait(&sum_bar[slot], (uint32_t)((i / FD_NS) & 1), err);
+      const float* sb = ring + (size_t)slot * FD_SUBC * D;
       for (int j0 = wid; j0 < cnt_i; j0 += 4 * FD_WARPS) {
         float part[4];
 #pragma unroll
@@ -223,9 +288,10 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
           const int j = j0 + u * FD_WARPS;
           float a = 0.f;
           if (j < cnt_i) {
-            const float* p = sb + (size_t)j * D + lane * PER;
+            float x[PER];
+            loadn<PER>(sb + (size_t)j * D + lane * PER, x);
 #pragma unroll
-            for (int e = 0; e < PER; ++e) a += p[e] * qv[e];
+            for (int e = 0; e < PER; ++e) a += x[e] * qv[e];
           }
           part[u] = a;
         }
@@ -235,45 +301,38 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int j = j0 + u * FD_WARPS;
-            if (j < cnt_i) sc[i * subc + j] = part[u] * scale + 0.0f;
+            if (j < cnt_i) sc[i * FD_SUBC + j] = part[u] * scale + 0.0f;
           }
         }
       }
       __syncthreads();  // slot consumed
-      if (tid == 0 && i + 2 < nsub) {
-        const int cnt_n = min(subc, nmine - (i + 2) * subc);
+      if (tid == 0 && i + FD_NS < nsub) {
+        const int cnt_n = min(FD_SUBC, nmine - (i + FD_NS) * FD_SUBC);
         mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt_n * D * 4));
-        bulk_g2s(sumbuf + (size_t)slot * subc * D, ks_row + (size_t)(m0 + (i + 2) * subc) * D,
+        bulk_g2s(ring + (size_t)slot * FD_SUBC * D, ks_row + (size_t)(m0 + (i + FD_NS) * FD_SUBC) * D,
                  (uint32_t)(cnt_n * D * 4), &sum_bar[slot]);
       }
     }
   }
+
   // ---- 2. this range's (max, sum exp) and best-first list
   {
-    float mx = -FLT_MAX;
-    for (int j = tid; j < nmine; j += FD_THREADS) mx = fmaxf(mx, sc[j]);
-    mx = warp_max(mx);
-    if (lane == 0) red[wid] = mx;
-    __syncthreads();
-    mx = -FLT_MAX;
-    for (int i = 0; i < FD_WARPS; ++i) mx = fmaxf(mx, red[i]);
-    __syncthreads();
-    float se = 0.f;
-    for (int j = tid; j < nmine; j += FD_THREADS) se += __expf(sc[j] - mx);
-    se = warp_sum(se);
-    if (lane == 0) red[wid] = se;
-    __syncthreads();
-    if (tid == 0) {
-      float a = 0.f;
-      for (int i = 0; i < FD_WARPS; ++i) a += red[i];
-      loc_mx = mx;
-      loc_se = a;
+    float lm = -FLT_MAX, ls = 0.f;
+    for (int j = tid; j < nmine; j += FD_THREADS) ms_merge(lm, ls, sc[j], 1.f);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const float m2 = __shfl_xor_sync(FULL, lm, off), s2 = __shfl_xor_sync(FULL, ls, off);
+      ms_merge(lm, ls, m2, s2);
+    }
+    if (lane == 0) {
+      wred_m[wid] = lm;
+      wred_s[wid] = ls;
     }
   }
-  int wsel = 0;  // which warp-list buffer holds this CTA's merged list (list 0)
-  if (topk > 0 && nmine <= FD_THREADS) {
-    // small range: one rank-counting pass over the whole range, one item per
-    // thread (broadcast shared-memory reads), straight into list 0 of A
+  const int my_len = topk > 0 ? min(topk, nmine) : 0;
+  const unsigned long long* mylist = mine;
+  if (topk > 0 && nmine <= 64) {
+    // small range: one rank-counting pass over the whole range
     if (tid < nmine) {
       const float sj = sc[tid];
       int rk = 0;
@@ -281,11 +340,10 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         const float sx = sc[x];
         rk += (sx > sj) || (sx == sj && x < tid);
       }
-      if (rk < topk) wa[rk] = cand_key(sj, m0 + tid);
+      if (rk < topk) mine[rk] = cand_key(sj, m0 + tid);
     }
-    if (tid == 0) wlen_a[0] = min(topk, nmine);
   } else if (topk > 0) {
-    // each warp ranks its contiguous share of the range
+    // each warp ranks its contiguous share, then one merge of the 8 lists
     const int pw = (nmine + FD_WARPS - 1) / FD_WARPS;
     const int a0 = min(nmine, wid * pw), a1 = min(nmine, a0 + pw);
     for (int j = a0 + lane; j < a1; j += 32) {
@@ -295,53 +353,54 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         const float sx = sc[x];
         rk += (sx > sj) || (sx == sj && x < j);
       }
-      if (rk < topk) wa[wid * kq + rk] = cand_key(sj, m0 + j);
+      if (rk < topk) wl[wid * kq + rk] = cand_key(sj, m0 + j);
     }
-    if (lane == 0) wlen_a[wid] = min(topk, a1 - a0);
+    if (lane == 0) wlen[wid] = min(topk, a1 - a0);
     __syncthreads();
-    wsel = tree_merge(wa, wlen_a, wb, wlen_b, FD_WARPS, lg, topk);
+    mylist = tree_merge(wl, wlen, wb, wlen_b, FD_WARPS, lg, topk) ? wb : wl;
   }
   __syncthreads();
-  // ---- push this CTA's list and partial sums into every CTA's stage slot
-  cluster_wait_acquire();  // every CTA of the cluster is running
+
+  // ---- push this CTA's list and (max, sum exp) into its slot of every CTA
+  cluster_wait_acquire();  // every CTA of the cluster has initialised its barriers
   {
-    const unsigned long long* mine = wsel ? wb : wa;
-    const int my_len = topk > 0 ? (wsel ? wlen_b[0] : wlen_a[0]) : 0;
+    const uint32_t lst = smem_u32(stage) + (uint32_t)(crank * kq * 8);
+    const uint32_t sst = smem_u32(sstat) + (uint32_t)(crank * 8);
+    const uint32_t lbar = smem_u32(list_bar);
     for (int e = tid; e < CS * (my_len + 1); e += FD_THREADS) {
       const int c = e / (my_len + 1), p = e - c * (my_len + 1);
       if (p < my_len) {
-        *cluster.map_shared_rank(sa + crank * kq + p, c) = mine[p];
+        st_async_u64(mapa(lst + 8u * p, c), mylist[p], mapa(lbar, c));
       } else {
-        *cluster.map_shared_rank(slen_a + crank, c) = my_len;
-        *cluster.map_shared_rank(smx + crank, c) = loc_mx;
-        *cluster.map_shared_rank(sse + crank, c) = loc_se;
+        float M = -FLT_MAX, S = 0.f;
+        for (int w = 0; w < FD_WARPS; ++w) ms_merge(M, S, wred_m[w], wred_s[w]);
+        st_async_f32x2(mapa(sst, c), M, S, mapa(lbar, c));
       }
     }
   }
-  cluster_arrive_release();
-  cluster_wait_acquire();  // all lists are in this CTA's shared memory
 
   // ---- 3. merge the CS lists (every CTA, identically) and the LSE
+  mbar_wait_cluster(list_bar, 0, err);
   float lse;
-  {
-    float M = -FLT_MAX;
-    for (int c = 0; c < CS; ++c) M = fmaxf(M, smx[c]);
-    float S = 0.f;
-    for (int c = 0; c < CS; ++c)
-      if (sse[c] > 0.f) S += sse[c] * __expf(smx[c] - M);
+  {  // every warp computes the same value
+    const float mx = lane < CS ? sstat[2 * lane] : -FLT_MAX;
+    const float se = lane < CS ? sstat[2 * lane + 1] : 0.f;
+    const float M = warp_max(mx);
+    const float S = warp_sum(se > 0.f ? se * __expf(mx - M) : 0.f);
     lse = (C > 0) ? M + __logf(S) : 0.f;
   }
   if (topk > 0) {
-    const int ssel = tree_merge(sa, slen_a, sb, slen_b, CS, lg, topk);
-    const unsigned long long* fk = ssel ? sb : sa;
-    for (int i = tid; i < kk; i += FD_THREADS) {  // ascending block order
-      const int mi = key_block(fk[i]);
-      int pos = 0;
-      for (int j = 0; j < kk; ++j) pos += key_block(fk[j]) < mi;
-      kidx[pos] = mi;
-      klogg[pos] = key_score(fk[i]) - lse;
+    if (kk > 0) {
+      topk_of_lists(stage, slen, CS, lg, topk, fin, tmp, mb, mblen, &surv_cnt);
+      for (int i = tid; i < kk; i += FD_THREADS) {  // ascending block order
+        const int mi = key_block(fin[i]);
+        int pos = 0;
+        for (int j = 0; j < kk; ++j) pos += key_block(fin[j]) < mi;
+        kidx[pos] = mi;
+        klogg[pos] = key_score(fin[i]) - lse;
+      }
+      __syncthreads();
     }
-    __syncthreads();
     if (crank == 0 && idx_out != nullptr)
       for (int i = tid; i < topk; i += FD_THREADS) idx_out[row * topk + i] = i < kk ? kidx[i] : -1;
   }
@@ -359,182 +418,213 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       atomicOr(err, kErrBadIndex);
       blk = t;
     }
-    const int slot = i & 1;
-    T* kdst = slot ? kv1 : kv0;
-    mbar_arrive_expect_tx(&kv_bar[slot], (uint32_t)(2 * TILE * sizeof(T)));
-    bulk_g2s(kdst, kc + kvrow + (size_t)blk * TILE, TILE * sizeof(T), &kv_bar[slot]);
-    bulk_g2s(kdst + TILE, vc + kvrow + (size_t)blk * TILE, TILE * sizeof(T), &kv_bar[slot]);
+    const int slot = i % NKV;
+    unsigned char* dst = U + (size_t)slot * kvslot;
+    mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * TILE * sizeof(T)));
+    bulk_g2s(dst, kc + kvrow + (size_t)blk * TILE, TILE * sizeof(T), &full[slot]);
+    bulk_g2s(dst + TILE * sizeof(T), vc + kvrow + (size_t)blk * TILE, TILE * sizeof(T),
+             &full[slot]);
   };
   if (tid == 0)
-    for (int i = own_cur ? 1 : 0; i < min(2, nu); ++i) issue_unit(i);
-  if (tid < G) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
-  }
-  constexpr int NITEM = (G * D / 2 + FD_THREADS - 1) / FD_THREADS;
-  float acc[NITEM][2];
+    for (int i = own_cur ? 1 : 0; i < min(NKV, nu); ++i) issue_unit(i);
+  float m_w[G], l_w[G], acc[G][CPL];
 #pragma unroll
-  for (int it = 0; it < NITEM; ++it) acc[it][0] = acc[it][1] = 0.f;
-  const int jq = lane >> 3, pp = lane & 7;
+  for (int h = 0; h < G; ++h) {
+    m_w[h] = -INFINITY;
+    l_w[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+  }
+  const int key = wid * 8 + (lane >> 2);  // this lane's key of the unit (4 lanes per key)
+  const int qq = lane & 3;                // and its quarter of each 16-byte chunk group
   for (int i = 0; i < nu; ++i) {
-    const int slot = i & 1;
+    const int slot = i % NKV;
     const int u = unit_of(i);
     const bool cur = (u == kk);
     const float bias = (!cur && gated) ? klogg[u] : 0.f;
-    if (!mbar_wait(&kv_bar[slot], (uint32_t)((i >> 1) & 1), err)) ok_s = 0;
-    const T* kt = slot ? kv1 : kv0;
+    mbar_wait(&full[slot], (uint32_t)((i / NKV) & 1), err);
+    const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot);
     const T* vt = kt + TILE;
-    for (int j0 = wid * 4; j0 < SAS_BLOCK; j0 += 4 * FD_WARPS) {
-      const int j = j0 + jq;
-      float kv[NCH * VEC];
+    float dot[G], dot1[G];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c)
-        Vec16<T>::load(kt + (size_t)j * D + c * 8 * VEC + pp * VEC, kv + c * VEC);
-      float dot[G];
+    for (int h = 0; h < G; ++h) dot[h] = dot1[h] = 0.f;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float a = 0.f;
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          const float* qp = q_s + h * D + c * 8 * VEC + pp * VEC;
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) a += kv[c * VEC + e] * qp[e];
-        }
-        dot[h] = a;
-      }
+    for (int c = 0; c < NCHK; ++c) {
+      const int d0 = c * 4 * VEC + qq * VEC;
+      float kv[VEC];
+      Vec16<T>::load(kt + (size_t)key * D + d0, kv);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 1);
-        dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 2);
-        dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 4);
-      }
-      if (pp == 0) {
-        const bool masked = cur && j >= ncur;
 #pragma unroll
-        for (int h = 0; h < G; ++h) zs[h * SAS_BLOCK + j] = masked ? -INFINITY : dot[h] * scale + bias;
-      }
-    }
-    __syncthreads();
-    for (int h = wid; h < G; h += FD_WARPS) {  // online softmax state per head
-      float* z = zs + h * SAS_BLOCK;
-      const float mx = warp_max(fmaxf(z[lane], z[lane + 32]));
-      const float mold = m_run[h];
-      const float mnew = fmaxf(mold, mx);
-      const float e0 = __expf(z[lane] - mnew), e1 = __expf(z[lane + 32] - mnew);
-      z[lane] = e0;
-      z[lane + 32] = e1;
-      const float sum = warp_sum(e0 + e1);
-      if (lane == 0) {
-        const float al = __expf(mold - mnew);
-        alpha_s[h] = al;
-        l_run[h] = l_run[h] * al + sum;
-        m_run[h] = mnew;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int it = 0; it < NITEM; ++it) {
-      const int pi = tid + it * FD_THREADS;
-      if (pi < G * D / 2) {
-        const int h = pi / (D / 2), c = (pi % (D / 2)) * 2;
-        const float* z = zs + h * SAS_BLOCK;
-        const float al = alpha_s[h];
-        float a0 = acc[it][0] * al, a1 = acc[it][1] * al;
-        float b0 = 0.f, b1 = 0.f;  // two independent chains per column
-#pragma unroll 8
-        for (int j = 0; j < SAS_BLOCK; j += 2) {
-          float2 v0, v1;
-          load2(vt + (size_t)j * D + c, v0);
-          load2(vt + (size_t)(j + 1) * D + c, v1);
-          a0 += z[j] * v0.x;
-          a1 += z[j] * v0.y;
-          b0 += z[j + 1] * v1.x;
-          b1 += z[j + 1] * v1.y;
+        for (int e = 0; e < VEC; e += 4) {
+          const float4 qv = *reinterpret_cast<const float4*>(q_s + h * D + d0 + e);
+          fma2(dot[h], dot1[h], kv[e], kv[e + 1], qv.x, qv.y);
+          fma2(dot[h], dot1[h], kv[e + 2], kv[e + 3], qv.z, qv.w);
         }
-        acc[it][0] = a0 + b0;
-        acc[it][1] = a1 + b1;
       }
     }
-    __syncthreads();  // slot and zs consumed
-    if (tid == 0 && i + 2 < nu) issue_unit(i + 2);
-  }
-  // ---- push this CTA's partial state of head h into CTA h's combine slot
 #pragma unroll
-  for (int it = 0; it < NITEM; ++it) {
-    const int pi = tid + it * FD_THREADS;
-    if (pi < G * D / 2) {
-      const int h = pi / (D / 2), c = (pi % (D / 2)) * 2;
-      float* dst = cluster.map_shared_rank(cacc + crank * D + c, h);
-      dst[0] = acc[it][0];
-      dst[1] = acc[it][1];
+    for (int h = 0; h < G; ++h) dot[h] += dot1[h];
+    float p[G], alpha[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float z = dot[h] + __shfl_xor_sync(FULL, dot[h], 1);
+      z += __shfl_xor_sync(FULL, z, 2);
+      z = (cur && key >= ncur) ? -INFINITY : z * scale + bias;
+      float zm = fmaxf(z, __shfl_xor_sync(FULL, z, 4));
+      zm = fmaxf(zm, __shfl_xor_sync(FULL, zm, 8));
+      zm = fmaxf(zm, __shfl_xor_sync(FULL, zm, 16));
+      const float mn = fmaxf(m_w[h], zm);
+      if (mn == -INFINITY) {  // every key seen so far is masked
+        p[h] = 0.f;
+        alpha[h] = 1.f;
+      } else {
+        p[h] = __expf(z - mn);
+        alpha[h] = __expf(m_w[h] - mn);
+      }
+      float ps = p[h] + __shfl_xor_sync(FULL, p[h], 4);
+      ps += __shfl_xor_sync(FULL, ps, 8);
+      ps += __shfl_xor_sync(FULL, ps, 16);
+      l_w[h] = l_w[h] * alpha[h] + ps;
+      m_w[h] = mn;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[h][c] *= alpha[h];
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys: p from the key's lanes
+      float v[CPL];
+      loadn<CPL>(vt + (size_t)(wid * 8 + k8) * D + lane * CPL, v);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pk = __shfl_sync(FULL, p[h], k8 * 4);
+#pragma unroll
+        for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk, pk, v[c], v[c + 1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
+      mbar_wait(&empty[slot], (uint32_t)((i / NKV) & 1), err);
+      issue_unit(i + NKV);
     }
   }
-  if (tid < G) {
-    *cluster.map_shared_rank(cm + crank, tid) = m_run[tid];
-    *cluster.map_shared_rank(cl + crank, tid) = l_run[tid];
-  }
-  if (tid == 0 && ok_s == 0) atomicOr(err, kErrWaitTimeout);
-  cluster_arrive_release();
-  cluster_wait_acquire();  // every partial state has arrived; no remote access follows
 
-  // ---- 5. CTA h < G combines head h (exact LSE rescaling)
+  // ---- 5. fold the warp states per head; push head h's state into CTA h
+  __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
+  float* wst = reinterpret_cast<float*>(U);  // [warp][head][D + 2]: acc, m, l
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float* w = wst + (size_t)(wid * G + h) * (D + 2);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) w[lane * CPL + c] = acc[h][c];
+    if (lane == 0) {
+      w[D] = m_w[h];
+      w[D + 1] = l_w[h];
+    }
+  }
+  __syncthreads();
+  {
+    const uint32_t cst_r = smem_u32(cst) + (uint32_t)(crank * D * 4);
+    const uint32_t cml_r = smem_u32(cml) + (uint32_t)(crank * 8);
+    const uint32_t sbar = smem_u32(state_bar);
+    for (int e = tid; e < G * (D / 4); e += FD_THREADS) {
+      const int h = e / (D / 4), c4 = (e % (D / 4)) * 4;
+      float M = -INFINITY;
+      for (int w = 0; w < FD_WARPS; ++w) {
+        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
+        if (ws[D + 1] > 0.f) M = fmaxf(M, ws[D]);
+      }
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, Ls = 0.f;
+      for (int w = 0; w < FD_WARPS; ++w) {
+        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
+        if (ws[D + 1] > 0.f) {
+          const float f = __expf(ws[D] - M);
+          Ls += ws[D + 1] * f;
+          a0 += ws[c4] * f;
+          a1 += ws[c4 + 1] * f;
+          a2 += ws[c4 + 2] * f;
+          a3 += ws[c4 + 3] * f;
+        }
+      }
+      st_async_f32x4(mapa(cst_r + 4u * c4, h), a0, a1, a2, a3, mapa(sbar, h));
+      if (c4 == 0) st_async_f32x2(mapa(cml_r, h), M, Ls, mapa(sbar, h));
+    }
+  }
+  cluster_arrive_release();
+
+  // ---- 6. CTA h < G combines head h (exact LSE rescaling)
   if (crank < G) {
+    mbar_wait_cluster(state_bar, 0, err);
     const int h = crank;
-    float M = -FLT_MAX;
-    for (int c = 0; c < CS; ++c) M = fmaxf(M, cm[c]);
-    float Lsum = 0.f;
+    float M = -INFINITY;
     for (int c = 0; c < CS; ++c)
-      if (cl[c] > 0.f) Lsum += cl[c] * __expf(cm[c] - M);
-    const float inv = 1.f / Lsum;
+      if (cml[2 * c + 1] > 0.f) M = fmaxf(M, cml[2 * c]);
+    float Ls = 0.f;
+    for (int c = 0; c < CS; ++c)
+      if (cml[2 * c + 1] > 0.f) Ls += cml[2 * c + 1] * __expf(cml[2 * c] - M);
+    const float inv = 1.f / Ls;
     for (int col = tid; col < D; col += FD_THREADS) {
       float a = 0.f;
       for (int c = 0; c < CS; ++c)
-        if (cl[c] > 0.f) a += cacc[c * D + col] * __expf(cm[c] - M);
+        if (cml[2 * c + 1] > 0.f) a += cst[c * D + col] * __expf(cml[2 * c] - M);
       o[((size_t)b * Hq + r * G + h) * D + col] = from_f<T>(a * inv);
     }
   }
+  cluster_wait_acquire();  // no CTA leaves while stores into it may be pending
 }
 
 // ------------------------------------------------------------------ host
-struct FdPlan {
-  int CS, subc, per_max;
-  size_t smem;
+namespace {
+
+struct FdPick {
+  int dev, rows, nblk, kq, CS;
 };
 
-static FdPlan fd_plan(int B, int Hkv, int Lmax, int d, int G, int es, int topk, int CS) {
-  FdPlan p;
-  p.CS = CS;
-  p.subc = 32;  // 2 x 32 summaries in flight per CTA; aliased with K/V slot 1
-  const int nblk = Lmax / SAS_BLOCK;
-  p.per_max = (nblk + CS - 1) / CS;
-  p.smem = fd_layout(d, G, es, p.subc, p.per_max, topk, CS).total;
-  (void)B; (void)Hkv;
-  return p;
-}
-
+// Cluster size for a shape: the largest of 16, 8, 4, 2, 1 (and >= G, since
+// CTA h combines head h) whose clusters of all rows are co-resident on the
+// GPU; if none is, the largest that launches. Cached per shape, so repeated
+// launches make no occupancy queries.
 template <typename T, int D, int G>
-static cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const float* ksum,
-                                  int B, int Hkv, int Lmax, const int32_t* lens, int topk,
-                                  int gated, float scale, void* o, int32_t* idx_out,
-                                  cudaStream_t st) {
-  auto kern = k_decode_fused<T, D, G>;
+cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
+  static std::mutex mu;
+  static FdPick cache[32];
+  static int ncache = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   const int rows = B * Hkv;
-  // 16-CTA clusters while the rows fill the GPU with them; 8 otherwise.
-  int CS = rows <= 9 ? 16 : 8;
-  for (;;) {
-    FdPlan p = fd_plan(B, Hkv, Lmax, D, G, (int)sizeof(T), topk, CS);
-    if (p.smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-    cudaError_t e = ensure_smem(kern, p.smem);
-    if (e != cudaSuccess) return e;
-    if (CS > 8) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) { cudaGetLastError(); CS = 8; continue; }
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < ncache; ++i)
+      if (cache[i].dev == dev && cache[i].rows == rows && cache[i].nblk == nblk &&
+          cache[i].kq == kq) {
+        CS_out = cache[i].CS;
+        return cudaSuccess;
+      }
+  }
+  auto kern = k_decode_fused<T, D, G>;
+  int best = 0, first = 0;
+  const int cands[5] = {16, 8, 4, 2, 1};
+  for (int ci = 0; ci < 5; ++ci) {
+    const int CS = cands[ci];
+    if (CS < G) break;
+    const size_t smem = fd_layout(D, G, (int)sizeof(T), (nblk + CS - 1) / CS, kq, CS).total;
+    if (smem > 227 * 1024) continue;
+    if (ensure_smem(kern, smem) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    if (CS > 8 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CS, Hkv, B);
     cfg.blockDim = dim3(FD_THREADS);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = st;
+    cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CS;
@@ -542,24 +632,60 @@ static cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int nclusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
-    if (e != cudaSuccess || nclusters < 1) {
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
       cudaGetLastError();
-      if (CS > 8) { CS = 8; continue; }
-      return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+      continue;
     }
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
-                              static_cast<const T*>(vc), ksum, Hkv, Lmax, lens, topk, gated,
-                              scale, p.subc, p.per_max, static_cast<T*>(o), idx_out);
+    if (ncl < 1) continue;
+    if (!first) first = CS;
+    if (ncl >= rows) {
+      best = CS;
+      break;
+    }
   }
+  CS_out = best ? best : first;
+  if (!CS_out) return cudaErrorInvalidConfiguration;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ncache < 32) cache[ncache++] = FdPick{dev, rows, nblk, kq, CS_out};
+  return cudaSuccess;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const float* ksum, int B,
+                           int Hkv, int Lmax, const int32_t* lens, int topk, int gated, float scale,
+                           void* o, int32_t* idx_out, cudaStream_t st) {
+  auto kern = k_decode_fused<T, D, G>;
+  const int nblk = Lmax / SAS_BLOCK;
+  const int kq = 1 << ceil_log2(topk > 0 ? topk : 1);
+  int CS = 0;
+  cudaError_t e = pick_cluster<T, D, G>(B, Hkv, nblk, kq, CS);
+  if (e != cudaSuccess) return e;
+  const int per_max = (nblk + CS - 1) / CS;
+  const size_t smem = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS).total;
+  e = ensure_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, Hkv, B);
+  cfg.blockDim = dim3(FD_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
+                            static_cast<const T*>(vc), ksum, Hkv, Lmax, lens, topk, gated, scale,
+                            per_max, static_cast<T*>(o), idx_out);
 }
 
 template <typename T, int D>
-static cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc,
-                                  const float* ksum, int B, int Hkv, int Lmax, const int32_t* lens,
-                                  int topk, int gated, float scale, void* o, int32_t* idx_out,
-                                  cudaStream_t st) {
+cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc, const float* ksum,
+                           int B, int Hkv, int Lmax, const int32_t* lens, int topk, int gated,
+                           float scale, void* o, int32_t* idx_out, cudaStream_t st) {
 #define SAS_FD(GG)                                                                              \
   return launch_fused_t<T, D, GG>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale, o, \
                                   idx_out, st)
@@ -572,6 +698,8 @@ static cudaError_t launch_fused_g(int G, const void* q, const void* kc, const vo
   }
 #undef SAS_FD
 }
+
+}  // namespace
 
 cudaError_t launch_decode_fused(const void* q, const void* kc, const void* vc, int bf16, int B,
                                 int Hq, int Hkv, int Lmax, int d, const int32_t* lens,

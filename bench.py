@@ -43,7 +43,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn decode GB/s vs HBM peak; prefill fwd+bwd TFLOP/s vs bf16 peak"
-DEFAULT_STEPS = {"c1": 200, "c2": 100000, "c3": 10, "c4": 4000, "c5": 20000}
+DEFAULT_STEPS = {"c1": 200, "c2": 100000, "c3": 200, "c4": 4000, "c5": 20000}
 DEFAULT_WARMUP = {"c1": 10, "c2": 1000, "c3": 3, "c4": 100, "c5": 500}
 
 

@@ -8,6 +8,7 @@
 
 #include "../../include/sas.h"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace {
 
@@ -326,6 +327,58 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                                               ksum, topk, gated, resolve_scale(scale, d), o,
                                               idx_out, (cudaStream_t)stream),
                      "sas_decode launch");
+}
+
+// ---------------------------------------------------------------- device status
+sas_status sas_device_status(int clear, sas_stream_t stream) {
+  g_last_error.clear();
+  struct Word {
+    const char* kernel;
+    uint32_t* (*addr)();
+  };
+  static const Word words[] = {
+      {"k_decode_fused", sas::decode_fused_error_word},
+      {"k_decode_attend", sas::decode_error_word},
+      {"k_attn_fwd_tc", sas::attn_fwd_tc_error_word},
+      {"k_attn_bwd_tc", sas::attn_bwd_tc_error_word},
+      {"k_attn_simt", sas::attn_simt_error_word},
+      {"k_wait_selftest", sas::selftest_error_word},
+  };
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "sas_device_status synchronize");
+  std::string msg;
+  uint32_t all = 0;
+  for (const Word& w : words) {
+    uint32_t* p = w.addr();
+    if (p == nullptr) return fail(SAS_ERR_CUDA, "sas_device_status: no address for %s", w.kernel);
+    uint32_t v = 0;
+    e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e, "sas_device_status read");
+    if (v) {
+      if (!msg.empty()) msg += "; ";
+      msg += w.kernel;
+      if (v & sas::kErrWaitTimeout) msg += ": a bounded wait gave up";
+      if (v & sas::kErrBadIndex) msg += (v & sas::kErrWaitTimeout) ? ", " : ": ";
+      if (v & sas::kErrBadIndex) msg += "a selection index out of range was replaced";
+    }
+    all |= v;
+    if (clear && v) {
+      e = cudaMemset(p, 0, sizeof(uint32_t));
+      if (e != cudaSuccess) return cuda_status(e, "sas_device_status clear");
+    }
+  }
+  if (clear) {
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e, "sas_device_status clear");
+  }
+  if (all & sas::kErrWaitTimeout) return fail(SAS_ERR_TIMEOUT, "%s", msg.c_str());
+  if (all) return fail(SAS_ERR_INTERNAL, "%s", msg.c_str());
+  return SAS_OK;
+}
+
+sas_status sas_debug_wait_timeout(sas_stream_t stream) {
+  g_last_error.clear();
+  return cuda_status(sas::launch_wait_selftest((cudaStream_t)stream), "sas_debug_wait_timeout");
 }
 
 }  // extern "C"

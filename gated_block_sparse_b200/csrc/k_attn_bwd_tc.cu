@@ -26,10 +26,14 @@
 //   warps 0-7: gradient rows: warps w and w+4 share the TMEM lanes of rows
 //           32(w%4).. and split the 64 key columns, two warps per SM
 //           sub-partition to hide instruction latency
-// dK^T / dV^T are added to the fp32 accumulators through a per-warp
-// shared-memory transpose and 16-byte vector reductions; no CTA-wide barrier
-// runs inside the unit loop.
-// 512 TMEM columns and about 193 KB of shared memory: one CTA per SM.
+// dK^T / dV^T reach the fp32 accumulators through a per-warp shared-memory
+// transpose into [8 keys][32 d] slices, each added by one TMA tensor
+// reduce-add (two slices per warp alternate); K/V stream through a
+// three-stage ring; no CTA-wide barrier runs inside the unit loop. These
+// reductions (64 KB per unit) bound the kernel: they drain at about 20 bytes
+// per cycle per SM whether issued as vector reductions or TMA reduce-adds of
+// 1 or 4 KB.
+// 512 TMEM columns and about 213 KB of shared memory: one CTA per SM.
 #include <cuda.h>
 #include <math.h>
 
@@ -53,24 +57,25 @@ constexpr uint32_t PT_BYTES = 128 * 64 * 2;          // P or dS: 16 KB
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_DO = OFF_Q + TILE128;
 constexpr uint32_t OFF_KV = OFF_DO + TILE128;
-constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE;
+constexpr int NKV = 3;                                // K/V ring stages
+constexpr uint32_t OFF_P = OFF_KV + NKV * KV_STAGE;
 constexpr uint32_t OFF_DS = OFF_P + PT_BYTES;
-constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [64 keys][128 d] transpose
-constexpr uint32_t OFF_DL = OFF_T + 64 * D * 4;      // fp32 [unit][warp] d(log g) partials
+constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [warp][2][8 keys][32 d] slices
+constexpr uint32_t OFF_DL = OFF_T + NGW * 2 * 8 * 32 * 4;  // fp32 [unit][warp] d(log g) partials
 constexpr uint32_t OFF_BAR = OFF_DL + 129 * 8 * 4 + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr float LOG2E = 1.4426950408889634f;
 
 enum Bar {
   B_Q = 0,     // Q and dO loaded
-  B_KVF = 1,   // [2] K/V stage full
-  B_KVE = 3,   // [2] K/V stage empty (all MMAs of its unit done)
-  B_SF = 5,    // S and dP of the unit in TMEM
-  B_SE = 6,    // S and dP read by the softmax warps (4 arrivals)
-  B_PF = 7,    // P and dS written (4 arrivals)
-  B_MD = 8,    // all MMAs of the unit done
-  B_TE = 9,    // [2] dK^T/dV^T TMEM buffer read (4 arrivals)
-  NBAR = 11
+  B_KVF = 1,   // [NKV] K/V stage full
+  B_KVE = 4,   // [NKV] K/V stage empty (all MMAs of its unit done)
+  B_SF = 7,    // S and dP of the unit in TMEM
+  B_SE = 8,    // S and dP read by the gradient warps (one arrival per warp)
+  B_PF = 9,    // P and dS written (one arrival per warp)
+  B_MD = 10,   // all MMAs of the unit done
+  B_TE = 11,   // [2] dK^T/dV^T TMEM buffer read (one arrival per warp)
+  NBAR = 13
 };
 
 // TMEM columns
@@ -87,10 +92,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap domap,
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+    const __grid_constant__ CUtensorMap dkmap, const __grid_constant__ CUtensorMap dvmap,
     const float* __restrict__ lse, int Hq, int Hkv, int N, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ cnt, const float* __restrict__ logg, int topk, float scale,
-    __nv_bfloat16* __restrict__ dq, float* __restrict__ dk_acc, float* __restrict__ dv_acc,
-    float* __restrict__ dlogg) {
+    __nv_bfloat16* __restrict__ dq, float* __restrict__ dlogg) {
   extern __shared__ __align__(1024) unsigned char sm[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + NBAR * 8);
@@ -144,8 +149,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
                           b * Hq + h0 + h, &bars[B_Q]);
         }
       for (int j = 0; j < nunits; ++j) {
-        const int s = j & 1;
-        if (j >= 2) mbar_wait(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
+        const int s = j % NKV;
+        if (j >= NKV) mbar_wait_data(&bars[B_KVE + s], ((j / NKV) - 1) & 1, err);
         const int blk = unit_block(j);
         if (j < kk && blk != idx_row[j]) atomicOr(err, kErrBadIndex);
         unsigned char* st = sm + OFF_KV + s * KV_STAGE;
@@ -165,15 +170,15 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
       constexpr uint32_t ID_T = tc::idesc_bf16(128, 64, 1, 1);       // dK^T, dV^T
       const uint32_t q_a = smem_u32(sm + OFF_Q), do_a = smem_u32(sm + OFF_DO);
       const uint32_t p_a = smem_u32(sm + OFF_P), ds_a = smem_u32(sm + OFF_DS);
-      mbar_wait(&bars[B_Q], 0, err);
+      mbar_wait_data(&bars[B_Q], 0, err);
       // S/dP of unit j+1 are issued as soon as the gradient warps have copied
       // S/dP of unit j into registers, so they run while unit j's P and dS are
       // being formed; the dQ / dK^T / dV^T products of unit j follow.
       auto issue_sdp = [&](int j) {
-        const int s = j & 1;
+        const int s = j % NKV;
         const uint32_t k_a = smem_u32(sm + OFF_KV + s * KV_STAGE);
         const uint32_t v_a = k_a + 16384;
-        mbar_wait(&bars[B_KVF + s], (j >> 1) & 1, err);
+        mbar_wait_data(&bars[B_KVF + s], (j / NKV) & 1, err);
         if (j >= 1) mbar_wait(&bars[B_SE], (j - 1) & 1, err);
         tc::fence_after_sync();
 #pragma unroll
@@ -187,8 +192,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         tc::commit(&bars[B_SF]);
       };
       auto issue_grad = [&](int j) {
-        const int s = j & 1;
-        const uint32_t k_a = smem_u32(sm + OFF_KV + s * KV_STAGE);
+        const int s = j & 1;  // dK^T / dV^T TMEM buffer
+        const int ks_ = j % NKV;
+        const uint32_t k_a = smem_u32(sm + OFF_KV + ks_ * KV_STAGE);
         mbar_wait(&bars[B_PF], j & 1, err);
         if (j >= 2) mbar_wait(&bars[B_TE + s], ((j >> 1) - 1) & 1, err);
         tc::fence_after_sync();
@@ -205,7 +211,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
                        tc::sw128_desc(p_a + ks * 2048, 8192, 1024), ID_T, ks > 0);
         }
         tc::commit(&bars[B_MD]);
-        tc::commit(&bars[B_KVE + s]);
+        tc::commit(&bars[B_KVE + ks_]);
       };
       issue_sdp(0);
       for (int j = 0; j < nunits; ++j) {
@@ -243,44 +249,48 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     }
     unsigned char* prow = sm + OFF_P + row * 128;
     unsigned char* dsrow = sm + OFF_DS + row * 128;
-    const size_t kvbase = ((size_t)b * Hkv + r) * N * D;
-    float* tsm = reinterpret_cast<float*>(sm + OFF_T);
+    const int plane = b * Hkv + r;
+    float* tw = reinterpret_cast<float*>(sm + OFF_T) + warp * 512;  // two [8][32] slices
     const int gtid = hc * 128 + row;  // 0..255 over the gradient warps
     // Add unit jj's dK^T / dV^T (TMEM lanes = d, columns = keys) to the fp32
-    // accumulators: transpose through shared memory into [key][d], then one
-    // 16-byte vector reduction per four head-dim values.
+    // accumulators: each group of 8 keys is transposed into a [key][d] slice
+    // and added by one TMA reduce-add (rows past N are clipped by the map; a
+    // group wholly past N is skipped). Slices alternate with the count of
+    // issued groups, so the reduce issued from a slice two groups earlier
+    // must have read it before the slice is rewritten.
+    int ngroups = 0;
     auto flush_kv = [&](int jj) {
       const int blk = unit_block(jj);
-      const int nkeys = min(64, N - 64 * blk);
       const uint32_t cb = tmem + (jj & 1) * C_BUF + lane_off;
-      float* tw = tsm + warp * 1024;  // this warp's [32 keys][32 d] slice
 #pragma unroll 1
       for (int m2 = 0; m2 < 2; ++m2) {
-        float* acc = m2 == 0 ? dk_acc : dv_acc;
         float kv[32];
         tc::tmem_ld32(cb + (m2 == 0 ? C_DKT : C_DVT) + 32 * hc, kv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) tw[i * 32 + lane] = kv[i];
-        __syncwarp();
-        float* dst = acc + kvbase + (size_t)(64 * blk + 32 * hc) * D + 32 * wq;
+        for (int g = 0; g < 4; ++g) {
+          const int key0 = 64 * blk + 32 * hc + 8 * g;
+          if (key0 >= N) continue;  // warp-uniform
+          float* sl = tw + ((ngroups & 1) << 8);
+          if (lane == 0) tc::bulk_wait_read<1>();
+          __syncwarp();
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int e = lane + 32 * it;
-          const int key = e >> 3, d4 = (e & 7) << 2;
-          if (32 * hc + key < nkeys) {
-            const float4 x = *reinterpret_cast<const float4*>(tw + key * 32 + d4);
-            tc::red_add_v4(dst + (size_t)key * D + d4, x.x, x.y, x.z, x.w);
+          for (int i = 0; i < 8; ++i) sl[i * 32 + lane] = kv[8 * g + i];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_reduce_add_3d(m2 == 0 ? &dkmap : &dvmap, sl, 32 * wq, key0, plane);
+            tc::bulk_commit();
           }
+          ++ngroups;
         }
-        __syncwarp();
       }
     };
     float* dl_s = reinterpret_cast<float*>(sm + OFF_DL);
     for (int j = 0; j < nunits; ++j) {
       const bool cur = (j == kk);
       const float bias = cur ? 0.f : logg_row[j] * LOG2E;
-      mbar_wait(&bars[B_SF], j & 1, err);
+      mbar_wait_data(&bars[B_SF], j & 1, err);
       tc::fence_after_sync();
       float sv[32], dp[32];
       tc::tmem_ld32(tmem + C_S + lane_off + 32 * hc, sv);
@@ -308,7 +318,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         dk2[i >> 1] = *reinterpret_cast<uint32_t*>(&hd2);
       }
       if (j >= 1) {  // MMAs of the previous unit done: P/dS buffers free, dK^T/dV^T ready
-        mbar_wait(&bars[B_MD], (j - 1) & 1, err);
+        mbar_wait_data(&bars[B_MD], (j - 1) & 1, err);
         tc::fence_after_sync();
       }
 #pragma unroll
@@ -334,9 +344,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         if (lane == 0) dl_s[j * NGW + warp] = dsum;
       }
     }
-    mbar_wait(&bars[B_MD], (nunits - 1) & 1, err);
+    mbar_wait_data(&bars[B_MD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
     flush_kv(nunits - 1);
+    if (lane == 0) tc::bulk_wait<0>();  // every reduce of this warp has completed
     named_bar_softmax();
     for (int j = gtid; j < kk; j += 2 * 128) {  // d(log g): fixed-order sum over the warps
       float a = 0.f;
@@ -399,17 +410,19 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(dlogg, 0, (size_t)B * Hkv * T_ * topk * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  CUtensorMap qm, km, vm, dom;
+  CUtensorMap qm, km, vm, dom, dkm, dvm;
   if (!make_map(&qm, q, N, B * Hq) || !make_map(&km, k, N, B * Hkv) ||
-      !make_map(&vm, v, N, B * Hkv) || !make_map(&dom, dout, N, B * Hq))
+      !make_map(&vm, v, N, B * Hkv) || !make_map(&dom, dout, N, B * Hq) ||
+      !make_tma_map_f32_3d(&dkm, dk_acc, D, N, B * Hkv, 32, 8) ||
+      !make_tma_map_f32_3d(&dvm, dv_acc, D, N, B * Hkv, 32, 8))
     return cudaErrorInvalidValue;
   e = ensure_smem(k_attn_bwd_tc, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(T_, Hkv * (Hq / Hkv / 2), B);
   k_attn_bwd_tc<<<grid, BT_THREADS, SMEM_BYTES, st>>>(
       qm, km, vm, dom, static_cast<const __nv_bfloat16*>(o),
-      static_cast<const __nv_bfloat16*>(dout), lse, Hq, Hkv, N, idx, cnt, logg, topk, scale,
-      static_cast<__nv_bfloat16*>(dq), dk_acc, dv_acc, dlogg);
+      static_cast<const __nv_bfloat16*>(dout), dkm, dvm, lse, Hq, Hkv, N, idx, cnt, logg, topk,
+      scale, static_cast<__nv_bfloat16*>(dq), dlogg);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int cgrid = (int)((nkv + 255) / 256 < 8192 ? (nkv + 255) / 256 : 8192);

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
                           b * Hq + h0 + h, &bars[B_Q]);
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
-        if (j >= 2) mbar_wait(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
+        if (j >= 2) mbar_wait_data(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
         int blk = (j < kk) ? idx_row[j] : t;
         if (blk < 0 || blk >= t) {
           if (j < kk) atomicOr(err, kErrBadIndex);
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       constexpr uint32_t ID_PV = tc::idesc_bf16(128, 128, 0, 1);
       const uint32_t q_addr = smem_u32(sm + OFF_Q);
       const uint32_t p_addr = smem_u32(sm + OFF_P);
-      mbar_wait(&bars[B_Q], 0, err);
+      mbar_wait_data(&bars[B_Q], 0, err);
       auto pv = [&](int j) {  // O += P_j V_j
         mbar_wait(&bars[B_PF], j & 1, err);
         tc::fence_after_sync();
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       };
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
-        mbar_wait(&bars[B_KVF + s], (j >> 1) & 1, err);
+        mbar_wait_data(&bars[B_KVF + s], (j >> 1) & 1, err);
         if (j >= 2) mbar_wait(&bars[B_SE + s], ((j >> 1) - 1) & 1, err);
         tc::fence_after_sync();
         const uint32_t k_addr = smem_u32(sm + OFF_KV + s * KV_STAGE_BYTES);
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       const int s = j & 1;
       const bool cur = (j == kk);
       const float bias = cur ? 0.f : logg_row[j] * LOG2E;
-      mbar_wait(&bars[B_SF + s], (j >> 1) & 1, err);
+      mbar_wait_data(&bars[B_SF + s], (j >> 1) & 1, err);
       tc::fence_after_sync();
       float z[64];
       {
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       }
       if (j > 0) {
         // PV_{j-1} must be done: O is stable and the P buffer is free
-        mbar_wait(&bars[B_OD], (j - 1) & 1, err);
+        mbar_wait_data(&bars[B_OD], (j - 1) & 1, err);
         tc::fence_after_sync();
         const float alpha = grow ? tc::ex2(m - muse) : 1.f;
         if (__any_sync(0xffffffffu, grow)) {
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       if (lane == 0) mbar_arrive(&bars[B_PF]);
     }
     // epilogue
-    mbar_wait(&bars[B_OD], (nunits - 1) & 1, err);
+    mbar_wait_data(&bars[B_OD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
     const float inv = 1.f / l;
     const bool valid = pos < N;

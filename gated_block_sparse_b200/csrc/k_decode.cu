@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode_attend(
     }
   }
   bool ok = true;
-  if (nu > 0) ok = mbar_wait(&bar, 0, &g_decode_err);
+  if (nu > 0) ok = mbar_wait_data(&bar, 0, &g_decode_err);
   ok = __syncthreads_and(ok) != 0;  // block-uniform before the barriers below
 
   if (nu > 0 && ok) {

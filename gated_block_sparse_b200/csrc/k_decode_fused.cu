@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     for (int i = 0; i < nsub; ++i) {
       const int slot = i % FD_NS;
       const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
-      mbar_wait(&sum_bar[slot], (uint32_t)((i / FD_NS) & 1), err);
+      mbar_wait_data(&sum_bar[slot], (uint32_t)((i / FD_NS) & 1), err);
       const float* sb = ring + (size_t)slot * FD_SUBC * D;
       for (int j0 = wid; j0 < cnt_i; j0 += 4 * FD_WARPS) {
         float part[4];
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const int u = unit_of(i);
     const bool cur = (u == kk);
     const float bias = (!cur && gated) ? klogg[u] : 0.f;
-    mbar_wait(&full[slot], (uint32_t)((i / NKV) & 1), err);
+    mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
     const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot);
     const T* vt = kt + TILE;
     float dot[G], dot1[G];

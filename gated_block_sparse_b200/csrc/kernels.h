@@ -12,6 +12,9 @@ namespace sas {
 // ({64, 64, 1} box, 128-byte swizzle, zero fill); false when encoding fails.
 bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int rows_per_plane,
                           int planes);
+// 3-D fp32 TMA tensor map with a {box_d, box_rows, 1} box, no swizzle.
+bool make_tma_map_f32_3d(CUtensorMap* map, const void* base, int d, int rows_per_plane,
+                         int planes, int box_d, int box_rows);
 
 // Block summaries: ksum[b,h,m] = mean of keys 64m..64m+63.
 cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
@@ -85,6 +88,12 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                const float* logg, int topk, float scale, void* dq, void* dk,
                                void* dv, float* dlogg, void* ws, cudaStream_t st);
 uint32_t* attn_bwd_tc_error_word();
+
+// Self-test of the bounded wait (k_status.cu): one warp waits on a barrier
+// that nothing completes; after the wait limit it records kErrWaitTimeout in
+// its own error word.
+cudaError_t launch_wait_selftest(cudaStream_t st);
+uint32_t* selftest_error_word();
 size_t attn_bwd_simt_ws_bytes(int B, int Hkv, int N, int d);
 cudaError_t launch_attn_bwd_simt(const void* q, const void* k, const void* v, const void* o,
                                  const void* dout, int bf16, int B, int Hq, int Hkv, int N, int d,

@@ -61,10 +61,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 // hardware-chosen time, so the bound is on time, not on the poll count.
 constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;  // 200 ms
 
-// Bounded wait for the phase with the given parity to complete. Returns false
-// if it gives up: after kWaitLimitNs, or at once when *err already carries
-// kErrWaitTimeout (a wait elsewhere timed out: the launch is aborting, so no
-// further wait may stall). A timeout sets kErrWaitTimeout in *err.
+// Bounded wait for the phase with the given parity to complete, for phases
+// completed by other threads' arrivals. Returns false if it gives up: after
+// kWaitLimitNs, or at once when *err already carries kErrWaitTimeout (a wait
+// elsewhere timed out: the launch is aborting, so no further wait may stall).
+// A timeout sets kErrWaitTimeout in *err.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
@@ -74,6 +75,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
       if (err && (*reinterpret_cast<volatile uint32_t*>(err) & kErrWaitTimeout)) return false;
       if (global_ns() - t0 > kWaitLimitNs) break;
     }
+  }
+  if (err) atomicOr(err, kErrWaitTimeout);
+  return false;
+}
+
+// Bounded wait for a phase completed by data this CTA has in flight (its own
+// TMA or bulk copies, its tensor-core operations through tcgen05.commit).
+// Bounded by kWaitLimitNs only: even when the launch is aborting it keeps
+// waiting, so that no copy or MMA still writes into this CTA's shared memory
+// or TMEM when the CTA frees them or exits. Every such operation is issued
+// on the abort path too, so these waits end promptly there.
+__device__ __forceinline__ bool mbar_wait_data(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
   }
   if (err) atomicOr(err, kErrWaitTimeout);
   return false;
@@ -138,16 +156,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
-// Bounded wait (as mbar_wait) on a barrier filled by other CTAs.
+// Bounded wait (as mbar_wait_data) on a barrier completed by other CTAs'
+// remote stores into this CTA: it keeps waiting while the launch aborts, so
+// the CTA does not leave while those stores may still land.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* err) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 15u) == 0) {
-      if (err && (*reinterpret_cast<volatile uint32_t*>(err) & kErrWaitTimeout)) return false;
-      if (global_ns() - t0 > kWaitLimitNs) break;
-    }
+    if ((i & 15u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
   }
   if (err) atomicOr(err, kErrWaitTimeout);
   return false;

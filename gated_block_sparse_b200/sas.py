@@ -43,6 +43,8 @@ SIGNATURES = {
                                _P, _P, _Z, _P]),
     "sas_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P, _P, _Z,
                         _P]),
+    "sas_device_status": (_I, [_I, _P]),
+    "sas_debug_wait_timeout": (_I, [_P]),
 }
 
 _lib = None
@@ -246,3 +248,21 @@ def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: fl
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
         float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
     return out
+
+
+def sas_device_status(clear: bool = False, stream=None) -> tuple[int, str]:
+    """Synchronise `stream` and read the kernels' device error words.
+
+    Returns (status, message): SAS_ERR_TIMEOUT (4) if a bounded wait gave up,
+    SAS_ERR_INTERNAL (5) if a selection index was out of range, 0 otherwise.
+    clear=True resets the words after reading them. Does not raise.
+    """
+    lib = load_library()
+    st = lib.sas_device_status(int(bool(clear)), _stream(stream))
+    return st, lib.sas_last_error_message().decode()
+
+
+def sas_debug_wait_timeout(stream=None) -> None:
+    """Launch the self-test kernel whose wait nothing completes (gives up after 200 ms)."""
+    lib = load_library()
+    _check("sas_debug_wait_timeout", lib.sas_debug_wait_timeout(_stream(stream)))

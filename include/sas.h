@@ -18,9 +18,10 @@
  *
  * Conventions shared by every call
  *   - Every tensor pointer is a DEVICE pointer, allocated and owned by the
- *     caller. The library never allocates, frees or synchronises; all work is
- *     enqueued on `stream` (NULL = the legacy default stream) and the call
- *     returns as soon as it is enqueued.
+ *     caller. The library never allocates, frees or synchronises (apart from
+ *     the two diagnostic calls at the end of this file); all work is enqueued
+ *     on `stream` (NULL = the legacy default stream) and the call returns as
+ *     soon as it is enqueued.
  *   - Layouts are dense row-major ("HND"): q, o, dO, dq [B][Hq][N][d];
  *     k, v, dk, dv [B][Hkv][N][d]; decode q/o [B][Hq][d]; caches
  *     [B][Hkv][Lmax][d]; block summaries [B][Hkv][N/64][d] fp32.
@@ -62,7 +63,7 @@ typedef enum sas_status {
   SAS_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or argument      */
   SAS_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, group, topk)    */
   SAS_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed          */
-  SAS_ERR_TIMEOUT = 4,      /* reserved: a bounded device wait gave up       */
+  SAS_ERR_TIMEOUT = 4,      /* a bounded device wait gave up (see below)     */
   SAS_ERR_INTERNAL = 5      /* an internal consistency check failed          */
 } sas_status;
 
@@ -212,6 +213,31 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              const int32_t* idx, const int32_t* cnt, const float* logg, int topk,
                              int gated, float scale, void* o, void* ws, size_t ws_bytes,
                              sas_stream_t stream);
+
+/*
+ * Device status. Kernels never trap: every wait on an mbarrier is bounded in
+ * wall-clock time (200 ms); a wait that gives up, or a selection index out of
+ * range (replaced by the current block), sets a bit in a per-kernel error
+ * word in device memory, and the launch runs to completion with unspecified
+ * results for the affected rows.
+ *
+ * sas_device_status synchronises `stream`, reads every kernel's error word
+ * (they are per process and device, shared by all streams) and returns
+ * SAS_ERR_TIMEOUT if any wait gave up, SAS_ERR_INTERNAL if only an index was
+ * out of range, SAS_OK otherwise; sas_last_error_message() names the
+ * kernels. clear != 0 resets the words afterwards (the status returned is
+ * the one read before clearing). This call and sas_debug_wait_timeout are
+ * the only ones that synchronise; they are for diagnostics and tests.
+ */
+sas_status sas_device_status(int clear, sas_stream_t stream);
+
+/*
+ * Test hook for the failure path: enqueues a one-warp kernel whose barrier
+ * nothing completes. It gives up after the wait limit (200 ms), records a
+ * timeout in its error word and exits; nothing hangs or faults. A following
+ * sas_device_status returns SAS_ERR_TIMEOUT naming k_wait_selftest.
+ */
+sas_status sas_debug_wait_timeout(sas_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -60,7 +60,7 @@ def measured_peaks() -> dict:
 def source_sha(name: str) -> str:
     """Hash of a kernel's source file and the shared device headers."""
     h = hashlib.sha256()
-    for f in (name, "common.cuh", "ptx.cuh"):
+    for f in (name, "common.cuh", "ptx.cuh", "tc.cuh"):
         h.update(open(os.path.join(ROOT, "gated_block_sparse_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

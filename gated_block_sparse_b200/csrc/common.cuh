@@ -157,41 +157,44 @@ __device__ inline int tree_merge(unsigned long long* A, int* Alen, unsigned long
 // counts the survivors above it, which is its global rank (every key above a
 // survivor is a survivor). Otherwise the lists are merged pairwise
 // (tree_merge over A and B, whose length arrays it overwrites). *cnt is 0 on
-// entry. All threads of the block call it; it ends with a barrier.
+// entry; th_s is one shared word for the threshold. All threads of the
+// block call it; it ends with a barrier.
 __device__ inline void topk_of_lists(unsigned long long* A, int* len, int nl, int lg, int k,
                                      unsigned long long* out, unsigned long long* tmp,
-                                     unsigned long long* B, int* Blen, int* cnt) {
+                                     unsigned long long* B, int* Blen, int* cnt,
+                                     unsigned long long* th_s) {
   const int kq = 1 << lg;
   const int lane = threadIdx.x & 31;
-  unsigned long long th = 0;
-  {
-    unsigned long long v = 0;
-    if (lane < nl && k > 0 && len[lane] >= k) v = A[(lane << lg) + k - 1];
+  if (threadIdx.x < 32) {  // one warp finds the threshold; the block reads it back
+    unsigned long long th = 0;
+    if (lane < nl && k > 0 && len[lane] >= k) th = A[(lane << lg) + k - 1];
 #pragma unroll
     for (int off = 16; off; off >>= 1) {
-      const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, off);
-      v = w > v ? w : v;
+      const unsigned long long w = __shfl_xor_sync(0xffffffffu, th, off);
+      th = w > th ? w : th;
     }
-    th = v;
-  }
-  // A tighter bound when k <= 32: the k-th largest of the 32 keys made of each
-  // list's first 32/nl' entries (nl' = nl rounded up to a power of two) is
-  // also at most the k-th largest of all keys. Each lane counts the keys of
-  // that sample above its own.
-  if (k <= 32) {
-    int nlp = 1;
-    while (nlp < nl) nlp <<= 1;
-    const int m = 32 / nlp, l = lane / m, p = lane % m;
-    const unsigned long long mine = (l < nl && p < len[l]) ? A[(l << lg) + p] : 0ull;
-    int above = 0;
+    // A tighter bound when k <= 32: the k-th largest of the 32 keys made of
+    // each list's first 32/nl' entries (nl' = nl rounded up to a power of
+    // two) is also at most the k-th largest of all keys. Each lane counts the
+    // keys of that sample above its own.
+    if (k <= 32) {
+      int nlp = 1;
+      while (nlp < nl) nlp <<= 1;
+      const int m = 32 / nlp, l = lane / m, p = lane % m;
+      const unsigned long long mine = (l < nl && p < len[l]) ? A[(l << lg) + p] : 0ull;
+      int above = 0;
 #pragma unroll 8
-    for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, mine, j) > mine;
-    const unsigned hit = __ballot_sync(0xffffffffu, mine != 0ull && above == k - 1);
-    if (hit) {
-      const unsigned long long kth = __shfl_sync(0xffffffffu, mine, __ffs(hit) - 1);
-      th = kth > th ? kth : th;
+      for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, mine, j) > mine;
+      const unsigned hit = __ballot_sync(0xffffffffu, mine != 0ull && above == k - 1);
+      if (hit) {
+        const unsigned long long kth = __shfl_sync(0xffffffffu, mine, __ffs(hit) - 1);
+        th = kth > th ? kth : th;
+      }
     }
+    if (lane == 0) *th_s = th;
   }
+  __syncthreads();
+  const unsigned long long th = *th_s;
   const int total = nl << lg;
   for (int e0 = 0; e0 < total; e0 += blockDim.x) {
     const int e = e0 + (int)threadIdx.x;
@@ -213,6 +216,7 @@ __device__ inline void topk_of_lists(unsigned long long* A, int* len, int nl, in
     for (int i = threadIdx.x; i < S; i += blockDim.x) {
       const unsigned long long key = tmp[i];
       int rank = 0;
+#pragma unroll 8
       for (int j = 0; j < S; ++j) rank += tmp[j] > key;
       if (rank < k) out[rank] = key;
     }

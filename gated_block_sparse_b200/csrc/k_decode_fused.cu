@@ -18,11 +18,13 @@
 //      min(k, n) candidates, and stores both into its slot of every CTA of
 //      the cluster with asynchronous remote stores that complete on the
 //      receiver's mbarrier;
-//   3. once all lists have landed, every CTA merges them identically (one
-//      level: each candidate counts the keys above it in the other lists)
-//      and holds the row's kept blocks (ascending) and the gate's LSE;
+//   3. once all lists have landed, every CTA computes the gate's LSE and the
+//      same Top-K: the keys above a pruning threshold are ranked among
+//      themselves, giving the kept blocks in score order (CTA 0 also writes
+//      them in ascending block order to idx_out);
 //   4. streams the K/V blocks of its share of the units (the current block
-//      first, then kept blocks) through a ring that reuses the summary ring.
+//      first, then kept blocks in score order) through a ring that reuses
+//      the summary ring.
 //      Each warp takes 8 keys of every unit and keeps its own online-softmax
 //      state (m, l, acc) for every head of the group, so no CTA-wide barrier
 //      runs per unit;
@@ -54,10 +56,11 @@ constexpr int FD_WARPS = FD_THREADS / 32;
 constexpr int FD_NS = 3;      // summary ring slots
 constexpr int FD_SUBC = 32;   // summaries per ring slot
 constexpr int FD_MAXKV = 4;   // K/V ring slots at most
+constexpr int FD_MAXCS = 16;  // cluster size at most
 constexpr unsigned FULL = 0xffffffffu;
 
 struct FdSmem {  // byte offsets into dynamic shared memory
-  size_t u, q, qbar, sc, mine, slen, stage, sstat, fin, kidx, klogg, cst, cml, bars, total;
+  size_t u, q, qbar, sc, mine, slen, stage, sstat, fin, cst, cml, zp, bars, total;
   size_t wl, wb, tmp, mb, mblen;  // list scratch inside region u, after K/V slot 0
   int nkv;                        // K/V ring slots held by region u
 };
@@ -92,10 +95,9 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int k
   L.stage = o; o += fd_al((size_t)CS * kq * 8);
   L.sstat = o; o += fd_al((size_t)CS * 8);
   L.fin = o; o += fd_al((size_t)kq * 8);
-  L.kidx = o; o += fd_al((size_t)kq * 4);
-  L.klogg = o; o += fd_al((size_t)kq * 4);
   L.cst = o; o += fd_al((size_t)CS * D * 4);
   L.cml = o; o += fd_al((size_t)CS * 8);
+  L.zp = o; o += fd_al((size_t)FD_WARPS * 2 * 8 * G * 4);  // per warp: z and p of its 8 keys
   L.bars = o; o += fd_al((size_t)(FD_NS + 2 * FD_MAXKV + 2) * 8);
   L.total = o;
   return L;
@@ -122,6 +124,24 @@ __device__ __forceinline__ void loadn(const float* p, float (&v)[N]) {
   } else {
     const float2 a = *reinterpret_cast<const float2*>(p);
     v[0] = a.x; v[1] = a.y;
+  }
+}
+
+// G consecutive fp32 values from shared memory (16-byte loads when G % 4 == 0).
+template <int G>
+__device__ __forceinline__ void loadg(const float* p, float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(p + i);
+      v[i] = a.x; v[i + 1] = a.y; v[i + 2] = a.z; v[i + 3] = a.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    v[0] = a.x; v[1] = a.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < G; ++i) v[i] = p[i];
   }
 }
 
@@ -179,10 +199,9 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   unsigned long long* stage = reinterpret_cast<unsigned long long*>(sm + L.stage);
   float* sstat = reinterpret_cast<float*>(sm + L.sstat);
   unsigned long long* fin = reinterpret_cast<unsigned long long*>(sm + L.fin);
-  int* kidx = reinterpret_cast<int*>(sm + L.kidx);
-  float* klogg = reinterpret_cast<float*>(sm + L.klogg);
   float* cst = reinterpret_cast<float*>(sm + L.cst);
   float* cml = reinterpret_cast<float*>(sm + L.cml);
+  float* zp = reinterpret_cast<float*>(sm + L.zp);
   uint64_t* sum_bar = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* full = sum_bar + FD_NS;
   uint64_t* empty = full + FD_MAXKV;
@@ -191,6 +210,9 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   __shared__ float wred_m[FD_WARPS], wred_s[FD_WARPS];
   __shared__ int wlen[FD_WARPS], wlen_b[FD_WARPS];
   __shared__ int surv_cnt;
+  __shared__ unsigned long long th_s;
+  __shared__ float cw[FD_MAXCS];                      // combine weights of the CS states
+  __shared__ float fw[FD_WARPS * 8], fm[8], fl[8];    // fold weights per (head, warp)
 
   const int r = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * G;
@@ -256,13 +278,19 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       bulk_g2s(U + TILE * sizeof(T), vc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &full[0]);
     }
   }
+  // Barriers are initialised and fenced (fence.mbarrier_init.release.cluster
+  // above): other CTAs may store into this one once every thread of the
+  // cluster has arrived. A relaxed arrive does not wait for this thread's
+  // loads in flight. A remote store that lands before the local expect_tx
+  // only drives the transaction count below zero for a while; the phase
+  // cannot complete before the local arrival.
+  cluster_arrive_relaxed();
 #pragma unroll
   for (int j = 0; j < QPT; ++j) {
     const int i = tid + j * FD_THREADS;
     if (i < G * D) q_s[i] = qreg[j];
   }
   __syncthreads();
-  cluster_arrive_release();  // barriers are initialised: other CTAs may store into this one
   for (int i = tid; i < D; i += FD_THREADS) {
     float a = 0.f;
 #pragma unroll
@@ -336,6 +364,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     if (tid < nmine) {
       const float sj = sc[tid];
       int rk = 0;
+#pragma unroll 8
       for (int x = 0; x < nmine; ++x) {
         const float sx = sc[x];
         rk += (sx > sj) || (sx == sj && x < tid);
@@ -372,8 +401,17 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       if (p < my_len) {
         st_async_u64(mapa(lst + 8u * p, c), mylist[p], mapa(lbar, c));
       } else {
-        float M = -FLT_MAX, S = 0.f;
-        for (int w = 0; w < FD_WARPS; ++w) ms_merge(M, S, wred_m[w], wred_s[w]);
+        float m4[4], s4[4];  // tree over the 8 warp pairs
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          m4[w] = wred_m[w];
+          s4[w] = wred_s[w];
+          ms_merge(m4[w], s4[w], wred_m[w + 4], wred_s[w + 4]);
+        }
+        ms_merge(m4[0], s4[0], m4[2], s4[2]);
+        ms_merge(m4[1], s4[1], m4[3], s4[3]);
+        ms_merge(m4[0], s4[0], m4[1], s4[1]);
+        const float M = m4[0], S = s4[0];
         st_async_f32x2(mapa(sst, c), M, S, mapa(lbar, c));
       }
     }
@@ -389,31 +427,21 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const float S = warp_sum(se > 0.f ? se * __expf(mx - M) : 0.f);
     lse = (C > 0) ? M + __logf(S) : 0.f;
   }
-  if (topk > 0) {
-    if (kk > 0) {
-      topk_of_lists(stage, slen, CS, lg, topk, fin, tmp, mb, mblen, &surv_cnt);
-      for (int i = tid; i < kk; i += FD_THREADS) {  // ascending block order
-        const int mi = key_block(fin[i]);
-        int pos = 0;
-        for (int j = 0; j < kk; ++j) pos += key_block(fin[j]) < mi;
-        kidx[pos] = mi;
-        klogg[pos] = key_score(fin[i]) - lse;
-      }
-      __syncthreads();
-    }
-    if (crank == 0 && idx_out != nullptr)
-      for (int i = tid; i < topk; i += FD_THREADS) idx_out[row * topk + i] = i < kk ? kidx[i] : -1;
-  }
+  // Units are taken in score order (fin[u], best first): a CTA knows its
+  // blocks as soon as the merge ends. Ascending block order is needed only
+  // for idx_out, which CTA 0 writes.
+  if (topk > 0 && kk > 0)
+    topk_of_lists(stage, slen, CS, lg, topk, fin, tmp, mb, mblen, &surv_cnt, &th_s);
 
   // ---- 4. attention over this CTA's units: the current block first when
-  // owned (already in flight in slot 0), then its kept blocks ascending.
+  // owned (already in flight in slot 0), then its kept blocks in score order.
   auto unit_of = [&](int i) -> int {
     if (own_cur) return i == 0 ? kk : u0 + i - 1;
     return u0 + i;
   };
   auto issue_unit = [&](int i) {
     const int u = unit_of(i);
-    int blk = (u == kk) ? t : kidx[u];
+    int blk = (u == kk) ? t : key_block(fin[u]);
     if (blk < 0 || blk >= nblk) {
       atomicOr(err, kErrBadIndex);
       blk = t;
@@ -427,6 +455,19 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   };
   if (tid == 0)
     for (int i = own_cur ? 1 : 0; i < min(NKV, nu); ++i) issue_unit(i);
+  if (crank == 0 && idx_out != nullptr && topk > 0) {  // kept blocks, ascending, -1 padded
+    for (int i = tid; i < topk; i += FD_THREADS) {
+      if (i >= kk) {
+        idx_out[row * topk + i] = -1;
+        continue;
+      }
+      const int mi = key_block(fin[i]);
+      int pos = 0;
+#pragma unroll 8
+      for (int j = 0; j < kk; ++j) pos += key_block(fin[j]) < mi;
+      idx_out[row * topk + pos] = mi;
+    }
+  }
   float m_w[G], l_w[G], acc[G][CPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -441,7 +482,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const int slot = i % NKV;
     const int u = unit_of(i);
     const bool cur = (u == kk);
-    const float bias = (!cur && gated) ? klogg[u] : 0.f;
+    const float bias = (!cur && gated) ? key_score(fin[u]) - lse : 0.f;
     mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
     const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot);
     const T* vt = kt + TILE;
@@ -465,44 +506,70 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) dot[h] += dot1[h];
-    float p[G], alpha[G];
+    // z of this lane's key (the four lanes of a key hold the same value);
+    // the warp's 8 keys meet in shared memory, read back by broadcast.
+    float* zw = zp + wid * (2 * 8 * G);  // [8 keys][G] z, then [8 keys][G] p
+    float* pw = zw + 8 * G;
+    float z[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float z = dot[h] + __shfl_xor_sync(FULL, dot[h], 1);
-      z += __shfl_xor_sync(FULL, z, 2);
-      z = (cur && key >= ncur) ? -INFINITY : z * scale + bias;
-      float zm = fmaxf(z, __shfl_xor_sync(FULL, z, 4));
-      zm = fmaxf(zm, __shfl_xor_sync(FULL, zm, 8));
-      zm = fmaxf(zm, __shfl_xor_sync(FULL, zm, 16));
-      const float mn = fmaxf(m_w[h], zm);
+      float d2 = dot[h] + __shfl_xor_sync(FULL, dot[h], 1);
+      d2 += __shfl_xor_sync(FULL, d2, 2);
+      z[h] = (cur && key >= ncur) ? -INFINITY : d2 * scale + bias;
+    }
+    const int kl = lane >> 2;
+    if (qq == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) zw[kl * G + h] = z[h];
+    }
+    __syncwarp();
+    float zmax[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) zmax[h] = -INFINITY;
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {
+      float zz[G];
+      loadg<G>(zw + k8 * G, zz);
+#pragma unroll
+      for (int h = 0; h < G; ++h) zmax[h] = fmaxf(zmax[h], zz[h]);
+    }
+    float alpha[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mn = fmaxf(m_w[h], zmax[h]);
+      float p;
       if (mn == -INFINITY) {  // every key seen so far is masked
-        p[h] = 0.f;
+        p = 0.f;
         alpha[h] = 1.f;
       } else {
-        p[h] = __expf(z - mn);
+        p = __expf(z[h] - mn);
         alpha[h] = __expf(m_w[h] - mn);
       }
-      float ps = p[h] + __shfl_xor_sync(FULL, p[h], 4);
-      ps += __shfl_xor_sync(FULL, ps, 8);
-      ps += __shfl_xor_sync(FULL, ps, 16);
-      l_w[h] = l_w[h] * alpha[h] + ps;
       m_w[h] = mn;
+      if (qq == 0) pw[kl * G + h] = p;
     }
+    __syncwarp();
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
       for (int c = 0; c < CPL; ++c) acc[h][c] *= alpha[h];
+    float psum[G];
 #pragma unroll
-    for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys: p from the key's lanes
-      float v[CPL];
+    for (int h = 0; h < G; ++h) psum[h] = 0.f;
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys
+      float pk[G], v[CPL];
+      loadg<G>(pw + k8 * G, pk);
       loadn<CPL>(vt + (size_t)(wid * 8 + k8) * D + lane * CPL, v);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pk = __shfl_sync(FULL, p[h], k8 * 4);
+        psum[h] += pk[h];
 #pragma unroll
-        for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk, pk, v[c], v[c + 1]);
+        for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk[h], pk[h], v[c], v[c + 1]);
       }
     }
+#pragma unroll
+    for (int h = 0; h < G; ++h) l_w[h] = l_w[h] * alpha[h] + psum[h];
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
     if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
@@ -525,51 +592,73 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
   }
   __syncthreads();
+  if (wid == 0) {  // fold weights: lane = (head within a group of 4, warp)
+    for (int h0 = 0; h0 < G; h0 += 4) {
+      const int h = h0 + (lane >> 3), w = lane & 7;
+      float m = -INFINITY, l = 0.f;
+      if (h < G) {
+        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
+        l = ws[D + 1];
+        if (l > 0.f) m = ws[D];
+      }
+      float M = m;
+      M = fmaxf(M, __shfl_xor_sync(FULL, M, 1));
+      M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
+      M = fmaxf(M, __shfl_xor_sync(FULL, M, 4));
+      const float f = l > 0.f ? __expf(m - M) : 0.f;
+      float Ls = l * f;
+      Ls += __shfl_xor_sync(FULL, Ls, 1);
+      Ls += __shfl_xor_sync(FULL, Ls, 2);
+      Ls += __shfl_xor_sync(FULL, Ls, 4);
+      if (h < G) {
+        fw[h * 8 + w] = f;
+        if (w == 0) {
+          fm[h] = M;
+          fl[h] = Ls;
+        }
+      }
+    }
+  }
+  __syncthreads();
   {
     const uint32_t cst_r = smem_u32(cst) + (uint32_t)(crank * D * 4);
     const uint32_t cml_r = smem_u32(cml) + (uint32_t)(crank * 8);
     const uint32_t sbar = smem_u32(state_bar);
     for (int e = tid; e < G * (D / 4); e += FD_THREADS) {
       const int h = e / (D / 4), c4 = (e % (D / 4)) * 4;
-      float M = -INFINITY;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
       for (int w = 0; w < FD_WARPS; ++w) {
-        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
-        if (ws[D + 1] > 0.f) M = fmaxf(M, ws[D]);
-      }
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, Ls = 0.f;
-      for (int w = 0; w < FD_WARPS; ++w) {
-        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
-        if (ws[D + 1] > 0.f) {
-          const float f = __expf(ws[D] - M);
-          Ls += ws[D + 1] * f;
-          a0 += ws[c4] * f;
-          a1 += ws[c4 + 1] * f;
-          a2 += ws[c4 + 2] * f;
-          a3 += ws[c4 + 3] * f;
-        }
+        const float* ws = wst + (size_t)(w * G + h) * (D + 2) + c4;
+        const float f = fw[h * 8 + w];
+        a0 += ws[0] * f;
+        a1 += ws[1] * f;
+        a2 += ws[2] * f;
+        a3 += ws[3] * f;
       }
       st_async_f32x4(mapa(cst_r + 4u * c4, h), a0, a1, a2, a3, mapa(sbar, h));
-      if (c4 == 0) st_async_f32x2(mapa(cml_r, h), M, Ls, mapa(sbar, h));
+      if (c4 == 0) st_async_f32x2(mapa(cml_r, h), fm[h], fl[h], mapa(sbar, h));
     }
   }
-  cluster_arrive_release();
+  cluster_arrive_relaxed();  // pairs with the wait at exit; carries no data
 
   // ---- 6. CTA h < G combines head h (exact LSE rescaling)
   if (crank < G) {
     mbar_wait_cluster(state_bar, 0, err);
+    if (wid == 0) {  // weights of the CS states, 1/L folded in
+      const bool ok = lane < CS && cml[2 * lane + 1] > 0.f;
+      const float m = ok ? cml[2 * lane] : -INFINITY;
+      const float M = warp_max(m);
+      const float f = ok ? __expf(m - M) : 0.f;
+      const float Ls = warp_sum(ok ? cml[2 * lane + 1] * f : 0.f);
+      if (lane < CS) cw[lane] = f / Ls;
+    }
+    __syncthreads();
     const int h = crank;
-    float M = -INFINITY;
-    for (int c = 0; c < CS; ++c)
-      if (cml[2 * c + 1] > 0.f) M = fmaxf(M, cml[2 * c]);
-    float Ls = 0.f;
-    for (int c = 0; c < CS; ++c)
-      if (cml[2 * c + 1] > 0.f) Ls += cml[2 * c + 1] * __expf(cml[2 * c] - M);
-    const float inv = 1.f / Ls;
     for (int col = tid; col < D; col += FD_THREADS) {
       float a = 0.f;
-      for (int c = 0; c < CS; ++c)
-        if (cml[2 * c + 1] > 0.f) a += cst[c * D + col] * __expf(cml[2 * c] - M);
-      o[((size_t)b * Hq + r * G + h) * D + col] = from_f<T>(a * inv);
+      for (int c = 0; c < CS; ++c) a += cst[c * D + col] * cw[c];
+      o[((size_t)b * Hq + r * G + h) * D + col] = from_f<T>(a);
     }
   }
   cluster_wait_acquire();  // no CTA leaves while stores into it may be pending

@@ -403,3 +403,66 @@ def decode_attend(q, kc, vc, lens, idx, cnt, logg, Hkv: int, gated: int = 1,
                 o[b, h] = (e / e.sum()) @ vr
                 lse[b, h] = mx + np.log(e.sum())
     return o, lse
+
+
+# --------------------------------------------------------------------------
+# Selector backward (section 2.3, eq. 8, sparse scope). The kept blocks'
+# log-gate gradients reach every visible block's score through the shared
+# normalisation log g = s - LSE(s); the parameter-free selector
+# s_m = scale * qbar . kbar_m then carries the score gradient to the query
+# and key means, and the means spread it over their rows.
+# --------------------------------------------------------------------------
+def select_backward(q, k, idx, cnt, dlogg, Hkv: int, scale: float | None = None,
+                    return_ds: bool = False):
+    """Gradient reaching q and k through the selector, given d(log g).
+
+    For each (b, kv group r, query block t) with C = t visible history blocks,
+    kept set I (the first cnt entries of idx) and g = softmax(s) over m < C:
+        ds_m = dlogg[slot of m] * [m in I]  -  g_m * sum_{l in I} dlogg[slot of l]
+    (eq. 8: for m outside I only the normalisation term remains). With
+    s_m = scale * qbar_t . kbar_m:
+        dqbar_t = scale * sum_m ds_m kbar_m,   dkbar_m += scale * ds_m qbar_t,
+    qbar_t being the mean over the group's G heads and the n_t rows of block t,
+    kbar_m the mean of block m's 64 keys; so each of those rows and heads gets
+    dqbar_t / (G n_t) and each of block m's keys gets dkbar_m / 64.
+    Returns (dq_sel [B][Hq][N][d], dk_sel [B][Hkv][N][d]) and, with
+    return_ds, the ds rows {(b, r, t): ds[0..C-1]}. All in float64.
+    """
+    q, k, dlogg = _f64(q), _f64(k), _f64(dlogg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    T = -(-N // BLOCK)
+    scale = _scale(d, scale)
+    ksum = block_summary(k)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    ds_rows = {}
+    for b in range(B):
+        for r in range(Hkv):
+            dkbar = np.zeros((ksum.shape[2], d))
+            for t in range(T):
+                C = t
+                if C == 0:
+                    continue
+                r0, r1 = t * BLOCK, min(N, (t + 1) * BLOCK)
+                rows = q[b, r * G:(r + 1) * G, r0:r1]
+                qbar = rows.reshape(-1, d).mean(axis=0)
+                s = scale * (ksum[b, r, :C] @ qbar)
+                g = np.exp(s - s.max())
+                g = g / g.sum()
+                kk = int(cnt[b, r, t])
+                kept = [int(m) for m in idx[b, r, t, :kk]]
+                total = sum(dlogg[b, r, t, j] for j in range(kk))
+                ds = -g * total
+                for j, m in enumerate(kept):
+                    ds[m] += dlogg[b, r, t, j]
+                ds_rows[(b, r, t)] = ds
+                dqbar = scale * (ds @ ksum[b, r, :C])
+                dq[b, r * G:(r + 1) * G, r0:r1] += dqbar / (G * (r1 - r0))
+                dkbar[:C] += scale * np.outer(ds, qbar)
+            for m in range(dkbar.shape[0]):
+                dk[b, r, m * BLOCK:(m + 1) * BLOCK] += dkbar[m] / BLOCK
+    if return_ds:
+        return dq, dk, ds_rows
+    return dq, dk

@@ -423,3 +423,79 @@ def test_stored_output_form_of_D():
                        o_stored=lambda rows: inputs.to_storage(rows, "bf16").double().numpy())
     for a, b in zip(moved, as_fn):
         assert np.abs(a - b).max() < 1e-13
+
+
+# ---------------------------------------------------------------- selector backward pins
+def _gated_loss(q, k, v, do, idx, cnt, Hkv):
+    """L(q, k) = sum(dO * o) with the selection (idx, cnt) held fixed and the
+    gate recomputed from q and k through the selector (summaries, scores,
+    log g = s - LSE(s) by the oracle's gate), then gated attention."""
+    ks = O.block_summary(k)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    T = -(-N // BLOCK)
+    scale = 1.0 / np.sqrt(d)
+    logg = np.zeros(idx.shape)
+    for b in range(B):
+        for r in range(Hkv):
+            for t in range(1, T):
+                rows = q[b, r * G:(r + 1) * G, t * BLOCK:min(N, (t + 1) * BLOCK)]
+                s = scale * (ks[b, r, :t] @ rows.reshape(-1, d).mean(axis=0))
+                _, _, logg_all = O.gate_and_topk(s, 1)
+                for j in range(int(cnt[b, r, t])):
+                    logg[b, r, t, j] = logg_all[idx[b, r, t, j]]
+    o, _ = O.attn_fwd(q, k, v, idx, cnt, logg)
+    return (o * do).sum(), logg
+
+
+def test_selector_backward_central_finite_differences():
+    """Attention backward + selector backward (eq. 8 through the parameter-free
+    selector) = the numerical gradient of the loss with the selection fixed;
+    the attention part alone does not match."""
+    Hkv = 2
+    q, k, v, do, idx, cnt, logg = _sparse_case(80, N=256, d=8, Hq=4, Hkv=Hkv, topk=2)
+    _, logg0 = _gated_loss(q, k, v, do, idx, cnt, Hkv)
+    assert np.abs(logg0 - logg).max() < 1e-12  # the selection's own gate
+    dq_a, dk_a, _, dlogg = O.attn_bwd(q, k, v, do, idx, cnt, logg)
+    dq_s, dk_s = O.select_backward(q, k, idx, cnt, dlogg, Hkv)
+    grads = {"q": dq_a + dq_s, "k": dk_a + dk_s}
+    alone = {"q": dq_a, "k": dk_a}
+    h = 1e-5
+    probes = [("q", (0, 1, 150, 3)), ("q", (0, 3, 70, 0)), ("q", (0, 2, 200, 5)),
+              ("k", (0, 0, 10, 5)), ("k", (0, 1, 130, 2)), ("k", (0, 1, 70, 7))]
+    misses = 0
+    for name, ix in probes:
+        args = dict(q=q, k=k)
+        xp, xm = args[name].copy(), args[name].copy()
+        xp[ix] += h
+        xm[ix] -= h
+        lp, _ = _gated_loss(**{**args, name: xp}, v=v, do=do, idx=idx, cnt=cnt, Hkv=Hkv)
+        lm, _ = _gated_loss(**{**args, name: xm}, v=v, do=do, idx=idx, cnt=cnt, Hkv=Hkv)
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - grads[name][ix]) <= 1e-7 * max(1.0, abs(fd)), (name, ix, fd, grads[name][ix])
+        misses += abs(fd - alone[name][ix]) > 1e-6 * max(1.0, abs(fd))
+    assert misses >= 4  # the selector's share is visible at most probes
+
+
+def test_selector_backward_eq8_structure():
+    """Per row: the score gradients sum to zero (softmax normalisation), and
+    every block outside the kept set gets -g_m times the kept gradients' sum
+    (eq. 8, sparse scope)."""
+    Hkv = 2
+    q, k, v, do, idx, cnt, logg = _sparse_case(81, N=512, d=16, Hq=4, Hkv=Hkv, topk=3)
+    _, _, _, dlogg = O.attn_bwd(q, k, v, do, idx, cnt, logg)
+    _, _, ds_rows = O.select_backward(q, k, idx, cnt, dlogg, Hkv, return_ds=True)
+    ks = O.block_summary(k)
+    assert len(ds_rows) == Hkv * 7
+    for (b, r, t), ds in ds_rows.items():
+        assert abs(ds.sum()) < 1e-12
+        qbar = q[b, r * 2:(r + 1) * 2, t * BLOCK:(t + 1) * BLOCK].reshape(-1, 16).mean(axis=0)
+        s = (ks[b, r, :t] @ qbar) / 4.0
+        g = np.exp(s - s.max())
+        g /= g.sum()
+        kk = int(cnt[b, r, t])
+        kept = set(int(m) for m in idx[b, r, t, :kk])
+        total = dlogg[b, r, t, :kk].sum()
+        for m in range(t):
+            if m not in kept:
+                assert abs(ds[m] + g[m] * total) < 1e-12

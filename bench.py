@@ -414,6 +414,8 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
                          dtype=torch.uint8, device=dev)
     bwd_ws = torch.empty(max(16, lib.sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt)),
                          dtype=torch.uint8, device=dev)
+    sbw_ws = torch.empty(max(16, lib.sas_select_bwd_workspace_size(B, Hq, Hkv, N, d)),
+                         dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
 
@@ -422,6 +424,8 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
         sas.sas_select(q, ks, Hkv, topk, "prefill", out=(idx, cnt, logg), ws=sel_ws)
         sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
         sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+        # the gradient through the selector (eq. 8), added into dq and dk
+        sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
 
     K, W = args.steps, args.warmup
     ms, clk = timed_graphs(step, K, W, world, stream, chunk=8, clocks=clocks)
@@ -433,8 +437,12 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
     def bwd_step(i):
         sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
 
+    def sbw_step(i):
+        sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
+
     ms_f, _ = timed_graphs(fwd_step, max(3, K), 2, world, stream, chunk=8)
     ms_b, _ = timed_graphs(bwd_step, max(3, K), 2, world, stream, chunk=8)
+    ms_s, _ = timed_graphs(sbw_step, max(3, K), 2, world, stream, chunk=8)
     tf, tb = ms_f / max(3, K) * 1e-3, ms_b / max(3, K) * 1e-3
     peaks = measured_peaks()
     tensor = c["dtype"] == "bf16" and d == 128 and (Hq // Hkv) % 2 == 0
@@ -456,7 +464,8 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
             "traffic": recorded_traffic(kern, srcs[i]), "peak_source": psrc,
             "algorithmic_flops_per_launch": kf, "launch_ms": round(kt * 1e3, 4),
             "fwd_ms": round(tf * 1e3, 4), "bwd_ms": round(tb * 1e3, 4),
-            "fwd_tflops": round(f_fwd / tf / 1e12, 2), "bwd_tflops": round(f_bwd / tb / 1e12, 2)}
+            "fwd_tflops": round(f_fwd / tf / 1e12, 2), "bwd_tflops": round(f_bwd / tb / 1e12, 2),
+            "select_bwd_ms": round(ms_s / max(3, K), 4)}
 
     # end to end: pinned host inputs in, gradients out
     pin = {n: torch.empty(h[n].shape, dtype=h[n].dtype, pin_memory=True) for n in ("q", "k", "v", "do")}
@@ -494,7 +503,9 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
         "roofline": roof,
         "e2e": {"value": round(total * E * world / (ms_e2e * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 7 * K,  # summary, query means, selection, forward, backward, 2 conversions
+        # summary, query means, selection, forward, backward, 2 conversions,
+        # selector backward (query means, rows, columns)
+        "gpu_launches": 10 * K,
         "clocks": clk,
     }
 

@@ -329,6 +329,37 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                      "sas_decode launch");
 }
 
+// ---------------------------------------------------------------- selector backward
+size_t sas_select_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  (void)Hq;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return 0;
+  return a16(sas::select_bwd_ws_bytes(B, Hkv, N, d));
+}
+
+sas_status sas_select_bwd(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
+                          int N, int d, int topk, float scale, const int32_t* idx,
+                          const int32_t* cnt, const float* dlogg, void* dq, void* dk, void* ws,
+                          size_t ws_bytes, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N == 0 || topk == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(idx);
+  REQUIRE_PTR(cnt);
+  REQUIRE_PTR(dlogg);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  const size_t need = sas_select_bwd_workspace_size(B, Hq, Hkv, N, d);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  return cuda_status(sas::launch_select_bwd(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
+                                            resolve_scale(scale, d), idx, cnt, dlogg, dq, dk, ws,
+                                            (cudaStream_t)stream),
+                     "sas_select_bwd launch");
+}
+
 // ---------------------------------------------------------------- device status
 sas_status sas_device_status(int clear, sas_stream_t stream) {
   g_last_error.clear();

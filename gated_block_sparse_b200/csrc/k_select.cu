@@ -223,6 +223,22 @@ static size_t prefill_select_smem(int d, int nchunk, int topk) {
   return n * 4 + 8;
 }
 
+cudaError_t launch_qbar_prefill(const void* q, int bf16, int B, int Hq, int Hkv, int N, int d,
+                                float* qbar, cudaStream_t st) {
+  const int T_ = (N + SAS_BLOCK - 1) / SAS_BLOCK;
+  if (B == 0 || T_ == 0) return cudaSuccess;
+  dim3 grid(T_, Hkv, B);
+#define SAS_QBAR(T, D) \
+  k_qbar_prefill<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(q), Hq, Hkv, N, qbar)
+  if (bf16) {
+    if (d == 128) SAS_QBAR(__nv_bfloat16, 128); else SAS_QBAR(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) SAS_QBAR(float, 128); else SAS_QBAR(float, 64);
+  }
+#undef SAS_QBAR
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
                                   int Hkv, int N, int d, int topk, float scale, int32_t* idx,
                                   int32_t* cnt, float* logg, void* ws, cudaStream_t st) {

@@ -35,6 +35,18 @@ cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, in
                                   int Hkv, int N, int d, int topk, float scale, int32_t* idx,
                                   int32_t* cnt, float* logg, void* ws, cudaStream_t st);
 size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d);
+// Query means of the prefill selector, qbar [B][Hkv][T][d] fp32.
+cudaError_t launch_qbar_prefill(const void* q, int bf16, int B, int Hq, int Hkv, int N, int d,
+                                float* qbar, cudaStream_t st);
+
+// ---- selector backward (k_select_bwd.cu)
+// Adds the gradient that reaches q and k through the selector (eq. 8 of the
+// gate, then s = scale qbar . kbar) into dq and dk. ws: qbar and the ds rows.
+size_t select_bwd_ws_bytes(int B, int Hkv, int N, int d);
+cudaError_t launch_select_bwd(const void* q, int bf16, const float* ksum, int B, int Hq, int Hkv,
+                              int N, int d, int topk, float scale, const int32_t* idx,
+                              const int32_t* cnt, const float* dlogg, void* dq, void* dk,
+                              void* ws, cudaStream_t st);
 // Prefill selection with its query-summary scratch in a fixed device array
 // of the library (no workspace argument); capacity in fp32 values.
 size_t select_prefill_static_capacity();

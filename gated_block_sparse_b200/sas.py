@@ -43,6 +43,9 @@ SIGNATURES = {
                                _P, _P, _Z, _P]),
     "sas_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P, _P, _Z,
                         _P]),
+    "sas_select_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "sas_select_bwd": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _Z,
+                            _P]),
     "sas_device_status": (_I, [_I, _P]),
     "sas_debug_wait_timeout": (_I, [_P]),
 }
@@ -248,6 +251,20 @@ def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: fl
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
         float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
     return out
+
+
+def sas_select_bwd(q, ksum, Hkv: int, idx, cnt, dlogg, dq, dk, scale: float = 0.0, ws=None,
+                   stream=None):
+    """Add the gradient through the selector (eq. 8 of the gate) into dq and dk, in place."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    topk = idx.shape[-1]
+    need = lib.sas_select_bwd_workspace_size(B, Hq, Hkv, N, d)
+    w = _ws(need, q.device, ws)
+    _check("sas_select_bwd", lib.sas_select_bwd(
+        _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, float(scale), _ptr(idx), _ptr(cnt),
+        _ptr(dlogg), _ptr(dq), _ptr(dk), _ptr(w), w.numel(), _stream(stream)))
+    return dq, dk
 
 
 def sas_device_status(clear: bool = False, stream=None) -> tuple[int, str]:

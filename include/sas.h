@@ -215,6 +215,29 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              sas_stream_t stream);
 
 /*
+ * Selector backward (SAS close reading, section 2.3, eq. 8, sparse scope),
+ * prefill rows: the gradient that reaches q and k through the selector,
+ * ADDED into dq and dk (typically the outputs of sas_attn_bwd, so the two
+ * calls give the full gradient). For each (b, r, t) with C = t visible
+ * history blocks, kept set I (idx, cnt) and g = softmax(s):
+ *   ds_m = dlogg[slot of m] [m in I] - g_m * sum_{l in I} dlogg[slot of l],
+ * then with s_m = scale * qbar_t . kbar_m (the parameter-free selector of
+ * sas_select): every row of block t and head of group r gets
+ * scale * sum_m ds_m kbar_m / (G n_t), and every key of block m gets
+ * scale * sum_t ds_tm qbar_t / 64.
+ *   q      [B][Hq][N][d], dt          ksum  [B][Hkv][N/64][d] fp32 (summaries)
+ *   idx, cnt, dlogg                   as sas_select / sas_attn_bwd (prefill rows)
+ *   dq     [B][Hq][N][d], dt (in/out) dk    [B][Hkv][N][d], dt (in/out)
+ *   ws     sas_select_bwd_workspace_size() bytes (query means and ds rows)
+ * topk = 0 or N <= 64 leave dq and dk unchanged.
+ */
+size_t sas_select_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
+sas_status sas_select_bwd(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
+                          int N, int d, int topk, float scale, const int32_t* idx,
+                          const int32_t* cnt, const float* dlogg, void* dq, void* dk, void* ws,
+                          size_t ws_bytes, sas_stream_t stream);
+
+/*
  * Device status. Kernels never trap: every wait on an mbarrier is bounded in
  * wall-clock time (200 ms); a wait that gives up, or a selection index out of
  * range (replaced by the current block), sets a bit in a per-kernel error

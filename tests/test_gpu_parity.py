@@ -331,3 +331,58 @@ def test_decode_attend_forced_selection():
         ref, _ = O.decode_attend(x["q"], x["kc"], x["vc"], x["lens"].numpy(), idx, cnt, logg,
                                  Hkv, gated=gated)
         assert excess(np64(o), ref, 2e-2, True) <= 0
+
+
+# ---------------------------------------------------------------- selector backward
+def _select_bwd_case(B, Hq, Hkv, N, d, dtype, topk, seed):
+    x = inputs.gen_prefill(B, Hq, Hkv, N, d, dtype, seed=seed)
+    q, k = x["q"], x["k"]
+    ks_ref = O.block_summary(k)
+    idx, cnt, _, _ = O.select_prefill(q, ks_ref, Hkv, topk)
+    T = -(-N // 64)
+    rng = np.random.Generator(np.random.PCG64(seed + 7))
+    dlogg = rng.standard_normal((B, Hkv, T, topk)).astype(np.float32)
+    for b in range(B):  # slots past cnt carry no gradient
+        for r in range(Hkv):
+            for t in range(T):
+                dlogg[b, r, t, cnt[b, r, t]:] = 0.0
+    dq_ref, dk_ref = O.select_backward(q, k, idx, cnt, dlogg, Hkv)
+    return q, k, idx, cnt, dlogg, dq_ref, dk_ref
+
+
+@pytest.mark.parametrize("N,d", [(512, 64), (1000, 128)])
+def test_select_bwd_fp32(N, d):
+    """Eq. 8 through the selector, fp32: relative error at fp32 accumulation level."""
+    q, k, idx, cnt, dlogg, dq_ref, dk_ref = _select_bwd_case(2, 8, 2, N, d, "f32", 3, 90 + N)
+    qd, kd = q.to(DEV), k.to(DEV)
+    ks = sas.sas_block_summary(kd)
+    dq = torch.zeros_like(qd)
+    dk = torch.zeros_like(kd)
+    sas.sas_select_bwd(qd, ks, 2, torch.from_numpy(idx).to(DEV), torch.from_numpy(cnt).to(DEV),
+                       torch.from_numpy(dlogg).to(DEV), dq, dk)
+    torch.cuda.synchronize()
+    for got, ref in ((dq, dq_ref), (dk, dk_ref)):
+        g = got.double().cpu().numpy()
+        scale_ = np.abs(ref).max()
+        assert scale_ > 0
+        assert np.abs(g - ref).max() <= 1e-5 * scale_ + 1e-7, np.abs(g - ref).max() / scale_
+
+
+def test_select_bwd_bf16_adds_in_place():
+    """bf16 ragged case; dq and dk start from nonzero values and receive the
+    selector's gradient added in place (one bf16 rounding of the sum)."""
+    B, Hq, Hkv, N, d = 1, 8, 2, 1000, 128
+    q, k, idx, cnt, dlogg, dq_ref, dk_ref = _select_bwd_case(B, Hq, Hkv, N, d, "bf16", 3, 95)
+    qd, kd = q.to(DEV), k.to(DEV)
+    ks = sas.sas_block_summary(kd)
+    g0 = torch.Generator().manual_seed(5)
+    dq0 = (torch.randn(q.shape, generator=g0) * 1e-2).to(torch.bfloat16)
+    dk0 = (torch.randn(k.shape, generator=g0) * 1e-2).to(torch.bfloat16)
+    dq, dk = dq0.to(DEV), dk0.to(DEV)
+    sas.sas_select_bwd(qd, ks, Hkv, torch.from_numpy(idx).to(DEV), torch.from_numpy(cnt).to(DEV),
+                       torch.from_numpy(dlogg).to(DEV), dq, dk)
+    torch.cuda.synchronize()
+    for got, init, ref in ((dq, dq0, dq_ref), (dk, dk0, dk_ref)):
+        want = init.double().numpy() + ref
+        g = got.double().cpu().numpy()
+        assert np.abs(g - want).max() <= 2.0 ** -8 * np.abs(want).max() + 1e-6

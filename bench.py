@@ -125,35 +125,18 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus: int):
-    import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return world, rank, local
+    from gated_block_sparse_b200 import dist as D
+    return D.setup()
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from gated_block_sparse_b200 import dist as D
+    D.barrier(world)
 
 
 def max_over_ranks(world, x: float) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from gated_block_sparse_b200 import dist as D
+    return D.max_over_ranks(world, x)
 
 
 def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: int = 512,
@@ -330,7 +313,8 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
     nb = q.numel() * q.element_size()
 
-    value = w.step_bytes * K * world / (ms * 1e-3) / 1e9
+    from gated_block_sparse_b200 import dist as D
+    value = D.whole_job_rate(w.step_bytes * K, world, ms) / 1e9
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
@@ -394,6 +378,7 @@ def prefill_flops(idx_cnt, N: int, Hq: int, Hkv: int, d: int):
 def bench_prefill_ours(args, world, rank, local) -> dict:
     import torch
 
+    from gated_block_sparse_b200 import dist as D
     from gated_block_sparse_b200 import inputs, sas
     name = args.config
     c = inputs.CONFIGS[name]
@@ -492,7 +477,7 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
     d2h = sum(t.numel() * t.element_size() for t in outs)
     total = f_fwd + f_bwd
     return {
-        "metric": METRIC, "value": round(total * K * world / (ms * 1e-3) / 1e12, 4),
+        "metric": METRIC, "value": round(D.whole_job_rate(total * K, world, ms) / 1e12, 4),
         "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if c["dtype"] == "bf16" else "f32", "data": "synthetic (seeded N(0,1), planted)",
@@ -587,9 +572,8 @@ def main():
         res["cpu_baseline"] = (cpu_baseline_decode(args.config, args.cpu_seconds, w) if decode
                                else cpu_baseline_prefill(args.config, args.cpu_seconds))
         print(json.dumps(res))
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    from gated_block_sparse_b200 import dist as D
+    D.teardown(world)
 
 
 if __name__ == "__main__":

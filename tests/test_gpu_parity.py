@@ -386,3 +386,28 @@ def test_select_bwd_bf16_adds_in_place():
         want = init.double().numpy() + ref
         g = got.double().cpu().numpy()
         assert np.abs(g - want).max() <= 2.0 ** -8 * np.abs(want).max() + 1e-6
+
+
+def test_select_bwd_c3_full():
+    """Selector backward on the full c3 workload, in the step's configuration
+    (after the GPU selection and attention backward): every element of the
+    selector's share of dq and dk against the oracle, given the GPU's dlogg."""
+    c = inputs.CONFIGS["c3"]
+    x = inputs.gen_config("c3")
+    q, k = x["q"], x["k"]
+    qd, kd = dev(q), dev(k)
+    ks = sas.sas_block_summary(kd)
+    ti, tc, tl = sas.sas_select(qd, ks, c["Hkv"], c["topk"], "prefill")
+    T = tl.shape[2]
+    g = torch.Generator().manual_seed(11)
+    dlogg = torch.randn(tl.shape, generator=g)  # both sides use only slots below cnt
+    dq = torch.zeros_like(qd)
+    dk = torch.zeros_like(kd)
+    sas.sas_select_bwd(qd, ks, c["Hkv"], ti, tc, dlogg.to(DEV), dq, dk)
+    torch.cuda.synchronize()
+    dq_ref, dk_ref = O.select_backward(q, k, ti.cpu().numpy(), tc.cpu().numpy(),
+                                       dlogg.numpy(), c["Hkv"])
+    assert T == 256
+    for got, ref in ((dq, dq_ref), (dk, dk_ref)):
+        gg = got.double().cpu().numpy()
+        assert np.abs(gg - ref).max() <= 2.0 ** -8 * np.abs(ref).max() + 1e-6

@@ -238,6 +238,21 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
         vcs.append(vc0.clone())
         kss.append(ks0.clone())
     topk, Hkv = c["topk"], c["Hkv"]
+    bt = None
+    if args.paged:  # the same caches scattered into 64-token pages, random page order
+        B_, _, Lmax_, d_ = kc0.shape
+        nblk = Lmax_ // 64
+        perm = torch.randperm(B_ * nblk, generator=torch.Generator().manual_seed(12345)).to(dev)
+        bt = perm.view(B_, nblk).to(torch.int32).contiguous()
+
+        def pages(x):
+            p = torch.empty((B_ * nblk, Hkv, 64, d_), dtype=x.dtype, device=dev)
+            p[perm] = x.view(B_, Hkv, nblk, 64, d_).permute(0, 2, 1, 3, 4).reshape(
+                B_ * nblk, Hkv, 64, d_)
+            return p
+        for j in range(L):
+            kcs[j], vcs[j] = pages(kcs[j]), pages(vcs[j])
+            kss[j] = sas.sas_block_summary(kcs[j]).view(B_ * nblk, Hkv, d_)
     o = torch.empty_like(q)
     ws = torch.empty(sas.sas_decode_workspace_size(c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk),
                      dtype=torch.uint8, device=dev)
@@ -245,14 +260,44 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     K, W = args.steps, args.warmup
 
+    def decode(j, qq, out):
+        if bt is not None:
+            sas.sas_decode_paged(qq, kcs[j], vcs[j], kss[j], bt, lens, topk, gated=c["gated"],
+                                 out=out)
+        else:
+            sas.sas_decode(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out,
+                           ws=ws)
+
     def step(i):
-        j = i % L
-        sas.sas_decode(q, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=o, ws=ws)
+        decode(i % L, q, o)
 
     ms, clk = timed_graphs(step, K, W, world, stream, clocks=clocks)
     clocks.stop()
 
-    # per-kernel timing for the roofline: selection alone, attention alone
+    # split path (contiguous caches only): selection alone, attention alone
+    split = None
+    if bt is None:
+        split = split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
+    peaks = measured_peaks()
+    # the step is one launch of the cluster kernel: its duration is the step's
+    kt = ms / K * 1e-3
+    ach = w.step_bytes / kt / 1e9
+    roof = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(ach, 1),
+            "peak": peaks["hbm"], "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
+            "traffic": recorded_traffic("k_decode_fused", "k_decode_fused.cu"),
+            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+            "algorithmic_bytes_per_launch": w.step_bytes, "launch_us": round(kt * 1e6, 3),
+            "selected_kv_bytes_per_launch": w.att_bytes, "split_path": split}
+    if bt is not None:
+        roof["traffic"] = None  # the ncu record is of the contiguous layout
+    return finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode,
+                         ms, clk, roof, l2, bt is not None)
+
+
+def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o):
+    import torch
+    dev = q.device
+    topk, Hkv = c["topk"], c["Hkv"]
     sel = [sas.sas_select(q, kss[j], Hkv, topk, "decode", lens=lens) for j in range(L)]
     sel_ws = torch.empty(max(16, sas.load_library().sas_select_workspace_size(
         c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk, 1)), dtype=torch.uint8, device=dev)
@@ -272,21 +317,17 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     ms_sel, _ = timed_graphs(sel_step, Kk, 10, world, stream)
     ms_att, _ = timed_graphs(att_step, Kk, 10, world, stream)
     t_sel, t_att = ms_sel / Kk * 1e-3, ms_att / Kk * 1e-3
-    peaks = measured_peaks()
-    # the step is one launch of the cluster kernel: its duration is the step's
-    kt = ms / K * 1e-3
-    ach = w.step_bytes / kt / 1e9
-    roof = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(ach, 1),
-            "peak": peaks["hbm"], "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
-            "traffic": recorded_traffic("k_decode_fused", "k_decode_fused.cu"),
-            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
-            "algorithmic_bytes_per_launch": w.step_bytes, "launch_us": round(kt * 1e6, 3),
-            "selected_kv_bytes_per_launch": w.att_bytes,
-            "split_path": {"k_select_decode": {"us": round(t_sel * 1e6, 3),
-                                               "GBps": round(w.sel_bytes / t_sel / 1e9, 1)},
-                           "k_decode_attend": {"us": round(t_att * 1e6, 3),
-                                               "GBps": round(w.att_bytes / t_att / 1e9, 1)}}}
+    return {"k_select_decode": {"us": round(t_sel * 1e6, 3),
+                                "GBps": round(w.sel_bytes / t_sel / 1e9, 1)},
+            "k_decode_attend": {"us": round(t_att * 1e6, 3),
+                                "GBps": round(w.att_bytes / t_att / 1e9, 1)}}
 
+
+def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode, ms, clk,
+                  roof, l2, paged) -> dict:
+    import torch
+
+    from gated_block_sparse_b200 import dist as D
     # end to end through the public API: pinned host q in, o out, every step
     qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     qh.copy_(q.cpu())
@@ -296,8 +337,7 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     with torch.cuda.stream(stream):
         for i in range(20):
             qd.copy_(qh, non_blocking=True)
-            sas.sas_decode(qd, kcs[i % L], vcs[i % L], lens, kss[i % L], topk, gated=c["gated"],
-                           out=o, ws=ws)
+            decode(i % L, qd, o)
             oh.copy_(o, non_blocking=True)
         torch.cuda.synchronize()
         barrier(world)
@@ -305,32 +345,31 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
         e0.record(stream)
         for i in range(E):
             qd.copy_(qh, non_blocking=True)
-            sas.sas_decode(qd, kcs[i % L], vcs[i % L], lens, kss[i % L], topk, gated=c["gated"],
-                           out=o, ws=ws)
+            decode(i % L, qd, o)
             oh.copy_(o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
     ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
     nb = q.numel() * q.element_size()
-
-    from gated_block_sparse_b200 import dist as D
+    api = "sas_decode_paged" if paged else "sas_decode"
     value = D.whole_job_rate(w.step_bytes * K, world, ms) / 1e9
-    res = {
+    return {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if c["dtype"] == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) with planted relevant blocks)",
         "config": {**w.describe(), "parallelism": f"replicas x{world}",
+                   "cache": ("paged: 64-token pages in a random page order" if paged
+                             else "contiguous [B][Hkv][Lmax][d]"),
                    "l2": f"rotating {L} layer copies of cache + summaries "
                          f"({w.step_bytes * L / 1e6:.0f} MB touched per rotation, L2 {l2 / 1e6:.0f} MB)"},
         "roofline": roof,
-        "e2e": {"value": round(w.step_bytes * E * world / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb,
-                "path": "pinned host q -> sas_decode (Python binding, C ABI) -> pinned host o"},
+        "e2e": {"value": round(D.whole_job_rate(w.step_bytes * E, world, ms_e2e) / 1e9, 2),
+                "unit": "GB/s", "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb,
+                "path": f"pinned host q -> {api} (Python binding, C ABI) -> pinned host o"},
         "gpu_launches": K,
         "clocks": clk,
     }
-    return res
 
 
 def one_thread():
@@ -536,6 +575,8 @@ def main():
     ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--paged", action="store_true",
+                    help="decode: read the caches through 64-token pages (sas_decode_paged)")
     ap.add_argument("--layers", type=int, default=0,
                     help="decode: number of rotated layer copies (default: enough for 3x L2)")
     args = ap.parse_args()

@@ -329,6 +329,34 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                      "sas_decode launch");
 }
 
+// ---------------------------------------------------------------- paged decode
+sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
+                            const float* kspool, sas_dtype dt, int B, int Hq, int Hkv, int npages,
+                            int d, const int32_t* block_table, int max_blocks,
+                            const int32_t* lens, int topk, int gated, float scale, void* o,
+                            int32_t* idx_out, sas_stream_t stream) {
+  g_last_error.clear();
+  REQUIRE(max_blocks >= 1 && max_blocks <= (1 << 24), SAS_ERR_INVALID_ARG,
+          "max_blocks must be in [1, 2^24] (got %d)", max_blocks);
+  sas_status s = check_decode(dt, B, Hq, Hkv, max_blocks * 64, d, topk, gated);
+  if (s != SAS_OK) return s;
+  REQUIRE(npages >= 1, SAS_ERR_INVALID_ARG, "npages must be >= 1 (got %d)", npages);
+  if (B == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kpool);
+  REQUIRE_PTR(vpool);
+  REQUIRE_PTR(kspool);
+  REQUIRE_PTR(block_table);
+  REQUIRE_PTR(lens);
+  REQUIRE_PTR(o);
+  if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
+  return cuda_status(sas::launch_decode_paged(q, kpool, vpool, dt == SAS_BF16, B, Hq, Hkv, npages,
+                                              d, block_table, max_blocks, lens, kspool, topk,
+                                              gated, resolve_scale(scale, d), o, idx_out,
+                                              (cudaStream_t)stream),
+                     "sas_decode_paged launch");
+}
+
 // ---------------------------------------------------------------- selector backward
 size_t sas_select_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   (void)Hq;

@@ -166,11 +166,16 @@ __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2)
 
 }  // namespace
 
-template <typename T, int D, int G>
+// PAGED: the caches are pools of 64-token pages, [npages][Hkv][64][D], the
+// summaries [npages][Hkv][D], and bt [B][max_blocks] maps a sequence's
+// logical block to its page (Lmax = 64 max_blocks). Otherwise kc, vc are
+// [B][Hkv][Lmax][D] and ksum [B][Hkv][Lmax/64][D].
+template <typename T, int D, int G, bool PAGED>
 __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
     const float* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
-    int gated, float scale, int per_max, T* __restrict__ o, int32_t* __restrict__ idx_out) {
+    int gated, float scale, int per_max, T* __restrict__ o, int32_t* __restrict__ idx_out,
+    const int32_t* __restrict__ bt, int npages) {
   constexpr int TILE = SAS_BLOCK * D;
   constexpr int VEC = Vec16<T>::N;     // elements per 16-byte vector
   constexpr int NCHK = D / (4 * VEC);  // 16-byte chunks of a key row per lane (4 lanes per key)
@@ -243,6 +248,37 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const size_t kvrow = row * (size_t)Lmax * D;
   const float* ks_row = ksum + row * (size_t)nblk * D;
   uint32_t* err = &g_decode_fused_err;
+  const int32_t* bt_row = PAGED ? bt + (size_t)b * nblk : nullptr;
+  // page of logical block m (paged caches); an out-of-range entry is flagged
+  // and replaced by page 0, so every copy stays inside the pools
+  auto page_of = [&](int m) -> int {
+    int p = bt_row[m];
+    if (p < 0 || p >= npages) {
+      atomicOr(err, kErrBadIndex);
+      p = 0;
+    }
+    return p;
+  };
+  // K (or V) tile of logical block blk
+  auto kv_tile = [&](const T* base, int blk) -> const T* {
+    if constexpr (PAGED) return base + ((size_t)page_of(blk) * Hkv + r) * TILE;
+    else return base + kvrow + (size_t)blk * TILE;
+  };
+  // summaries [first, first + cnt) of this CTA's range into ring slot `slot`:
+  // one bulk copy (contiguous), or one row copy per lane of warp 0 (paged)
+  auto issue_summaries = [&](int slot, int first, int cnt) {
+    float* dst = ring + (size_t)slot * FD_SUBC * D;
+    if constexpr (PAGED) {
+      if (lane == 0) mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * 4));
+      __syncwarp();
+      for (int j = lane; j < cnt; j += 32)
+        bulk_g2s(dst + (size_t)j * D, ksum + ((size_t)page_of(m0 + first + j) * Hkv + r) * D,
+                 (uint32_t)(D * 4), &sum_bar[slot]);
+    } else {
+      mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * 4));
+      bulk_g2s(dst, ks_row + (size_t)(m0 + first) * D, (uint32_t)(cnt * D * 4), &sum_bar[slot]);
+    }
+  };
 
   // ---- 0. barriers, expected remote bytes, first copies, q and qbar
   if (tid < CS) {
@@ -266,18 +302,16 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
     mbar_arrive_expect_tx(list_bar, lb);
     if (crank < G) mbar_arrive_expect_tx(state_bar, (uint32_t)CS * (D * 4 + 8));
-    for (int i = 0; i < min(FD_NS, nsub); ++i) {
-      const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
-      mbar_arrive_expect_tx(&sum_bar[i], (uint32_t)(cnt_i * D * 4));
-      bulk_g2s(ring + (size_t)i * FD_SUBC * D, ks_row + (size_t)(m0 + i * FD_SUBC) * D,
-               (uint32_t)(cnt_i * D * 4), &sum_bar[i]);
-    }
     if (own_cur) {  // the current block is unit 0 of this CTA's order, slot 0
       mbar_arrive_expect_tx(&full[0], (uint32_t)(2 * TILE * sizeof(T)));
-      bulk_g2s(U, kc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &full[0]);
-      bulk_g2s(U + TILE * sizeof(T), vc + kvrow + (size_t)t * TILE, TILE * sizeof(T), &full[0]);
+      bulk_g2s(U, kv_tile(kc, t), TILE * sizeof(T), &full[0]);
+      bulk_g2s(U + TILE * sizeof(T), kv_tile(vc, t), TILE * sizeof(T), &full[0]);
     }
   }
+  if (wid == 0) __syncwarp();  // lane 0 initialised the barriers
+  if (PAGED ? wid == 0 : tid == 0)
+    for (int i = 0; i < min(FD_NS, nsub); ++i)
+      issue_summaries(i, i * FD_SUBC, min(FD_SUBC, nmine - i * FD_SUBC));
   // Barriers are initialised and fenced (fence.mbarrier_init.release.cluster
   // above): other CTAs may store into this one once every thread of the
   // cluster has arrived. A relaxed arrive does not wait for this thread's
@@ -334,12 +368,9 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         }
       }
       __syncthreads();  // slot consumed
-      if (tid == 0 && i + FD_NS < nsub) {
-        const int cnt_n = min(FD_SUBC, nmine - (i + FD_NS) * FD_SUBC);
-        mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt_n * D * 4));
-        bulk_g2s(ring + (size_t)slot * FD_SUBC * D, ks_row + (size_t)(m0 + (i + FD_NS) * FD_SUBC) * D,
-                 (uint32_t)(cnt_n * D * 4), &sum_bar[slot]);
-      }
+      if ((PAGED ? wid == 0 : tid == 0) && i + FD_NS < nsub)
+        issue_summaries(slot, (i + FD_NS) * FD_SUBC,
+                        min(FD_SUBC, nmine - (i + FD_NS) * FD_SUBC));
     }
   }
 
@@ -449,9 +480,8 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const int slot = i % NKV;
     unsigned char* dst = U + (size_t)slot * kvslot;
     mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * TILE * sizeof(T)));
-    bulk_g2s(dst, kc + kvrow + (size_t)blk * TILE, TILE * sizeof(T), &full[slot]);
-    bulk_g2s(dst + TILE * sizeof(T), vc + kvrow + (size_t)blk * TILE, TILE * sizeof(T),
-             &full[slot]);
+    bulk_g2s(dst, kv_tile(kc, blk), TILE * sizeof(T), &full[slot]);
+    bulk_g2s(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), &full[slot]);
   };
   if (tid == 0)
     for (int i = own_cur ? 1 : 0; i < min(NKV, nu); ++i) issue_unit(i);
@@ -675,7 +705,7 @@ struct FdPick {
 // CTA h combines head h) whose clusters of all rows are co-resident on the
 // GPU; if none is, the largest that launches. Cached per shape, so repeated
 // launches make no occupancy queries.
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
   static std::mutex mu;
   static FdPick cache[32];
@@ -693,7 +723,7 @@ cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
         return cudaSuccess;
       }
   }
-  auto kern = k_decode_fused<T, D, G>;
+  auto kern = k_decode_fused<T, D, G, PAGED>;
   int best = 0, first = 0;
   const int cands[5] = {16, 8, 4, 2, 1};
   for (int ci = 0; ci < 5; ++ci) {
@@ -740,15 +770,16 @@ cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
   return cudaSuccess;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool PAGED>
 cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const float* ksum, int B,
                            int Hkv, int Lmax, const int32_t* lens, int topk, int gated, float scale,
-                           void* o, int32_t* idx_out, cudaStream_t st) {
-  auto kern = k_decode_fused<T, D, G>;
+                           void* o, int32_t* idx_out, const int32_t* bt, int npages,
+                           cudaStream_t st) {
+  auto kern = k_decode_fused<T, D, G, PAGED>;
   const int nblk = Lmax / SAS_BLOCK;
   const int kq = 1 << ceil_log2(topk > 0 ? topk : 1);
   int CS = 0;
-  cudaError_t e = pick_cluster<T, D, G>(B, Hkv, nblk, kq, CS);
+  cudaError_t e = pick_cluster<T, D, G, PAGED>(B, Hkv, nblk, kq, CS);
   if (e != cudaSuccess) return e;
   const int per_max = (nblk + CS - 1) / CS;
   const size_t smem = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS).total;
@@ -768,16 +799,19 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
                             static_cast<const T*>(vc), ksum, Hkv, Lmax, lens, topk, gated, scale,
-                            per_max, static_cast<T*>(o), idx_out);
+                            per_max, static_cast<T*>(o), idx_out, bt, npages);
 }
 
 template <typename T, int D>
 cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc, const float* ksum,
                            int B, int Hkv, int Lmax, const int32_t* lens, int topk, int gated,
-                           float scale, void* o, int32_t* idx_out, cudaStream_t st) {
+                           float scale, void* o, int32_t* idx_out, const int32_t* bt, int npages,
+                           cudaStream_t st) {
 #define SAS_FD(GG)                                                                              \
-  return launch_fused_t<T, D, GG>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale, o, \
-                                  idx_out, st)
+  return bt ? launch_fused_t<T, D, GG, true>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated,  \
+                                             scale, o, idx_out, bt, npages, st)                 \
+            : launch_fused_t<T, D, GG, false>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, \
+                                              scale, o, idx_out, nullptr, 0, st)
   switch (G) {
     case 1: SAS_FD(1);
     case 2: SAS_FD(2);
@@ -788,26 +822,43 @@ cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc,
 #undef SAS_FD
 }
 
+cudaError_t launch_fused(const void* q, const void* kc, const void* vc, int bf16, int B, int Hq,
+                         int Hkv, int Lmax, int d, const int32_t* lens, const float* ksum,
+                         int topk, int gated, float scale, void* o, int32_t* idx_out,
+                         const int32_t* bt, int npages, cudaStream_t st) {
+  if (B == 0) return cudaSuccess;
+  const int G = Hq / Hkv;
+  if (bf16) {
+    if (d == 128)
+      return launch_fused_g<__nv_bfloat16, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,
+                                                gated, scale, o, idx_out, bt, npages, st);
+    return launch_fused_g<__nv_bfloat16, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated,
+                                             scale, o, idx_out, bt, npages, st);
+  }
+  if (d == 128)
+    return launch_fused_g<float, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale,
+                                      o, idx_out, bt, npages, st);
+  return launch_fused_g<float, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale, o,
+                                   idx_out, bt, npages, st);
+}
+
 }  // namespace
 
 cudaError_t launch_decode_fused(const void* q, const void* kc, const void* vc, int bf16, int B,
                                 int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
                                 const float* ksum, int topk, int gated, float scale, void* o,
                                 int32_t* idx_out, cudaStream_t st) {
-  if (B == 0) return cudaSuccess;
-  const int G = Hq / Hkv;
-  if (bf16) {
-    if (d == 128)
-      return launch_fused_g<__nv_bfloat16, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,
-                                                gated, scale, o, idx_out, st);
-    return launch_fused_g<__nv_bfloat16, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated,
-                                             scale, o, idx_out, st);
-  }
-  if (d == 128)
-    return launch_fused_g<float, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale,
-                                      o, idx_out, st);
-  return launch_fused_g<float, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale, o,
-                                   idx_out, st);
+  return launch_fused(q, kc, vc, bf16, B, Hq, Hkv, Lmax, d, lens, ksum, topk, gated, scale, o,
+                      idx_out, nullptr, 0, st);
+}
+
+cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vpool, int bf16,
+                                int B, int Hq, int Hkv, int npages, int d,
+                                const int32_t* block_table, int max_blocks, const int32_t* lens,
+                                const float* kspool, int topk, int gated, float scale, void* o,
+                                int32_t* idx_out, cudaStream_t st) {
+  return launch_fused(q, kpool, vpool, bf16, B, Hq, Hkv, max_blocks * SAS_BLOCK, d, lens, kspool,
+                      topk, gated, scale, o, idx_out, block_table, npages, st);
 }
 
 uint32_t* decode_fused_error_word() {

@@ -43,6 +43,8 @@ SIGNATURES = {
                                _P, _P, _Z, _P]),
     "sas_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P, _P, _Z,
                         _P]),
+    "sas_decode_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I, _F,
+                              _P, _P, _P]),
     "sas_select_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sas_select_bwd": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _Z,
                             _P]),
@@ -250,6 +252,23 @@ def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: fl
         _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens),
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
         float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
+    return out
+
+
+def sas_decode_paged(q, kpool, vpool, kspool, block_table, lens, topk: int, gated: int = 1,
+                     scale: float = 0.0, out=None, idx_out=None, stream=None):
+    """Decode over paged caches: kpool, vpool [npages][Hkv][64][d], kspool
+    [npages][Hkv][d] fp32, block_table [B][max_blocks] -> o [B][Hq][d]."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    npages, Hkv = kpool.shape[0], kpool.shape[1]
+    max_blocks = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _check("sas_decode_paged", lib.sas_decode_paged(
+        _ptr(q), _ptr(kpool), _ptr(vpool), _ptr(kspool), _dt(q), B, Hq, Hkv, npages, d,
+        _ptr(block_table), max_blocks, _ptr(lens), topk, int(gated), float(scale), _ptr(out),
+        _ptr(idx_out), _stream(stream)))
     return out
 
 

@@ -215,6 +215,29 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              sas_stream_t stream);
 
 /*
+ * Decode over a paged cache (the serving layout of the pages' SGLang /
+ * FlashInfer setting; SAS close reading, section 2.4): as sas_decode, but
+ * the caches are pools of 64-token pages, one page per (block, kv head):
+ *   kpool, vpool  [npages][Hkv][64][d], dt
+ *   kspool        [npages][Hkv][d] fp32: the summary (mean of the 64 keys) of
+ *                 every full page; sas_block_summary over the pools viewed as
+ *                 [npages][Hkv][64][d] (B = npages, N = 64) computes it, and
+ *                 a serving loop refreshes it when a page fills
+ *   block_table   [B][max_blocks] int32: page of each logical 64-token block
+ *                 of sequence b (entries past ceil(lens[b]/64) unused;
+ *                 out-of-range ids are replaced by page 0 and flagged, see
+ *                 sas_device_status)
+ *   lens          [B] int32, 1 <= lens[b] <= 64 max_blocks
+ * idx_out holds logical block indices. Pages may be shared between
+ * sequences (read only). Needs no workspace.
+ */
+sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
+                            const float* kspool, sas_dtype dt, int B, int Hq, int Hkv, int npages,
+                            int d, const int32_t* block_table, int max_blocks,
+                            const int32_t* lens, int topk, int gated, float scale, void* o,
+                            int32_t* idx_out, sas_stream_t stream);
+
+/*
  * Selector backward (SAS close reading, section 2.3, eq. 8, sparse scope),
  * prefill rows: the gradient that reaches q and k through the selector,
  * ADDED into dq and dk (typically the outputs of sas_attn_bwd, so the two

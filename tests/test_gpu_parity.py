@@ -411,3 +411,60 @@ def test_select_bwd_c3_full():
     for got, ref in ((dq, dq_ref), (dk, dk_ref)):
         gg = got.double().cpu().numpy()
         assert np.abs(gg - ref).max() <= 2.0 ** -8 * np.abs(ref).max() + 1e-6
+
+
+# ---------------------------------------------------------------- paged decode
+def _to_pages(kc, vc, lens, seed, share_prefix=None):
+    """Scatter contiguous caches [B][Hkv][Lmax][d] into page pools
+    [npages][Hkv][64][d] under a random page order; share_prefix=(a, b, n)
+    makes sequence b's first n blocks use sequence a's pages."""
+    B, Hkv, Lmax, d = kc.shape
+    nblk = Lmax // 64
+    rng = np.random.Generator(np.random.PCG64(seed))
+    npages = B * nblk + 5  # a few pages no sequence uses
+    perm = rng.permutation(npages)
+    bt = np.zeros((B, nblk), dtype=np.int32)
+    kpool = torch.zeros((npages, Hkv, 64, d), dtype=kc.dtype)
+    vpool = torch.zeros_like(kpool)
+    nxt = 0
+    for b in range(B):
+        for m in range(nblk):
+            if share_prefix and b == share_prefix[1] and m < share_prefix[2]:
+                bt[b, m] = bt[share_prefix[0], m]
+                continue
+            p = int(perm[nxt])
+            nxt += 1
+            bt[b, m] = p
+            kpool[p] = kc[b, :, m * 64:(m + 1) * 64]
+            vpool[p] = vc[b, :, m * 64:(m + 1) * 64]
+    return kpool, vpool, bt
+
+
+@pytest.mark.parametrize("gated", [1, 0])
+def test_decode_paged_matches_contiguous_and_oracle(gated):
+    """Paged decode against the contiguous kernel (same arithmetic: identical
+    selection and output) and against the oracle on the gathered cache; one
+    sequence shares a 20-block prefix with another."""
+    B, Hq, Hkv, Lmax, d, topk = 3, 32, 8, 8192, 128, 15
+    x = inputs.gen_decode(B, Hq, Hkv, Lmax, d, [8192, 5000, 7777], "bf16", seed=71, planted=16)
+    q, kc, vc, lens = x["q"], x["kc"].clone(), x["vc"].clone(), x["lens"]
+    kc[2, :, :20 * 64] = kc[0, :, :20 * 64]  # the shared prefix has the same content
+    vc[2, :, :20 * 64] = vc[0, :, :20 * 64]
+    kpool, vpool, bt = _to_pages(kc, vc, lens, seed=72, share_prefix=(0, 2, 20))
+    kspool = sas.sas_block_summary(dev(kpool.view(-1, Hkv, 64, d))).view(-1, Hkv, d)
+    idx_p = torch.empty((B, Hkv, topk), dtype=torch.int32, device=DEV)
+    o_p = sas.sas_decode_paged(dev(q), dev(kpool), dev(vpool), kspool, dev(torch.from_numpy(bt)),
+                               dev(lens), topk, gated=gated, idx_out=idx_p)
+    ks = sas.sas_block_summary(dev(kc))
+    idx_c = torch.empty_like(idx_p)
+    o_c = sas.sas_decode(dev(q), dev(kc), dev(vc), dev(lens), ks, topk, gated=gated,
+                         idx_out=idx_c)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_p, idx_c)
+    assert torch.equal(o_p, o_c)
+    oks = O.block_summary(kc)
+    oo, oi, _, _ = O.decode(q, kc, vc, lens.numpy(), oks, Hkv, topk, gated=gated)
+    assert np.array_equal(idx_p.cpu().numpy(), oi)
+    assert excess(np64(o_p), oo, 2e-2, True) <= 0
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg

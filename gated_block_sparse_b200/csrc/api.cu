@@ -329,6 +329,46 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                      "sas_decode launch");
 }
 
+// ---------------------------------------------------------------- decode from host buffers
+sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, const void* vc,
+                           sas_dtype dt, int B, int Hq, int Hkv, int Lmax, int d,
+                           const int32_t* lens, const float* ksum, int topk, int gated,
+                           float scale, void* o_dev, void* o_host, int32_t* idx_out,
+                           sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_decode(dt, B, Hq, Hkv, Lmax, d, topk, gated);
+  if (s != SAS_OK) return s;
+  if (B == 0) return SAS_OK;
+  REQUIRE(q_host != nullptr && o_host != nullptr, SAS_ERR_INVALID_ARG,
+          "q_host and o_host must not be NULL");
+  REQUIRE_PTR(q_dev);
+  REQUIRE_PTR(kc);
+  REQUIRE_PTR(vc);
+  REQUIRE_PTR(lens);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(o_dev);
+  if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
+  const size_t bytes = (size_t)B * Hq * d * (dt == SAS_BF16 ? 2 : 4);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_decode_host copy in");
+  // A page-locked o_host is addressable from the device (unified addressing):
+  // the combining CTAs then write o straight into it, with no separate copy.
+  void* o_out = nullptr;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, o_host) == cudaSuccess && at.type == cudaMemoryTypeHost &&
+      at.devicePointer != nullptr && aligned16(at.devicePointer))
+    o_out = at.devicePointer;
+  cudaGetLastError();  // a pageable pointer is not an error here
+  e = sas::launch_decode_fused(q_dev, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, ksum,
+                               topk, gated, resolve_scale(scale, d), o_out ? o_out : o_dev,
+                               idx_out, st);
+  if (e != cudaSuccess) return cuda_status(e, "sas_decode_host launch");
+  if (o_out) return SAS_OK;
+  return cuda_status(cudaMemcpyAsync(o_host, o_dev, bytes, cudaMemcpyDeviceToHost, st),
+                     "sas_decode_host copy out");
+}
+
 // ---------------------------------------------------------------- paged decode
 sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
                             const float* kspool, sas_dtype dt, int B, int Hq, int Hkv, int npages,

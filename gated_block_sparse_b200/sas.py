@@ -45,6 +45,8 @@ SIGNATURES = {
                         _P]),
     "sas_decode_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I, _F,
                               _P, _P, _P]),
+    "sas_decode_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P,
+                             _P, _P]),
     "sas_select_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sas_select_bwd": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _Z,
                             _P]),
@@ -253,6 +255,22 @@ def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: fl
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
         float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
     return out
+
+
+def sas_decode_host(q_host, q_dev, kc, vc, lens, ksum, topk: int, o_dev, o_host, gated: int = 1,
+                    scale: float = 0.0, idx_out=None, stream=None):
+    """One decode step from pinned host q to pinned host o (copies and the
+    kernel enqueued by one C call); q_dev and o_dev are device staging."""
+    lib = load_library()
+    if q_host.is_cuda or o_host.is_cuda:
+        raise ValueError("q_host and o_host must be host tensors")
+    B, Hq, d = q_dev.shape
+    Hkv, Lmax = kc.shape[1], kc.shape[2]
+    _check("sas_decode_host", lib.sas_decode_host(
+        q_host.data_ptr(), _ptr(q_dev), _ptr(kc), _ptr(vc), _dt(q_dev), B, Hq, Hkv, Lmax, d,
+        _ptr(lens), _ptr(ksum), topk, int(gated), float(scale), _ptr(o_dev), o_host.data_ptr(),
+        _ptr(idx_out), _stream(stream)))
+    return o_host
 
 
 def sas_decode_paged(q, kpool, vpool, kspool, block_table, lens, topk: int, gated: int = 1,

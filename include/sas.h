@@ -215,6 +215,22 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              sas_stream_t stream);
 
 /*
+ * One decode step from and to host memory: enqueues on `stream` the copy of
+ * q_host ([B][Hq][d], dt; page-locked for the copy to be asynchronous) into
+ * q_dev and the sas_decode step. When o_host is page-locked host memory
+ * (cudaHostAlloc / cudaMallocHost), the step writes o straight into it over
+ * the bus and o_dev is not touched; otherwise it writes o_dev and a copy
+ * into o_host follows. The caches, lens and summaries are device memory as
+ * in sas_decode. Returns once the work is enqueued; o_host is valid after
+ * the stream reaches that point.
+ */
+sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, const void* vc,
+                           sas_dtype dt, int B, int Hq, int Hkv, int Lmax, int d,
+                           const int32_t* lens, const float* ksum, int topk, int gated,
+                           float scale, void* o_dev, void* o_host, int32_t* idx_out,
+                           sas_stream_t stream);
+
+/*
  * Decode over a paged cache (the serving layout of the pages' SGLang /
  * FlashInfer setting; SAS close reading, section 2.4): as sas_decode, but
  * the caches are pools of 64-token pages, one page per (block, kv head):

@@ -468,3 +468,19 @@ def test_decode_paged_matches_contiguous_and_oracle(gated):
     assert excess(np64(o_p), oo, 2e-2, True) <= 0
     st, msg = sas.sas_device_status()
     assert st == 0, msg
+
+
+def test_decode_host_buffers_match_device_call():
+    """sas_decode_host (pinned host q in, pinned host o out, one C call) gives
+    the device call's output exactly."""
+    x = inputs.gen_decode(2, 32, 8, 4096, 128, [4096, 3000], "bf16", seed=73, planted=8)
+    q, kc, vc, lens = x["q"], dev(x["kc"]), dev(x["vc"]), dev(x["lens"])
+    ks = sas.sas_block_summary(kc)
+    o_ref = sas.sas_decode(dev(q), kc, vc, lens, ks, 15).cpu()
+    qh = q.clone().pin_memory()
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    qd = torch.empty(q.shape, dtype=q.dtype, device=DEV)
+    od = torch.empty_like(qd)
+    sas.sas_decode_host(qh, qd, kc, vc, lens, ks, 15, od, oh)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o_ref)

@@ -26,13 +26,15 @@
 //   warps 0-7: gradient rows: warps w and w+4 share the TMEM lanes of rows
 //           32(w%4).. and split the 64 key columns, two warps per SM
 //           sub-partition to hide instruction latency
-// dK^T / dV^T reach the fp32 accumulators through a per-warp shared-memory
-// transpose into [8 keys][32 d] slices, each added by one TMA tensor
-// reduce-add (two slices per warp alternate); K/V stream through a
-// three-stage ring; no CTA-wide barrier runs inside the unit loop. These
-// reductions (64 KB per unit) bound the kernel: they drain at about 20 bytes
-// per cycle per SM whether issued as vector reductions or TMA reduce-adds of
-// 1 or 4 KB.
+//   warps 10-13: flush of dK^T / dV^T (TMEM lanes 32(w%4).. = head dims)
+// dK^T / dV^T reach the fp32 accumulators through four flush warps (one per
+// TMEM lane quarter): each moves its quarter of unit j's dK^T / dV^T into
+// [8 keys][32 d] shared-memory slices, each added by one TMA tensor
+// reduce-add (two slices per warp alternate), while the gradient warps
+// already work on unit j+1; K/V stream through a three-stage ring; no
+// CTA-wide barrier runs inside the unit loop. The reductions (64 KB per
+// unit) drain at about 20 bytes per cycle per SM, so the flush warps take
+// them off the gradient warps' path.
 // 512 TMEM columns and about 213 KB of shared memory: one CTA per SM.
 #include <cuda.h>
 #include <math.h>
@@ -48,8 +50,9 @@ __device__ uint32_t g_attn_bwd_tc_err = 0;
 
 namespace {
 
-constexpr int BT_THREADS = 320;  // 8 gradient warps, TMA warp, MMA warp
+constexpr int BT_THREADS = 448;  // 8 gradient warps, TMA warp, MMA warp, 4 flush warps
 constexpr int NGW = 8;           // gradient warps
+constexpr int NFW = 4;           // flush warps (warps 10-13)
 constexpr int D = 128;
 constexpr uint32_t TILE128 = 128 * D * 2;            // Q or dO: 32 KB
 constexpr uint32_t KV_STAGE = 2 * 64 * D * 2;        // K + V: 32 KB
@@ -61,7 +64,8 @@ constexpr int NKV = 3;                                // K/V ring stages
 constexpr uint32_t OFF_P = OFF_KV + NKV * KV_STAGE;
 constexpr uint32_t OFF_DS = OFF_P + PT_BYTES;
 constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [warp][2][8 keys][32 d] slices
-constexpr uint32_t OFF_DL = OFF_T + NGW * 2 * 8 * 32 * 4;  // fp32 [unit][warp] d(log g) partials
+constexpr int FSLOT = 1;         // [32 keys][32 d] slices per flush warp
+constexpr uint32_t OFF_DL = OFF_T + NFW * FSLOT * 32 * 32 * 4;  // fp32 [unit][warp] d(log g) partials
 constexpr uint32_t OFF_BAR = OFF_DL + 129 * 8 * 4 + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -74,8 +78,9 @@ enum Bar {
   B_SE = 8,    // S and dP read by the gradient warps (one arrival per warp)
   B_PF = 9,    // P and dS written (one arrival per warp)
   B_MD = 10,   // all MMAs of the unit done
-  B_TE = 11,   // [2] dK^T/dV^T TMEM buffer read (one arrival per warp)
-  NBAR = 13
+  B_TE = 11,   // [2] dK^T/dV^T TMEM buffer read (one arrival per flush warp)
+  B_KF = 13,   // [2] dK^T/dV^T TMEM buffer written (its unit's MMAs done)
+  NBAR = 15
 };
 
 // TMEM columns
@@ -122,8 +127,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   };
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) {
-      const bool per_warp = (i == B_SE || i == B_PF || i == B_TE || i == B_TE + 1);
-      mbar_init(&bars[i], per_warp ? NGW : 1);
+      const bool grad = (i == B_SE || i == B_PF), flush = (i == B_TE || i == B_TE + 1);
+      mbar_init(&bars[i], grad ? NGW : (flush ? NFW : 1));
     }
     fence_mbar_init();
   }
@@ -212,6 +217,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         }
         tc::commit(&bars[B_MD]);
         tc::commit(&bars[B_KVE + ks_]);
+        tc::commit(&bars[B_KF + s]);
       };
       issue_sdp(0);
       for (int j = 0; j < nunits; ++j) {
@@ -219,6 +225,57 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         issue_grad(j);
       }
     }
+  } else if (warp >= 8 + 2) {
+    // ---------------------------------------------------------------- flush
+    // Warp 10 + i owns TMEM lanes 32((10 + i) % 4).. = head dims of dK^T /
+    // dV^T. For each unit, once its MMAs are done, it moves its lane quarter
+    // (all 64 keys, both matrices) into [32 keys][32 d] fp32 slices and adds
+    // each with one TMA reduce-add (rows past N are clipped by the map; a
+    // slice wholly past N is skipped). It releases the unit's TMEM buffer
+    // after its last TMEM read. Slices rotate with the count of issued
+    // groups: the reduce issued from a slice FSLOT groups earlier must have
+    // read it before it is rewritten.
+    const int fq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(fq * 32) << 16;
+    float* tw = reinterpret_cast<float*>(sm + OFF_T) + (warp - 10) * FSLOT * 1024;  // [32][32] slices
+    const int plane = b * Hkv + r;
+    int ngroups = 0;
+    for (int j = 0; j < nunits; ++j) {
+      // buffer j & 1 holds unit j: its phase cannot advance again before this
+      // warp releases the buffer, so the parity below is never ambiguous
+      mbar_wait_data(&bars[B_KF + (j & 1)], (j >> 1) & 1, err);
+      tc::fence_after_sync();
+      const int blk = unit_block(j);
+      const uint32_t cb = tmem + (j & 1) * C_BUF + lane_off;
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {  // (matrix, key half)
+        const int m2 = part >> 1, hk = part & 1;
+        float kv[32];
+        tc::tmem_ld32(cb + (m2 == 0 ? C_DKT : C_DVT) + 32 * hk, kv);
+        tc::tmem_wait_ld();
+        if (part == 3) {  // the unit's TMEM buffer is no longer read
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[B_TE + (j & 1)]);
+        }
+        const int key0 = 64 * blk + 32 * hk;
+        if (key0 < N) {  // warp-uniform; rows past N are clipped by the map
+          float* sl = tw + ((ngroups % FSLOT) << 10);
+          if (lane == 0) tc::bulk_wait_read<FSLOT - 1>();
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sl[i * 32 + lane] = kv[i];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_reduce_add_3d(m2 == 0 ? &dkmap : &dvmap, sl, 32 * fq, key0, plane);
+            tc::bulk_commit();
+          }
+          ++ngroups;
+        }
+      }
+    }
+    if (lane == 0) tc::bulk_wait<0>();  // every reduce of this warp has completed
   } else {
     // ---------------------------------------------------------------- gradient rows
     // Warps w and w + 4 share TMEM lanes 32(w%4)..+31 (query rows for S/dP/dQ,
@@ -249,43 +306,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     }
     unsigned char* prow = sm + OFF_P + row * 128;
     unsigned char* dsrow = sm + OFF_DS + row * 128;
-    const int plane = b * Hkv + r;
-    float* tw = reinterpret_cast<float*>(sm + OFF_T) + warp * 512;  // two [8][32] slices
     const int gtid = hc * 128 + row;  // 0..255 over the gradient warps
-    // Add unit jj's dK^T / dV^T (TMEM lanes = d, columns = keys) to the fp32
-    // accumulators: each group of 8 keys is transposed into a [key][d] slice
-    // and added by one TMA reduce-add (rows past N are clipped by the map; a
-    // group wholly past N is skipped). Slices alternate with the count of
-    // issued groups, so the reduce issued from a slice two groups earlier
-    // must have read it before the slice is rewritten.
-    int ngroups = 0;
-    auto flush_kv = [&](int jj) {
-      const int blk = unit_block(jj);
-      const uint32_t cb = tmem + (jj & 1) * C_BUF + lane_off;
-#pragma unroll 1
-      for (int m2 = 0; m2 < 2; ++m2) {
-        float kv[32];
-        tc::tmem_ld32(cb + (m2 == 0 ? C_DKT : C_DVT) + 32 * hc, kv);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int key0 = 64 * blk + 32 * hc + 8 * g;
-          if (key0 >= N) continue;  // warp-uniform
-          float* sl = tw + ((ngroups & 1) << 8);
-          if (lane == 0) tc::bulk_wait_read<1>();
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sl[i * 32 + lane] = kv[8 * g + i];
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tc::tma_reduce_add_3d(m2 == 0 ? &dkmap : &dvmap, sl, 32 * wq, key0, plane);
-            tc::bulk_commit();
-          }
-          ++ngroups;
-        }
-      }
-    };
     float* dl_s = reinterpret_cast<float*>(sm + OFF_DL);
     for (int j = 0; j < nunits; ++j) {
       const bool cur = (j == kk);
@@ -333,12 +354,6 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PF]);
-      if (j >= 1) {
-        flush_kv(j - 1);
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_TE + ((j - 1) & 1)]);
-      }
       if (!cur) {  // this warp's part of d(log g) of the slot, summed at the end
         dsum = warp_sum(dsum);
         if (lane == 0) dl_s[j * NGW + warp] = dsum;
@@ -346,8 +361,6 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     }
     mbar_wait_data(&bars[B_MD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
-    flush_kv(nunits - 1);
-    if (lane == 0) tc::bulk_wait<0>();  // every reduce of this warp has completed
     named_bar_softmax();
     for (int j = gtid; j < kk; j += 2 * 128) {  // d(log g): fixed-order sum over the warps
       float a = 0.f;
@@ -413,8 +426,8 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   CUtensorMap qm, km, vm, dom, dkm, dvm;
   if (!make_map(&qm, q, N, B * Hq) || !make_map(&km, k, N, B * Hkv) ||
       !make_map(&vm, v, N, B * Hkv) || !make_map(&dom, dout, N, B * Hq) ||
-      !make_tma_map_f32_3d(&dkm, dk_acc, D, N, B * Hkv, 32, 8) ||
-      !make_tma_map_f32_3d(&dvm, dv_acc, D, N, B * Hkv, 32, 8))
+      !make_tma_map_f32_3d(&dkm, dk_acc, D, N, B * Hkv, 32, 32) ||
+      !make_tma_map_f32_3d(&dvm, dv_acc, D, N, B * Hkv, 32, 32))
     return cudaErrorInvalidValue;
   e = ensure_smem(k_attn_bwd_tc, SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -72,6 +72,17 @@ def block_summary(k, lens=None) -> np.ndarray:
     return out
 
 
+def round_bf16(x) -> np.ndarray:
+    """The nearest bf16 value of each element (8 significant bits, ties to
+    even), as float64: summaries stored in bf16 halve the bytes the
+    long-context selection scans, and the selection then runs on these
+    rounded values. Normal range only (summaries are means of the keys)."""
+    x = _f64(x)
+    m, e = np.frexp(x)  # x = m 2^e, 0.5 <= |m| < 1
+    ulp = np.ldexp(1.0, e - 8)
+    return np.round(x / ulp) * ulp  # numpy rounds halves to even
+
+
 # --------------------------------------------------------------------------
 # Selector score, normalised gate, Top-K (sections 2.1 and 2.2).
 # --------------------------------------------------------------------------

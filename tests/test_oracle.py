@@ -499,3 +499,17 @@ def test_selector_backward_eq8_structure():
         for m in range(t):
             if m not in kept:
                 assert abs(ds[m] + g[m] * total) < 1e-12
+
+
+# ---------------------------------------------------------------- bf16 summaries
+def test_round_bf16_matches_library_conversion():
+    """The oracle's bf16 rounding equals torch's float32 -> bfloat16 conversion
+    (round to nearest even) on float32 values, including exact midpoints."""
+    x = rnd(20000, 97).astype(np.float32) * np.float32(3.0)
+    mids = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(2.0 + 2.0 ** -7), 0.5 + 2.0 ** -9,
+                     0.0], dtype=np.float32)  # halfway cases tie to the even neighbour
+    xs = np.concatenate([x, mids])
+    want = torch.from_numpy(xs).to(torch.bfloat16).double().numpy()
+    got = O.round_bf16(xs.astype(np.float64))
+    assert np.array_equal(got, want)
+    assert got[-5] == 1.0 and got[-4] == 1.0 + 2 * 2.0 ** -7 and got[-3] == -2.0

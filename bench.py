@@ -186,9 +186,10 @@ def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: 
 
 # ----------------------------------------------------------------- decode
 class DecodeWorkload:
-    def __init__(self, name: str):
+    def __init__(self, name: str, summary: str = "f32"):
         from gated_block_sparse_b200 import inputs
         self.name = name
+        self.summary = summary
         self.c = inputs.CONFIGS[name]
         self.host = inputs.gen_config(name)
         c = self.c
@@ -198,8 +199,9 @@ class DecodeWorkload:
         kk = [min(c["topk"], C) for C in self.C]
         ncur = [int(n) - 64 * C for n, C in zip(lens, self.C)]
         d, Hkv, es = c["d"], c["Hkv"], 2 if c["dtype"] == "bf16" else 4
+        ses = 2 if summary == "bf16" else 4  # bytes per stored summary element
         # algorithmic bytes per step, by kernel
-        self.sel_bytes = sum(Hkv * C * d * 4 for C in self.C) + c["B"] * c["Hq"] * d * es
+        self.sel_bytes = sum(Hkv * C * d * ses for C in self.C) + c["B"] * c["Hq"] * d * es
         self.att_bytes = (sum(Hkv * (k * 64 + nc) * d * es * 2 for k, nc in zip(kk, ncur))
                           + 2 * c["B"] * c["Hq"] * d * es)
         self.step_bytes = self.sel_bytes + self.att_bytes - c["B"] * c["Hq"] * d * es  # q once
@@ -211,6 +213,7 @@ class DecodeWorkload:
                 "q_heads": c["Hq"], "kv_heads": c["Hkv"], "head_dim": c["d"],
                 "context": c["Lmax"] if c["lens"][0] == c["lens"][1] else list(c["lens"]),
                 "topk": c["topk"], "gated": c["gated"], "block": 64,
+                "summaries": "bf16" if self.summary == "bf16" else "fp32",
                 "bytes_per_step": self.step_bytes}
 
 
@@ -224,9 +227,13 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     q = h["q"].to(dev)
     lens = h["lens"].to(dev)
     kc0, vc0 = h["kc"].to(dev), h["vc"].to(dev)
-    ks0 = sas.sas_block_summary(kc0)
+    bf16_sum = w.summary == "bf16"
+    if bf16_sum and args.paged:
+        raise SystemExit("--summary bf16 reads contiguous caches only")
+    ks0 = (sas.sas_block_summary_ex(kc0, torch.bfloat16) if bf16_sum
+           else sas.sas_block_summary(kc0))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    per_layer = kc0.numel() * kc0.element_size() * 2 + ks0.numel() * 4
+    per_layer = kc0.numel() * kc0.element_size() * 2 + ks0.numel() * ks0.element_size()
     free = torch.cuda.mem_get_info(dev)[0]
     L = max(2, math.ceil(3 * l2 / w.step_bytes))
     L = min(L, max(2, int(0.6 * free // per_layer)))
@@ -264,6 +271,8 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
         if bt is not None:
             sas.sas_decode_paged(qq, kcs[j], vcs[j], kss[j], bt, lens, topk, gated=c["gated"],
                                  out=out)
+        elif bf16_sum:
+            sas.sas_decode_ex(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out)
         else:
             sas.sas_decode(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out,
                            ws=ws)
@@ -274,9 +283,9 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     ms, clk = timed_graphs(step, K, W, world, stream, clocks=clocks)
     clocks.stop()
 
-    # split path (contiguous caches only): selection alone, attention alone
+    # split path (contiguous caches, fp32 summaries): selection alone, attention alone
     split = None
-    if bt is None:
+    if bt is None and not bf16_sum:
         split = split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
     peaks = measured_peaks()
     # the step is one launch of the cluster kernel: its duration is the step's
@@ -288,10 +297,10 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
             "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
             "algorithmic_bytes_per_launch": w.step_bytes, "launch_us": round(kt * 1e6, 3),
             "selected_kv_bytes_per_launch": w.att_bytes, "split_path": split}
-    if bt is not None:
-        roof["traffic"] = None  # the ncu record is of the contiguous layout
+    if bt is not None or bf16_sum:
+        roof["traffic"] = None  # the ncu record is of contiguous caches with fp32 summaries
     return finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode,
-                         ms, clk, roof, l2, bt is not None)
+                         ms, clk, roof, l2, bt is not None or bf16_sum, bt is not None)
 
 
 def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o):
@@ -324,7 +333,7 @@ def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
 
 
 def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode, ms, clk,
-                  roof, l2, paged) -> dict:
+                  roof, l2, torch_copies, paged) -> dict:
     import torch
 
     from gated_block_sparse_b200 import dist as D
@@ -337,7 +346,7 @@ def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, 
 
     def e2e_step(i):
         j = i % L
-        if paged:  # host copies through torch around the paged call
+        if torch_copies:  # host copies through torch around the call
             qd.copy_(qh, non_blocking=True)
             decode(j, qd, o)
             oh.copy_(o, non_blocking=True)
@@ -359,6 +368,7 @@ def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, 
     ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
     nb = q.numel() * q.element_size()
     api = ("sas_decode_paged with torch copies" if paged
+           else "sas_decode_ex with torch copies" if torch_copies
            else "sas_decode_host (copy in, then the step writing o into pinned host memory)")
     value = D.whole_job_rate(w.step_bytes * K, world, ms) / 1e9
     return {
@@ -386,14 +396,17 @@ def one_thread():
     return threadpool_limits(limits=1)
 
 
-def cpu_baseline_decode(name: str, seconds: float, w: "DecodeWorkload | None" = None) -> dict:
+def cpu_baseline_decode(name: str, seconds: float, w: "DecodeWorkload | None" = None,
+                        summary: str = "f32") -> dict:
     """The fp64 oracle on whole decode steps of the workload, for ~`seconds`."""
     from oracle import sas_oracle as O
-    w = DecodeWorkload(name) if w is None else w
+    w = DecodeWorkload(name, summary) if w is None else w
     c = w.c
     h = w.host
     with one_thread():
         ks = O.block_summary(h["kc"])  # summaries are built outside the step, as on the GPU
+        if w.summary == "bf16":
+            ks = O.round_bf16(ks)
         lens = h["lens"].numpy()
         n, t0 = 0, time.perf_counter()
         while True:
@@ -585,6 +598,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--paged", action="store_true",
                     help="decode: read the caches through 64-token pages (sas_decode_paged)")
+    ap.add_argument("--summary", default="f32", choices=["f32", "bf16"],
+                    help="decode: store block summaries in fp32 or bf16 (sas_decode_ex)")
     ap.add_argument("--layers", type=int, default=0,
                     help="decode: number of rotated layer copies (default: enough for 3x L2)")
     args = ap.parse_args()
@@ -597,7 +612,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        base = (cpu_baseline_decode(args.config, args.cpu_seconds) if decode
+        base = (cpu_baseline_decode(args.config, args.cpu_seconds, summary=args.summary) if decode
                 else cpu_baseline_prefill(args.config, args.cpu_seconds))
         from gated_block_sparse_b200 import inputs
         print(json.dumps({
@@ -613,7 +628,7 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     if decode:
-        w = DecodeWorkload(args.config)
+        w = DecodeWorkload(args.config, args.summary)
         res = bench_decode_ours(args, world, rank, local, w)
     else:
         res = bench_prefill_ours(args, world, rank, local)

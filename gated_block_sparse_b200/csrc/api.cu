@@ -92,6 +92,25 @@ sas_status sas_block_summary(const void* k, sas_dtype dt, int B, int H, int N, i
                      "sas_block_summary launch");
 }
 
+sas_status sas_block_summary_ex(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                                const int32_t* lens, void* ksum, sas_dtype sum_dt,
+                                sas_stream_t stream) {
+  g_last_error.clear();
+  REQUIRE(sum_dt == SAS_F32 || sum_dt == SAS_BF16, SAS_ERR_INVALID_ARG,
+          "summary dtype must be SAS_F32 or SAS_BF16");
+  if (sum_dt == SAS_F32)
+    return sas_block_summary(k, dt, B, H, N, d, lens, static_cast<float*>(ksum), stream);
+  sas_status s = check_common(dt, B, H, H, N, d, 0);
+  if (s != SAS_OK) return s;
+  if (B == 0 || N / 64 == 0) return SAS_OK;
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(ksum);
+  if (lens) REQUIRE(aligned16(lens), SAS_ERR_INVALID_ARG, "lens must be 16-byte aligned");
+  return cuda_status(sas::launch_block_summary_bf16(k, dt == SAS_BF16, B, H, N, d, lens, ksum,
+                                                    (cudaStream_t)stream),
+                     "sas_block_summary_ex launch");
+}
+
 size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_mode mode) {
   if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || topk < 0) return 0;
   if (mode == SAS_PREFILL) return a16(sas::select_prefill_ws_bytes(B, Hkv, N, d));
@@ -327,6 +346,30 @@ sas_status sas_decode(const void* q, const void* kc, const void* vc, sas_dtype d
                                               ksum, topk, gated, resolve_scale(scale, d), o,
                                               idx_out, (cudaStream_t)stream),
                      "sas_decode launch");
+}
+
+sas_status sas_decode_ex(const void* q, const void* kc, const void* vc, sas_dtype dt, int B,
+                         int Hq, int Hkv, int Lmax, int d, const int32_t* lens, const void* ksum,
+                         sas_dtype sum_dt, int topk, int gated, float scale, void* o,
+                         int32_t* idx_out, sas_stream_t stream) {
+  g_last_error.clear();
+  REQUIRE(sum_dt == SAS_F32 || sum_dt == SAS_BF16, SAS_ERR_INVALID_ARG,
+          "summary dtype must be SAS_F32 or SAS_BF16");
+  sas_status s = check_decode(dt, B, Hq, Hkv, Lmax, d, topk, gated);
+  if (s != SAS_OK) return s;
+  if (B == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kc);
+  REQUIRE_PTR(vc);
+  REQUIRE_PTR(lens);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(o);
+  if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
+  return cuda_status(sas::launch_decode_fused_ex(q, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d,
+                                                 lens, ksum, sum_dt == SAS_BF16, topk, gated,
+                                                 resolve_scale(scale, d), o, idx_out,
+                                                 (cudaStream_t)stream),
+                     "sas_decode_ex launch");
 }
 
 // ---------------------------------------------------------------- decode from host buffers

@@ -70,7 +70,8 @@ __host__ __device__ inline size_t fd_al(size_t x) { return (x + 127) & ~(size_t)
 // Region u: K/V slot 0 followed by the summary ring during the scan, then by
 // the list scratch (warp lists, survivors, merge buffer) during selection;
 // K/V slots 0 .. nkv-1 afterwards; the per-warp states at the end.
-__host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int kq, int CS) {
+__host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int kq, int CS,
+                                             int ses) {
   FdSmem L;
   const size_t kvslot = (size_t)2 * SAS_BLOCK * D * es;
   L.wl = kvslot;
@@ -78,7 +79,7 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int k
   L.tmp = L.wb + (size_t)FD_WARPS * kq * 8;
   L.mb = L.tmp + (size_t)CS * kq * 8;
   L.mblen = L.mb + (size_t)CS * kq * 8;
-  size_t ub = kvslot + (size_t)FD_NS * FD_SUBC * D * 4;
+  size_t ub = kvslot + (size_t)FD_NS * FD_SUBC * D * ses;
   if (ub < L.mblen + 128) ub = L.mblen + 128;
   if (ub < 2 * kvslot) ub = 2 * kvslot;
   const size_t comb = (size_t)FD_WARPS * G * (D + 2) * 4;
@@ -170,10 +171,11 @@ __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2)
 // summaries [npages][Hkv][D], and bt [B][max_blocks] maps a sequence's
 // logical block to its page (Lmax = 64 max_blocks). Otherwise kc, vc are
 // [B][Hkv][Lmax][D] and ksum [B][Hkv][Lmax/64][D].
-template <typename T, int D, int G, bool PAGED>
+// S: the summaries' element type (float, or bf16 for half the scan bytes).
+template <typename T, int D, int G, bool PAGED, typename S>
 __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-    const float* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
+    const S* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
     int gated, float scale, int per_max, T* __restrict__ o, int32_t* __restrict__ idx_out,
     const int32_t* __restrict__ bt, int npages) {
   constexpr int TILE = SAS_BLOCK * D;
@@ -187,10 +189,10 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int crank = (int)cluster.block_rank();
   const int lg = ceil_log2(topk > 0 ? topk : 1);
   const int kq = 1 << lg;  // list stride (power of two)
-  const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS);
+  const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S));
   unsigned char* U = sm + L.u;
   const size_t kvslot = (size_t)2 * TILE * sizeof(T);
-  float* ring = reinterpret_cast<float*>(U + kvslot);
+  S* ring = reinterpret_cast<S*>(U + kvslot);
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qbar = reinterpret_cast<float*>(sm + L.qbar);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int nsub = (nmine + FD_SUBC - 1) / FD_SUBC;
   const int NKV = L.nkv;
   const size_t kvrow = row * (size_t)Lmax * D;
-  const float* ks_row = ksum + row * (size_t)nblk * D;
+  const S* ks_row = ksum + row * (size_t)nblk * D;
   uint32_t* err = &g_decode_fused_err;
   const int32_t* bt_row = PAGED ? bt + (size_t)b * nblk : nullptr;
   // page of logical block m (paged caches); an out-of-range entry is flagged
@@ -267,16 +269,17 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   // summaries [first, first + cnt) of this CTA's range into ring slot `slot`:
   // one bulk copy (contiguous), or one row copy per lane of warp 0 (paged)
   auto issue_summaries = [&](int slot, int first, int cnt) {
-    float* dst = ring + (size_t)slot * FD_SUBC * D;
+    S* dst = ring + (size_t)slot * FD_SUBC * D;
     if constexpr (PAGED) {
-      if (lane == 0) mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * 4));
+      if (lane == 0) mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * sizeof(S)));
       __syncwarp();
       for (int j = lane; j < cnt; j += 32)
         bulk_g2s(dst + (size_t)j * D, ksum + ((size_t)page_of(m0 + first + j) * Hkv + r) * D,
-                 (uint32_t)(D * 4), &sum_bar[slot]);
+                 (uint32_t)(D * sizeof(S)), &sum_bar[slot]);
     } else {
-      mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * 4));
-      bulk_g2s(dst, ks_row + (size_t)(m0 + first) * D, (uint32_t)(cnt * D * 4), &sum_bar[slot]);
+      mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * sizeof(S)));
+      bulk_g2s(dst, ks_row + (size_t)(m0 + first) * D, (uint32_t)(cnt * D * sizeof(S)),
+               &sum_bar[slot]);
     }
   };
 
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       const int slot = i % FD_NS;
       const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
       mbar_wait_data(&sum_bar[slot], (uint32_t)((i / FD_NS) & 1), err);
-      const float* sb = ring + (size_t)slot * FD_SUBC * D;
+      const S* sb = ring + (size_t)slot * FD_SUBC * D;
       for (int j0 = wid; j0 < cnt_i; j0 += 4 * FD_WARPS) {
         float part[4];
 #pragma unroll
@@ -705,7 +708,7 @@ struct FdPick {
 // CTA h combines head h) whose clusters of all rows are co-resident on the
 // GPU; if none is, the largest that launches. Cached per shape, so repeated
 // launches make no occupancy queries.
-template <typename T, int D, int G, bool PAGED>
+template <typename T, int D, int G, bool PAGED, typename S>
 cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
   static std::mutex mu;
   static FdPick cache[32];
@@ -723,13 +726,14 @@ cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
         return cudaSuccess;
       }
   }
-  auto kern = k_decode_fused<T, D, G, PAGED>;
+  auto kern = k_decode_fused<T, D, G, PAGED, S>;
   int best = 0, first = 0;
   const int cands[5] = {16, 8, 4, 2, 1};
   for (int ci = 0; ci < 5; ++ci) {
     const int CS = cands[ci];
     if (CS < G) break;
-    const size_t smem = fd_layout(D, G, (int)sizeof(T), (nblk + CS - 1) / CS, kq, CS).total;
+    const size_t smem =
+        fd_layout(D, G, (int)sizeof(T), (nblk + CS - 1) / CS, kq, CS, (int)sizeof(S)).total;
     if (smem > 227 * 1024) continue;
     if (ensure_smem(kern, smem) != cudaSuccess) {
       cudaGetLastError();
@@ -770,19 +774,19 @@ cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
   return cudaSuccess;
 }
 
-template <typename T, int D, int G, bool PAGED>
-cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const float* ksum, int B,
+template <typename T, int D, int G, bool PAGED, typename S>
+cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const void* ksum, int B,
                            int Hkv, int Lmax, const int32_t* lens, int topk, int gated, float scale,
                            void* o, int32_t* idx_out, const int32_t* bt, int npages,
                            cudaStream_t st) {
-  auto kern = k_decode_fused<T, D, G, PAGED>;
+  auto kern = k_decode_fused<T, D, G, PAGED, S>;
   const int nblk = Lmax / SAS_BLOCK;
   const int kq = 1 << ceil_log2(topk > 0 ? topk : 1);
   int CS = 0;
-  cudaError_t e = pick_cluster<T, D, G, PAGED>(B, Hkv, nblk, kq, CS);
+  cudaError_t e = pick_cluster<T, D, G, PAGED, S>(B, Hkv, nblk, kq, CS);
   if (e != cudaSuccess) return e;
   const int per_max = (nblk + CS - 1) / CS;
-  const size_t smem = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS).total;
+  const size_t smem = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S)).total;
   e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -798,20 +802,26 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
-                            static_cast<const T*>(vc), ksum, Hkv, Lmax, lens, topk, gated, scale,
+                            static_cast<const T*>(vc), static_cast<const S*>(ksum), Hkv, Lmax,
+                            lens, topk, gated, scale,
                             per_max, static_cast<T*>(o), idx_out, bt, npages);
 }
 
 template <typename T, int D>
-cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc, const float* ksum,
-                           int B, int Hkv, int Lmax, const int32_t* lens, int topk, int gated,
-                           float scale, void* o, int32_t* idx_out, const int32_t* bt, int npages,
-                           cudaStream_t st) {
+cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc, const void* ksum,
+                           int sum_bf16, int B, int Hkv, int Lmax, const int32_t* lens, int topk,
+                           int gated, float scale, void* o, int32_t* idx_out, const int32_t* bt,
+                           int npages, cudaStream_t st) {
 #define SAS_FD(GG)                                                                              \
-  return bt ? launch_fused_t<T, D, GG, true>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated,  \
-                                             scale, o, idx_out, bt, npages, st)                 \
-            : launch_fused_t<T, D, GG, false>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, \
-                                              scale, o, idx_out, nullptr, 0, st)
+  if (bt)                                                                                       \
+    return launch_fused_t<T, D, GG, true, float>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,     \
+                                                 gated, scale, o, idx_out, bt, npages, st);     \
+  if (sum_bf16)                                                                                 \
+    return launch_fused_t<T, D, GG, false, __nv_bfloat16>(q, kc, vc, ksum, B, Hkv, Lmax, lens,  \
+                                                          topk, gated, scale, o, idx_out,       \
+                                                          nullptr, 0, st);                      \
+  return launch_fused_t<T, D, GG, false, float>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,      \
+                                                gated, scale, o, idx_out, nullptr, 0, st)
   switch (G) {
     case 1: SAS_FD(1);
     case 2: SAS_FD(2);
@@ -823,23 +833,23 @@ cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc,
 }
 
 cudaError_t launch_fused(const void* q, const void* kc, const void* vc, int bf16, int B, int Hq,
-                         int Hkv, int Lmax, int d, const int32_t* lens, const float* ksum,
-                         int topk, int gated, float scale, void* o, int32_t* idx_out,
-                         const int32_t* bt, int npages, cudaStream_t st) {
+                         int Hkv, int Lmax, int d, const int32_t* lens, const void* ksum,
+                         int sum_bf16, int topk, int gated, float scale, void* o,
+                         int32_t* idx_out, const int32_t* bt, int npages, cudaStream_t st) {
   if (B == 0) return cudaSuccess;
   const int G = Hq / Hkv;
   if (bf16) {
     if (d == 128)
-      return launch_fused_g<__nv_bfloat16, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,
-                                                gated, scale, o, idx_out, bt, npages, st);
-    return launch_fused_g<__nv_bfloat16, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated,
-                                             scale, o, idx_out, bt, npages, st);
+      return launch_fused_g<__nv_bfloat16, 128>(G, q, kc, vc, ksum, sum_bf16, B, Hkv, Lmax, lens,
+                                                topk, gated, scale, o, idx_out, bt, npages, st);
+    return launch_fused_g<__nv_bfloat16, 64>(G, q, kc, vc, ksum, sum_bf16, B, Hkv, Lmax, lens,
+                                             topk, gated, scale, o, idx_out, bt, npages, st);
   }
   if (d == 128)
-    return launch_fused_g<float, 128>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale,
-                                      o, idx_out, bt, npages, st);
-  return launch_fused_g<float, 64>(G, q, kc, vc, ksum, B, Hkv, Lmax, lens, topk, gated, scale, o,
-                                   idx_out, bt, npages, st);
+    return launch_fused_g<float, 128>(G, q, kc, vc, ksum, sum_bf16, B, Hkv, Lmax, lens, topk,
+                                      gated, scale, o, idx_out, bt, npages, st);
+  return launch_fused_g<float, 64>(G, q, kc, vc, ksum, sum_bf16, B, Hkv, Lmax, lens, topk, gated,
+                                   scale, o, idx_out, bt, npages, st);
 }
 
 }  // namespace
@@ -848,8 +858,16 @@ cudaError_t launch_decode_fused(const void* q, const void* kc, const void* vc, i
                                 int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
                                 const float* ksum, int topk, int gated, float scale, void* o,
                                 int32_t* idx_out, cudaStream_t st) {
-  return launch_fused(q, kc, vc, bf16, B, Hq, Hkv, Lmax, d, lens, ksum, topk, gated, scale, o,
+  return launch_fused(q, kc, vc, bf16, B, Hq, Hkv, Lmax, d, lens, ksum, 0, topk, gated, scale, o,
                       idx_out, nullptr, 0, st);
+}
+
+cudaError_t launch_decode_fused_ex(const void* q, const void* kc, const void* vc, int bf16, int B,
+                                   int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                                   const void* ksum, int sum_bf16, int topk, int gated,
+                                   float scale, void* o, int32_t* idx_out, cudaStream_t st) {
+  return launch_fused(q, kc, vc, bf16, B, Hq, Hkv, Lmax, d, lens, ksum, sum_bf16, topk, gated,
+                      scale, o, idx_out, nullptr, 0, st);
 }
 
 cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vpool, int bf16,
@@ -858,7 +876,7 @@ cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vp
                                 const float* kspool, int topk, int gated, float scale, void* o,
                                 int32_t* idx_out, cudaStream_t st) {
   return launch_fused(q, kpool, vpool, bf16, B, Hq, Hkv, max_blocks * SAS_BLOCK, d, lens, kspool,
-                      topk, gated, scale, o, idx_out, block_table, npages, st);
+                      0, topk, gated, scale, o, idx_out, block_table, npages, st);
 }
 
 uint32_t* decode_fused_error_word() {

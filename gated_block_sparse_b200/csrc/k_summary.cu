@@ -5,16 +5,17 @@
 // One CTA per (block m, head h, sequence b); 256 threads. Each thread loads
 // 16-byte vectors of one key row and accumulates fp32 column sums; the row
 // groups are reduced through shared memory. HBM-bound: every key is read
-// once, 4 bytes per column are written per block.
+// once, 4 bytes per column are written per block (2 with bf16 summaries,
+// the fp32 mean rounded to nearest even).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace sas {
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 __global__ void __launch_bounds__(256) k_block_summary(const T* __restrict__ k, int N, int nblk,
                                                        const int32_t* __restrict__ lens,
-                                                       float* __restrict__ ksum) {
+                                                       S* __restrict__ ksum) {
   constexpr int VEC = Vec16<T>::N;
   constexpr int TPR = D / VEC;   // threads per key row
   constexpr int RP = 256 / TPR;  // key rows per pass
@@ -39,22 +40,23 @@ __global__ void __launch_bounds__(256) k_block_summary(const T* __restrict__ k, 
 #pragma unroll
   for (int i = 0; i < VEC; ++i) red[rg][c * VEC + i] = acc[i];
   __syncthreads();
-  float* out = ksum + (((size_t)b * H + h) * nblk + m) * D;
+  S* out = ksum + (((size_t)b * H + h) * nblk + m) * D;
   for (int col = tid; col < D; col += 256) {
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < RP; ++r) s += red[r][col];
-    out[col] = (m < nvalid) ? s * (1.0f / SAS_BLOCK) : 0.f;
+    out[col] = from_f<S>((m < nvalid) ? s * (1.0f / SAS_BLOCK) : 0.f);
   }
 }
 
-cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
-                                 const int32_t* lens, float* ksum, cudaStream_t st) {
+template <typename S>
+static cudaError_t block_summary_s(const void* k, int bf16, int B, int H, int N, int d,
+                                   const int32_t* lens, S* ksum, cudaStream_t st) {
   const int nblk = N / SAS_BLOCK;
   if (nblk == 0 || B == 0 || H == 0) return cudaSuccess;
   dim3 grid(nblk, H, B);
 #define SAS_SUM(T, D) \
-  k_block_summary<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(k), N, nblk, lens, ksum)
+  k_block_summary<T, D, S><<<grid, 256, 0, st>>>(static_cast<const T*>(k), N, nblk, lens, ksum)
   if (bf16) {
     if (d == 128) SAS_SUM(__nv_bfloat16, 128); else SAS_SUM(__nv_bfloat16, 64);
   } else {
@@ -62,6 +64,17 @@ cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, i
   }
 #undef SAS_SUM
   return cudaGetLastError();
+}
+
+cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
+                                 const int32_t* lens, float* ksum, cudaStream_t st) {
+  return block_summary_s<float>(k, bf16, B, H, N, d, lens, ksum, st);
+}
+
+cudaError_t launch_block_summary_bf16(const void* k, int bf16, int B, int H, int N, int d,
+                                      const int32_t* lens, void* ksum, cudaStream_t st) {
+  return block_summary_s<__nv_bfloat16>(k, bf16, B, H, N, d, lens,
+                                        static_cast<__nv_bfloat16*>(ksum), st);
 }
 
 }  // namespace sas

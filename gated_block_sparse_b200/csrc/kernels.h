@@ -19,6 +19,9 @@ bool make_tma_map_f32_3d(CUtensorMap* map, const void* base, int d, int rows_per
 // Block summaries: ksum[b,h,m] = mean of keys 64m..64m+63.
 cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, int d,
                                  const int32_t* lens, float* ksum, cudaStream_t st);
+// The same, summaries stored in bf16 (the fp32 mean rounded to nearest even).
+cudaError_t launch_block_summary_bf16(const void* k, int bf16, int B, int H, int N, int d,
+                                      const int32_t* lens, void* ksum, cudaStream_t st);
 
 // ---- selection
 // Shared layout of one row's per-chunk partial results (decode scratch).
@@ -78,6 +81,12 @@ cudaError_t launch_decode_fused(const void* q, const void* kc, const void* vc, i
                                 int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
                                 const float* ksum, int topk, int gated, float scale, void* o,
                                 int32_t* idx_out, cudaStream_t st);
+// The same with the summaries' element type chosen: fp32 (sum_bf16 = 0) or
+// bf16 (half the bytes of the summary scan).
+cudaError_t launch_decode_fused_ex(const void* q, const void* kc, const void* vc, int bf16, int B,
+                                   int Hq, int Hkv, int Lmax, int d, const int32_t* lens,
+                                   const void* ksum, int sum_bf16, int topk, int gated,
+                                   float scale, void* o, int32_t* idx_out, cudaStream_t st);
 // Paged caches: kpool, vpool [npages][Hkv][64][d], kspool [npages][Hkv][d]
 // fp32 (the summary of each page), block_table [B][max_blocks] page ids.
 cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vpool, int bf16,

@@ -47,6 +47,9 @@ SIGNATURES = {
                               _P, _P, _P]),
     "sas_decode_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P,
                              _P, _P]),
+    "sas_block_summary_ex": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "sas_decode_ex": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P,
+                           _P]),
     "sas_select_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sas_select_bwd": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P, _Z,
                             _P]),
@@ -254,6 +257,31 @@ def sas_decode_attend(q, kc, vc, lens, idx, cnt, logg, gated: int = 1, scale: fl
         _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens),
         _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, topk, int(gated),
         float(scale), _ptr(out), _ptr(w), w.numel(), _stream(stream)))
+    return out
+
+
+def sas_block_summary_ex(k, sum_dtype=torch.float32, lens=None, out=None, stream=None):
+    """Block summaries stored as sum_dtype (torch.float32 or torch.bfloat16)."""
+    lib = load_library()
+    B, H, N, d = k.shape
+    if out is None:
+        out = torch.empty((B, H, N // 64, d), dtype=sum_dtype, device=k.device)
+    _check("sas_block_summary_ex", lib.sas_block_summary_ex(
+        _ptr(k), _dt(k), B, H, N, d, _ptr(lens), _ptr(out), _dt(out), _stream(stream)))
+    return out
+
+
+def sas_decode_ex(q, kc, vc, lens, ksum, topk: int, gated: int = 1, scale: float = 0.0, out=None,
+                  idx_out=None, stream=None):
+    """sas_decode reading summaries of ksum's dtype (fp32 or bf16)."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    Hkv, Lmax = kc.shape[1], kc.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check("sas_decode_ex", lib.sas_decode_ex(
+        _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens), _ptr(ksum),
+        _dt(ksum), topk, int(gated), float(scale), _ptr(out), _ptr(idx_out), _stream(stream)))
     return out
 
 

@@ -215,6 +215,22 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              sas_stream_t stream);
 
 /*
+ * Summaries in bf16 (cheaper long-context selection: the summary scan is the
+ * length-dependent part of a decode step, and bf16 halves its bytes).
+ * sas_block_summary_ex writes the summaries in sum_dt: SAS_F32 as
+ * sas_block_summary, or SAS_BF16, the fp32 mean rounded to nearest even.
+ * sas_decode_ex is sas_decode reading summaries of type sum_dt; the scores
+ * are computed from the stored (rounded) summaries.
+ */
+sas_status sas_block_summary_ex(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                                const int32_t* lens, void* ksum, sas_dtype sum_dt,
+                                sas_stream_t stream);
+sas_status sas_decode_ex(const void* q, const void* kc, const void* vc, sas_dtype dt, int B,
+                         int Hq, int Hkv, int Lmax, int d, const int32_t* lens, const void* ksum,
+                         sas_dtype sum_dt, int topk, int gated, float scale, void* o,
+                         int32_t* idx_out, sas_stream_t stream);
+
+/*
  * One decode step from and to host memory: enqueues on `stream` the copy of
  * q_host ([B][Hq][d], dt; page-locked for the copy to be asynchronous) into
  * q_dev and the sas_decode step. When o_host is page-locked host memory

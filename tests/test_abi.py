@@ -27,7 +27,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 22
+    assert len(names) == 24
     for n in names:
         assert hasattr(lib, n), n
         assert n in sas.SIGNATURES, n
@@ -96,6 +96,14 @@ def test_rejects_bad_decode_shapes(lib):
                         None, FAKE, ws, None)
     assert st == 1 and b"gated" in lib.sas_last_error_message()
 
+
+
+def test_rejects_bad_summary_dtype(lib):
+    st = lib.sas_block_summary_ex(FAKE, 1, 1, 8, 1024, 128, None, FAKE, 7, None)
+    assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
+    st = lib.sas_decode_ex(FAKE, FAKE, FAKE, 1, 1, 32, 8, 65536, 128, FAKE, FAKE, 7, 15, 1, 0.0,
+                           FAKE, None, None)
+    assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
 
 def test_empty_inputs_are_noops(lib):
     # B = 0 or N = 0: nothing to do, no pointer needed, no launch

@@ -94,6 +94,29 @@ def test_block_summary_lens():
     assert maxerr(np64(got), O.block_summary(k, lens=lens.numpy())) < 1e-5
 
 
+
+def _bf16_ulp(x):
+    e = np.frexp(np.where(x == 0, 1.0, x))[1]
+    return np.ldexp(1.0, e - 8)
+
+
+@pytest.mark.parametrize("dtype,d,N", [("bf16", 128, 1000), ("f32", 64, 640)])
+def test_block_summary_bf16(dtype, d, N):
+    """Summaries stored in bf16: the kernel's fp32 mean (within 1e-5 of the
+    exact one) rounded to nearest even, against the exact mean rounded. They
+    may differ only where the exact mean lies that close to a halfway point,
+    and then by one bf16 ulp."""
+    k = inputs.gen_prefill(2, 2, 2, N, d, dtype, seed=13)["k"]
+    got = sas.sas_block_summary_ex(dev(k), torch.bfloat16)
+    torch.cuda.synchronize()
+    assert got.dtype == torch.bfloat16
+    ref = O.round_bf16(O.block_summary(k))
+    diff = np.abs(np64(got) - ref)
+    assert np.all(diff <= _bf16_ulp(ref) * 1.0001)
+    assert (diff > 0).mean() < 1e-3
+    f32 = sas.sas_block_summary_ex(dev(k), torch.float32)
+    assert torch.equal(f32, sas.sas_block_summary(dev(k)))
+
 # ------------------------------------------------------------------ selection
 def _check_select(q, k, Hkv, topk, tol):
     ks = sas.sas_block_summary(dev(k))
@@ -297,6 +320,40 @@ def test_decode_full_configs(name):
     scores = _decode_check(inputs.gen_config(name), c["Hkv"], c["topk"], c["gated"])
     assert boundary_gap(scores, c["topk"]) >= 1.5e-3
 
+
+
+def _decode_bf16_summary_check(x, Hkv, topk, gated, tol=2e-2):
+    q, kc, vc, lens = x["q"], x["kc"], x["vc"], x["lens"]
+    ks = sas.sas_block_summary_ex(dev(kc), torch.bfloat16, lens=dev(lens))
+    idx = torch.empty((q.shape[0], Hkv, topk), dtype=torch.int32, device=DEV)
+    o = sas.sas_decode_ex(dev(q), dev(kc), dev(vc), dev(lens), ks, topk, gated=gated,
+                          idx_out=idx if topk else None)
+    torch.cuda.synchronize()
+    oks = O.round_bf16(O.block_summary(kc, lens=lens.numpy()))
+    oo, oi, _, _ = O.decode(q, kc, vc, lens.numpy(), oks, Hkv, topk, gated=gated)
+    if topk:
+        assert np.array_equal(idx.cpu().numpy(), oi)
+    err = excess(np64(o), oo, tol, q.dtype == torch.bfloat16)
+    assert err <= 0, err
+    _, _, _, scores = O.select_decode(q, oks, lens.numpy(), Hkv, topk)
+    return scores
+
+
+@pytest.mark.parametrize("name", ["c2", "c5"])
+def test_decode_bf16_summaries_full_configs(name):
+    """Decode reading bf16 summaries against the oracle scoring the exact
+    means rounded to bf16 (selection on the stored summaries)."""
+    c = inputs.CONFIGS[name]
+    scores = _decode_bf16_summary_check(inputs.gen_config(name), c["Hkv"], c["topk"], c["gated"])
+    assert boundary_gap(scores, c["topk"]) >= 1.5e-3
+
+
+@pytest.mark.parametrize("G,d,dtype,lens", [(1, 64, "f32", [2048, 1500]),
+                                            (4, 128, "bf16", [700, 65]),
+                                            (8, 64, "bf16", [1, 2048])])
+def test_decode_bf16_summaries_small(G, d, dtype, lens):
+    x = inputs.gen_decode(2, 2 * G, 2, 2048, d, lens, dtype, seed=64, planted=6)
+    _decode_bf16_summary_check(x, 2, 5, 1, tol=TOL[dtype])
 
 def test_decode_repeat_is_bitwise_stable():
     x = inputs.gen_decode(1, 32, 8, 8192, 128, [8100], "bf16", seed=64, planted=16)

@@ -11,13 +11,15 @@
 // Cluster of CS CTAs (16 when the rows fit the GPU that way, else fewer).
 // CTA c of the cluster:
 //   1. bulk-copies its contiguous range of the row's block summaries through
-//      a three-slot shared-memory ring and scores them against qbar (mean of
+//      a four-slot shared-memory ring and scores them against qbar (mean of
 //      the group's query heads); the current block's K/V, known before any
-//      selection, is prefetched at the same time by the CTA that owns it;
+//      selection, is copied by the CTA that owns it as soon as the ring is
+//      free, under the selection;
 //   2. reduces its range to (max, sum exp) and a best-first list of
-//      min(k, n) candidates, and stores both into its slot of every CTA of
-//      the cluster with asynchronous remote stores that complete on the
-//      receiver's mbarrier;
+//      min(k, n) candidates (the keys at or above the k-th key of a strided
+//      sample, ranked among themselves), and stores both into its slot of
+//      every CTA of the cluster with asynchronous remote stores that
+//      complete on the receiver's mbarrier;
 //   3. once all lists have landed, every CTA computes the gate's LSE and the
 //      same Top-K: the keys above a pruning threshold are ranked among
 //      themselves, giving the kept blocks in score order (CTA 0 also writes
@@ -53,22 +55,23 @@ namespace {
 
 constexpr int FD_THREADS = 256;
 constexpr int FD_WARPS = FD_THREADS / 32;
-constexpr int FD_NS = 3;      // summary ring slots
-constexpr int FD_SUBC = 32;   // summaries per ring slot
+constexpr int FD_NS = 4;      // summary ring slots
 constexpr int FD_MAXKV = 4;   // K/V ring slots at most
 constexpr int FD_MAXCS = 16;  // cluster size at most
 constexpr unsigned FULL = 0xffffffffu;
 
 struct FdSmem {  // byte offsets into dynamic shared memory
   size_t u, q, qbar, sc, mine, slen, stage, sstat, fin, cst, cml, zp, bars, total;
-  size_t wl, wb, tmp, mb, mblen;  // list scratch inside region u, after K/V slot 0
-  int nkv;                        // K/V ring slots held by region u
+  size_t wl, wb, samp, surv;                  // list scratch inside region u, after K/V slot 0
+  int nkv;                                    // K/V ring slots held by region u
+  int subc;                                   // summaries per ring slot
 };
 
 __host__ __device__ inline size_t fd_al(size_t x) { return (x + 127) & ~(size_t)127; }
 
-// Region u: K/V slot 0 followed by the summary ring during the scan, then by
-// the list scratch (warp lists, survivors, merge buffer) during selection;
+// Region u: the summary ring (FD_NS equal slots over the whole region)
+// during the scan; then K/V slot 0 (the current block) followed by the list
+// scratch (warp lists, sample, survivors, merge buffer) during selection;
 // K/V slots 0 .. nkv-1 afterwards; the per-warp states at the end.
 __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int kq, int CS,
                                              int ses) {
@@ -76,16 +79,15 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int k
   const size_t kvslot = (size_t)2 * SAS_BLOCK * D * es;
   L.wl = kvslot;
   L.wb = L.wl + (size_t)FD_WARPS * kq * 8;
-  L.tmp = L.wb + (size_t)FD_WARPS * kq * 8;
-  L.mb = L.tmp + (size_t)CS * kq * 8;
-  L.mblen = L.mb + (size_t)CS * kq * 8;
-  size_t ub = kvslot + (size_t)FD_NS * FD_SUBC * D * ses;
-  if (ub < L.mblen + 128) ub = L.mblen + 128;
-  if (ub < 2 * kvslot) ub = 2 * kvslot;
+  L.samp = fd_al(L.wb + (size_t)FD_WARPS * kq * 8);
+  L.surv = L.samp + 256 * 8;
+  size_t ub = 2 * kvslot;
+  if (ub < L.surv + 512 * 8) ub = L.surv + 512 * 8;
   const size_t comb = (size_t)FD_WARPS * G * (D + 2) * 4;
   if (ub < comb) ub = comb;
   L.nkv = (int)(ub / kvslot);
   if (L.nkv > FD_MAXKV) L.nkv = FD_MAXKV;
+  L.subc = (int)(ub / ((size_t)FD_NS * D * ses));
   size_t o = 0;
   L.u = o; o += fd_al(ub);
   L.q = o; o += fd_al((size_t)G * D * 4);
@@ -192,15 +194,15 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S));
   unsigned char* U = sm + L.u;
   const size_t kvslot = (size_t)2 * TILE * sizeof(T);
-  S* ring = reinterpret_cast<S*>(U + kvslot);
+  S* ring = reinterpret_cast<S*>(U);
+  const int SUBC = L.subc;
   float* q_s = reinterpret_cast<float*>(sm + L.q);
   float* qbar = reinterpret_cast<float*>(sm + L.qbar);
   float* sc = reinterpret_cast<float*>(sm + L.sc);
   unsigned long long* wl = reinterpret_cast<unsigned long long*>(U + L.wl);
   unsigned long long* wb = reinterpret_cast<unsigned long long*>(U + L.wb);
-  unsigned long long* tmp = reinterpret_cast<unsigned long long*>(U + L.tmp);
-  unsigned long long* mb = reinterpret_cast<unsigned long long*>(U + L.mb);
-  int* mblen = reinterpret_cast<int*>(U + L.mblen);
+  unsigned long long* samp = reinterpret_cast<unsigned long long*>(U + L.samp);
+  unsigned long long* surv = reinterpret_cast<unsigned long long*>(U + L.surv);
   unsigned long long* mine = reinterpret_cast<unsigned long long*>(sm + L.mine);
   int* slen = reinterpret_cast<int*>(sm + L.slen);
   unsigned long long* stage = reinterpret_cast<unsigned long long*>(sm + L.stage);
@@ -216,8 +218,8 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   uint64_t* state_bar = list_bar + 1;
   __shared__ float wred_m[FD_WARPS], wred_s[FD_WARPS];
   __shared__ int wlen[FD_WARPS], wlen_b[FD_WARPS];
-  __shared__ int surv_cnt;
-  __shared__ unsigned long long th_s;
+  __shared__ int loc_cnt;
+  __shared__ unsigned long long red8[FD_WARPS];
   __shared__ float cw[FD_MAXCS];                      // combine weights of the CS states
   __shared__ float fw[FD_WARPS * 8], fm[8], fl[8];    // fold weights per (head, warp)
 
@@ -234,19 +236,14 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   }
   const size_t row = (size_t)b * Hkv + r;
   const int nblk = Lmax / SAS_BLOCK;
-  const int n = min(max(lens[b], 1), Lmax);
-  const int t = (n - 1) / SAS_BLOCK;  // current block; C = t history blocks
-  const int C = t;
-  const int ncur = n - t * SAS_BLOCK;
-  const int kk = min(topk, C);
-  const int units = kk + 1;
-  const int per = (C + CS - 1) / CS;  // history blocks scored by each CTA
-  const int m0 = min(C, crank * per), m1 = min(C, m0 + per), nmine = m1 - m0;
-  const int upc = (units + CS - 1) / CS;  // units attended by each CTA
-  const int u0 = min(units, crank * upc), u1 = min(units, u0 + upc), nu = u1 - u0;
-  const bool own_cur = (kk >= u0 && kk < u1);
-  const int nsub = (nmine + FD_SUBC - 1) / FD_SUBC;
-  const int NKV = L.nkv;
+  // This CTA's range of the row's history summaries: a split of the Lmax/64
+  // blocks that does not depend on the sequence length, so that the first
+  // copies start before the length is read. Blocks at or past C are copied
+  // (contiguous caches) but not scored.
+  const int per = per_max;
+  const int m0 = crank * per;
+  const int nstat = max(0, min(nblk, m0 + per) - m0);
+  const int nsub_s = (nstat + SUBC - 1) / SUBC;
   const size_t kvrow = row * (size_t)Lmax * D;
   const S* ks_row = ksum + row * (size_t)nblk * D;
   uint32_t* err = &g_decode_fused_err;
@@ -269,7 +266,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   // summaries [first, first + cnt) of this CTA's range into ring slot `slot`:
   // one bulk copy (contiguous), or one row copy per lane of warp 0 (paged)
   auto issue_summaries = [&](int slot, int first, int cnt) {
-    S* dst = ring + (size_t)slot * FD_SUBC * D;
+    S* dst = ring + (size_t)slot * SUBC * D;
     if constexpr (PAGED) {
       if (lane == 0) mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * sizeof(S)));
       __syncwarp();
@@ -283,13 +280,37 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
   };
 
+
+  if (tid == 0) {
+    for (int i = 0; i < FD_NS; ++i) mbar_init(&sum_bar[i], 1);
+    fence_mbar_init();
+    if constexpr (!PAGED)
+      for (int i = 0; i < min(FD_NS, nsub_s); ++i)
+        issue_summaries(i, i * SUBC, min(SUBC, nstat - i * SUBC));
+  }
+
+  const int n = min(max(lens[b], 1), Lmax);
+  const int t = (n - 1) / SAS_BLOCK;  // current block; C = t history blocks
+  const int C = t;
+  const int ncur = n - t * SAS_BLOCK;
+  const int kk = min(topk, C);
+  const int units = kk + 1;
+  const int nmine = max(0, min(C, m0 + per) - m0);  // blocks this CTA scores
+  const int upc = (units + CS - 1) / CS;  // units attended by each CTA
+  const int u0 = min(units, crank * upc), u1 = min(units, u0 + upc), nu = u1 - u0;
+  const bool own_cur = (kk >= u0 && kk < u1);
+  const int nsub = (nmine + SUBC - 1) / SUBC;
+  // chunks to wait for: the scored ones and, for contiguous caches, every
+  // chunk copied before the length was known
+  const int nwait = PAGED ? nsub : max(nsub, min(FD_NS, nsub_s));
+  const int NKV = L.nkv;
+
   // ---- 0. barriers, expected remote bytes, first copies, q and qbar
   if (tid < CS) {
     const int nm = min(C, (tid + 1) * per) - min(C, tid * per);
     slen[tid] = topk > 0 ? min(topk, nm) : 0;
   }
   if (tid == 0) {
-    for (int i = 0; i < FD_NS; ++i) mbar_init(&sum_bar[i], 1);
     for (int i = 0; i < FD_MAXKV; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], FD_WARPS);
@@ -297,7 +318,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     mbar_init(list_bar, 1);
     mbar_init(state_bar, 1);
     fence_mbar_init();
-    surv_cnt = 0;
+    loc_cnt = 0;
     uint32_t lb = 0;  // every CTA's list and (max, sum exp)
     for (int c = 0; c < CS; ++c) {
       const int nm = min(C, (c + 1) * per) - min(C, c * per);
@@ -305,16 +326,14 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
     mbar_arrive_expect_tx(list_bar, lb);
     if (crank < G) mbar_arrive_expect_tx(state_bar, (uint32_t)CS * (D * 4 + 8));
-    if (own_cur) {  // the current block is unit 0 of this CTA's order, slot 0
-      mbar_arrive_expect_tx(&full[0], (uint32_t)(2 * TILE * sizeof(T)));
-      bulk_g2s(U, kv_tile(kc, t), TILE * sizeof(T), &full[0]);
-      bulk_g2s(U + TILE * sizeof(T), kv_tile(vc, t), TILE * sizeof(T), &full[0]);
+  }
+  if constexpr (PAGED) {
+    if (wid == 0) {
+      __syncwarp();  // lane 0 initialised the barriers
+      for (int i = 0; i < min(FD_NS, nsub); ++i)
+        issue_summaries(i, i * SUBC, min(SUBC, nmine - i * SUBC));
     }
   }
-  if (wid == 0) __syncwarp();  // lane 0 initialised the barriers
-  if (PAGED ? wid == 0 : tid == 0)
-    for (int i = 0; i < min(FD_NS, nsub); ++i)
-      issue_summaries(i, i * FD_SUBC, min(FD_SUBC, nmine - i * FD_SUBC));
   // Barriers are initialised and fenced (fence.mbarrier_init.release.cluster
   // above): other CTAs may store into this one once every thread of the
   // cluster has arrived. A relaxed arrive does not wait for this thread's
@@ -336,45 +355,58 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   }
   __syncthreads();
 
-  // ---- 1. score this CTA's range of history blocks (4 blocks per warp in flight)
+  // ---- 1. score this CTA's range of history blocks. A quarter-warp takes
+  // one summary: its 8 lanes read 16-byte chunks p, p + 8, ... so that each
+  // quarter reads 128 contiguous bytes per load, and the dot product ends in
+  // three shuffle levels (a warp reduces 4 summaries with one chain).
   {
-    float qv[PER];
+    constexpr int SV = Vec16<S>::N;    // summary elements per 16-byte chunk
+    constexpr int NCL = D / (8 * SV);  // chunks per lane
+    const int qw = lane >> 3, p8 = lane & 7;
+    float qv[NCL * SV];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) qv[i] = qbar[lane * PER + i];
-    for (int i = 0; i < nsub; ++i) {
+    for (int c = 0; c < NCL; ++c)
+#pragma unroll
+      for (int e = 0; e < SV; ++e) qv[c * SV + e] = qbar[(c * 8 + p8) * SV + e];
+    for (int i = 0; i < nwait; ++i) {
       const int slot = i % FD_NS;
-      const int cnt_i = min(FD_SUBC, nmine - i * FD_SUBC);
+      const int cnt_i = max(0, min(SUBC, nmine - i * SUBC));
       mbar_wait_data(&sum_bar[slot], (uint32_t)((i / FD_NS) & 1), err);
-      const S* sb = ring + (size_t)slot * FD_SUBC * D;
-      for (int j0 = wid; j0 < cnt_i; j0 += 4 * FD_WARPS) {
-        float part[4];
+      const S* sb = ring + (size_t)slot * SUBC * D;
+#pragma unroll 2
+      for (int j0 = wid * 4; j0 < cnt_i; j0 += 4 * FD_WARPS) {
+        const int j = j0 + qw;
+        float a0 = 0.f, a1 = 0.f;
+        if (j < cnt_i) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = j0 + u * FD_WARPS;
-          float a = 0.f;
-          if (j < cnt_i) {
-            float x[PER];
-            loadn<PER>(sb + (size_t)j * D + lane * PER, x);
+          for (int c = 0; c < NCL; ++c) {
+            float x[SV];
+            Vec16<S>::load(sb + (size_t)j * D + (c * 8 + p8) * SV, x);
 #pragma unroll
-            for (int e = 0; e < PER; ++e) a += x[e] * qv[e];
-          }
-          part[u] = a;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) part[u] = warp_sum(part[u]);
-        if (lane == 0) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = j0 + u * FD_WARPS;
-            if (j < cnt_i) sc[i * FD_SUBC + j] = part[u] * scale + 0.0f;
+            for (int e = 0; e < SV; e += 2) {
+              a0 = fmaf(x[e], qv[c * SV + e], a0);
+              a1 = fmaf(x[e + 1], qv[c * SV + e + 1], a1);
+            }
           }
         }
+        float a = a0 + a1;
+        a += __shfl_xor_sync(FULL, a, 4);
+        a += __shfl_xor_sync(FULL, a, 2);
+        a += __shfl_xor_sync(FULL, a, 1);
+        if (p8 == 0 && j < cnt_i) sc[i * SUBC + j] = a * scale + 0.0f;
       }
       __syncthreads();  // slot consumed
       if ((PAGED ? wid == 0 : tid == 0) && i + FD_NS < nsub)
-        issue_summaries(slot, (i + FD_NS) * FD_SUBC,
-                        min(FD_SUBC, nmine - (i + FD_NS) * FD_SUBC));
+        issue_summaries(slot, (i + FD_NS) * SUBC, min(SUBC, nmine - (i + FD_NS) * SUBC));
     }
+  }
+  // The ring is consumed (the scan's last barrier): K/V slot 0 takes the
+  // current block, unit 0 of this CTA's order when it owns it; the copy
+  // overlaps the selection below.
+  if (tid == 0 && own_cur) {
+    mbar_arrive_expect_tx(&full[0], (uint32_t)(2 * TILE * sizeof(T)));
+    bulk_g2s(U, kv_tile(kc, t), TILE * sizeof(T), &full[0]);
+    bulk_g2s(U + TILE * sizeof(T), kv_tile(vc, t), TILE * sizeof(T), &full[0]);
   }
 
   // ---- 2. this range's (max, sum exp) and best-first list
@@ -391,38 +423,95 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       wred_s[wid] = ls;
     }
   }
+  // Top-k of nl descending lists of stride kq (a tree of bitonic merges;
+  // the buffers and length arrays are overwritten)
+  auto merge_lists = [&](unsigned long long* A, int* len, unsigned long long* B, int* Blen,
+                         int nl, unsigned long long* out) {
+    if (lg <= 5) merge_tree_topk<1>(A, len, B, Blen, nl, lg, topk, out);
+    else if (lg == 6) merge_tree_topk<2>(A, len, B, Blen, nl, lg, topk, out);
+    else merge_tree_topk<4>(A, len, B, Blen, nl, lg, topk, out);
+  };
   const int my_len = topk > 0 ? min(topk, nmine) : 0;
   const unsigned long long* mylist = mine;
   if (topk > 0 && nmine <= 64) {
-    // small range: one rank-counting pass over the whole range
-    if (tid < nmine) {
-      const float sj = sc[tid];
-      int rk = 0;
-#pragma unroll 8
-      for (int x = 0; x < nmine; ++x) {
+    // small range: each key counts the keys above it, four threads per key
+    // (a quarter of the range each)
+    const int c = tid >> 2, qd = tid & 3;
+    float sj = 0.f;
+    int rk = 0;
+    if (c < nmine) {
+      sj = sc[c];
+      const int x1 = min(nmine, qd * 16 + 16);
+#pragma unroll 4
+      for (int x = qd * 16; x < x1; ++x) {
         const float sx = sc[x];
-        rk += (sx > sj) || (sx == sj && x < tid);
+        rk += (sx > sj) || (sx == sj && x < c);
       }
-      if (rk < topk) mine[rk] = cand_key(sj, m0 + tid);
     }
-  } else if (topk > 0) {
-    // each warp ranks its contiguous share, then one merge of the 8 lists
+    rk += __shfl_xor_sync(FULL, rk, 1);
+    rk += __shfl_xor_sync(FULL, rk, 2);
+    if (c < nmine && qd == 0 && rk < topk) mine[rk] = cand_key(sj, m0 + c);
+  } else if (topk > 0 && nmine <= 64 * FD_WARPS) {
+    // each warp sorts its share (at most 64 keys) in registers; the 8
+    // sorted lists are merged by rank
     const int pw = (nmine + FD_WARPS - 1) / FD_WARPS;
-    const int a0 = min(nmine, wid * pw), a1 = min(nmine, a0 + pw);
-    for (int j = a0 + lane; j < a1; j += 32) {
-      const float sj = sc[j];
-      int rk = 0;
-      for (int x = a0; x < a1; ++x) {
-        const float sx = sc[x];
-        rk += (sx > sj) || (sx == sj && x < j);
-      }
-      if (rk < topk) wl[wid * kq + rk] = cand_key(sj, m0 + j);
+    const int a0 = min(nmine, wid * pw), cnt = min(nmine, a0 + pw) - a0;
+    unsigned long long v[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int i = j * 32 + lane;
+      v[j] = i < cnt ? cand_key(sc[a0 + i], m0 + a0 + i) : 0ull;
     }
-    if (lane == 0) wlen[wid] = min(topk, a1 - a0);
+    warp_sort64_desc(v);
+    const int wlen_w = min(topk, cnt);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (j * 32 + lane < wlen_w) wl[wid * kq + j * 32 + lane] = v[j];
+    if (lane == 0) wlen[wid] = wlen_w;
     __syncthreads();
-    mylist = tree_merge(wl, wlen, wb, wlen_b, FD_WARPS, lg, topk) ? wb : wl;
+    merge_lists(wl, wlen, wb, wlen_b, FD_WARPS, mine);
+  } else if (topk > 0) {
+    // A lower bound of the k-th key: the k-th key of a strided sample of at
+    // most 256 of the range's keys. The keys at or above it are ranked.
+    const int st = (nmine + 255) / 256;
+    const int ns = (nmine + st - 1) / st;
+    for (int i = tid; i < ns; i += FD_THREADS) samp[i] = cand_key(sc[i * st], m0 + i * st);
+    __syncthreads();
+    const unsigned long long th_loc = block_max_u64(sample_kth(samp, ns, topk), red8);
+    auto key_of = [&](int e, unsigned long long& key) -> bool {
+      key = cand_key(sc[e], m0 + e);
+      return true;
+    };
+    if (!rank_survivors(key_of, nmine, th_loc, topk, mine, surv, &loc_cnt)) {
+      // more than 512 keys at or above the bound: each warp ranks its
+      // contiguous share, then one merge of the 8 lists
+      const int pw = (nmine + FD_WARPS - 1) / FD_WARPS;
+      const int a0 = min(nmine, wid * pw), a1 = min(nmine, a0 + pw);
+      for (int j = a0 + lane; j < a1; j += 32) {
+        const float sj = sc[j];
+        int rk = 0;
+        for (int x = a0; x < a1; ++x) {
+          const float sx = sc[x];
+          rk += (sx > sj) || (sx == sj && x < j);
+        }
+        if (rk < topk) wl[wid * kq + rk] = cand_key(sj, m0 + j);
+      }
+      if (lane == 0) wlen[wid] = min(topk, a1 - a0);
+      __syncthreads();
+      mylist = tree_merge(wl, wlen, wb, wlen_b, FD_WARPS, lg, topk) ? wb : wl;
+    }
   }
   __syncthreads();
+  // The head of this CTA's list is likely among the kept blocks: its K/V
+  // starts towards L2 now, under the exchange and the merge (the CTA that
+  // attends a block after the merge may be another one).
+  if (tid < min(my_len, (topk + CS - 1) / CS + 1)) {
+    const int blk = key_block(mylist[tid]);
+    if (blk >= 0 && blk < nblk) {
+      bulk_prefetch_l2(kv_tile(kc, blk), TILE * sizeof(T));
+      bulk_prefetch_l2(kv_tile(vc, blk), TILE * sizeof(T));
+    }
+  }
 
   // ---- push this CTA's list and (max, sum exp) into its slot of every CTA
   cluster_wait_acquire();  // every CTA of the cluster has initialised its barriers
@@ -445,8 +534,8 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         ms_merge(m4[0], s4[0], m4[2], s4[2]);
         ms_merge(m4[1], s4[1], m4[3], s4[3]);
         ms_merge(m4[0], s4[0], m4[1], s4[1]);
-        const float M = m4[0], S = s4[0];
-        st_async_f32x2(mapa(sst, c), M, S, mapa(lbar, c));
+        const float M = m4[0], Z = s4[0];
+        st_async_f32x2(mapa(sst, c), M, Z, mapa(lbar, c));
       }
     }
   }
@@ -458,14 +547,14 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const float mx = lane < CS ? sstat[2 * lane] : -FLT_MAX;
     const float se = lane < CS ? sstat[2 * lane + 1] : 0.f;
     const float M = warp_max(mx);
-    const float S = warp_sum(se > 0.f ? se * __expf(mx - M) : 0.f);
-    lse = (C > 0) ? M + __logf(S) : 0.f;
+    const float Z = warp_sum(se > 0.f ? se * __expf(mx - M) : 0.f);
+    lse = (C > 0) ? M + __logf(Z) : 0.f;
   }
   // Units are taken in score order (fin[u], best first): a CTA knows its
   // blocks as soon as the merge ends. Ascending block order is needed only
   // for idx_out, which CTA 0 writes.
   if (topk > 0 && kk > 0)
-    topk_of_lists(stage, slen, CS, lg, topk, fin, tmp, mb, mblen, &surv_cnt, &th_s);
+    merge_lists(stage, slen, wl, wlen_b, CS, fin);
 
   // ---- 4. attention over this CTA's units: the current block first when
   // owned (already in flight in slot 0), then its kept blocks in score order.
@@ -486,8 +575,10 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     bulk_g2s(dst, kv_tile(kc, blk), TILE * sizeof(T), &full[slot]);
     bulk_g2s(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), &full[slot]);
   };
-  if (tid == 0)
+  if (tid == 0) {
+    fence_proxy_async_smem();  // the list scratch written above becomes K/V slots
     for (int i = own_cur ? 1 : 0; i < min(NKV, nu); ++i) issue_unit(i);
+  }
   if (crank == 0 && idx_out != nullptr && topk > 0) {  // kept blocks, ascending, -1 padded
     for (int i = tid; i < topk; i += FD_THREADS) {
       if (i >= kk) {

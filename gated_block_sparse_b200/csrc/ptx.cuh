@@ -97,6 +97,12 @@ __device__ __forceinline__ bool mbar_wait_data(uint64_t* bar, uint32_t parity, u
   return false;
 }
 
+// Asynchronous hint to bring `bytes` (multiple of 16, address 16-byte
+// aligned) of global memory into L2; no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
 // global to this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,

@@ -355,6 +355,15 @@ def test_decode_bf16_summaries_small(G, d, dtype, lens):
     x = inputs.gen_decode(2, 2 * G, 2, 2048, d, lens, dtype, seed=64, planted=6)
     _decode_bf16_summary_check(x, 2, 5, 1, tol=TOL[dtype])
 
+@pytest.mark.parametrize("Lmax,d,topk,G", [(589824, 64, 63, 2), (262144, 128, 128, 4)])
+def test_decode_long_rows_and_large_topk(Lmax, d, topk, G):
+    """One long row: more than 512 history blocks per CTA of the cluster (the
+    per-CTA list then comes from a sampled bound), and the largest top-k (128:
+    lists longer than one warp's sorted share)."""
+    x = inputs.gen_decode(1, G, 1, Lmax, d, [Lmax - 5], "bf16", seed=66, planted=2 * topk)
+    scores = _decode_check(x, 1, topk, 1)
+    assert boundary_gap(scores, topk) >= 1.5e-3
+
 def test_decode_repeat_is_bitwise_stable():
     x = inputs.gen_decode(1, 32, 8, 8192, 128, [8100], "bf16", seed=64, planted=16)
     ks = sas.sas_block_summary(dev(x["kc"]))

@@ -226,6 +226,12 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int r = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * G;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // Programmatic dependent launch: the next kernel of the stream may be
+  // scheduled now (it waits for this grid's completion before its own first
+  // global read), and this grid reads nothing the previous one may still
+  // write before that grid has completed.
+  grid_dep_launch();
+  grid_dep_wait();
   // the group's queries and the sequence length first: both loads in flight together
   constexpr int QPT = (G * D + FD_THREADS - 1) / FD_THREADS;
   float qreg[QPT];
@@ -885,13 +891,15 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   cfg.blockDim = dim3(FD_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
                             static_cast<const T*>(vc), static_cast<const S*>(ksum), Hkv, Lmax,
                             lens, topk, gated, scale,

@@ -111,6 +111,26 @@ sas_status sas_block_summary_ex(const void* k, sas_dtype dt, int B, int H, int N
                      "sas_block_summary_ex launch");
 }
 
+sas_status sas_block_summary_last(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                                  const int32_t* lens, void* ksum, sas_dtype sum_dt,
+                                  const int32_t* block_table, int npages, sas_stream_t stream) {
+  g_last_error.clear();
+  REQUIRE(sum_dt == SAS_F32 || sum_dt == SAS_BF16, SAS_ERR_INVALID_ARG,
+          "summary dtype must be SAS_F32 or SAS_BF16");
+  sas_status s = check_common(dt, B, H, H, N, d, 0);
+  if (s != SAS_OK) return s;
+  REQUIRE(N % 64 == 0, SAS_ERR_INVALID_ARG, "N must be a multiple of 64 (got %d)", N);
+  if (block_table) REQUIRE(npages >= 1, SAS_ERR_INVALID_ARG, "npages must be >= 1 (got %d)", npages);
+  if (B == 0 || N < 128) return SAS_OK;
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(lens);
+  return cuda_status(sas::launch_summary_last(k, dt == SAS_BF16, B, H, N, d, lens, ksum,
+                                              sum_dt == SAS_BF16, block_table, N / 64, npages,
+                                              (cudaStream_t)stream),
+                     "sas_block_summary_last launch");
+}
+
 size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_mode mode) {
   if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || topk < 0) return 0;
   if (mode == SAS_PREFILL) return a16(sas::select_prefill_ws_bytes(B, Hkv, N, d));
@@ -485,6 +505,7 @@ sas_status sas_device_status(int clear, sas_stream_t stream) {
       {"k_attn_bwd_tc", sas::attn_bwd_tc_error_word},
       {"k_attn_simt", sas::attn_simt_error_word},
       {"k_wait_selftest", sas::selftest_error_word},
+      {"k_summary_last", sas::summary_error_word},
   };
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "sas_device_status synchronize");

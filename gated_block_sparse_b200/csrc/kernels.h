@@ -22,6 +22,13 @@ cudaError_t launch_block_summary(const void* k, int bf16, int B, int H, int N, i
 // The same, summaries stored in bf16 (the fp32 mean rounded to nearest even).
 cudaError_t launch_block_summary_bf16(const void* k, int bf16, int B, int H, int N, int d,
                                       const int32_t* lens, void* ksum, cudaStream_t st);
+// Summary of each (sequence, head)'s last complete block, (lens[b]-1)/64 - 1
+// (nothing when there is none); paged when bt != nullptr.
+cudaError_t launch_summary_last(const void* k, int bf16, int B, int H, int N, int d,
+                                const int32_t* lens, void* ksum, int sum_bf16,
+                                const int32_t* bt, int max_blocks, int npages,
+                                cudaStream_t st);
+uint32_t* summary_error_word();
 
 // ---- selection
 // Shared layout of one row's per-chunk partial results (decode scratch).

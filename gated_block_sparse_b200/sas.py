@@ -48,6 +48,7 @@ SIGNATURES = {
     "sas_decode_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P,
                              _P, _P]),
     "sas_block_summary_ex": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "sas_block_summary_last": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _P]),
     "sas_decode_ex": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P,
                            _P]),
     "sas_select_bwd_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
@@ -269,6 +270,26 @@ def sas_block_summary_ex(k, sum_dtype=torch.float32, lens=None, out=None, stream
     _check("sas_block_summary_ex", lib.sas_block_summary_ex(
         _ptr(k), _dt(k), B, H, N, d, _ptr(lens), _ptr(out), _dt(out), _stream(stream)))
     return out
+
+
+def sas_block_summary_last(k, lens, ksum, block_table=None, npages: int = 0, stream=None):
+    """Refresh each row's last complete block summary in place (decode upkeep).
+
+    Contiguous: k [B][H][N][d], ksum [B][H][N/64][d]. Paged (block_table
+    [B][max_blocks]): k is the pool [npages][H][64][d], ksum [npages][H][d],
+    N = 64 * max_blocks. ksum's dtype (fp32 or bf16) is the summary type.
+    """
+    lib = load_library()
+    if block_table is None:
+        B, H, N, d = k.shape
+    else:
+        B, N = block_table.shape[0], 64 * block_table.shape[1]
+        npages = npages or k.shape[0]
+        H, d = k.shape[1], k.shape[3]
+    _check("sas_block_summary_last", lib.sas_block_summary_last(
+        _ptr(k), _dt(k), B, H, N, d, _ptr(lens), _ptr(ksum), _dt(ksum), _ptr(block_table),
+        int(npages), _stream(stream)))
+    return ksum
 
 
 def sas_decode_ex(q, kc, vc, lens, ksum, topk: int, gated: int = 1, scale: float = 0.0, out=None,

@@ -231,6 +231,26 @@ sas_status sas_decode_ex(const void* q, const void* kc, const void* vc, sas_dtyp
                          int32_t* idx_out, sas_stream_t stream);
 
 /*
+ * Summary upkeep during decode (SAS close reading, section 2.4: serving keeps
+ * the block summaries beside the cache). For every (sequence b, head h),
+ * writes the summary of block C - 1, C = (lens[b] - 1) / 64: the last
+ * complete block before the current one, which completed when the current
+ * block began. Rows with C = 0 are left alone. Calling it once per decode
+ * step keeps the summaries current as long as at most 64 tokens are appended
+ * between calls (sas_block_summary rebuilds all of them otherwise).
+ *   block_table NULL: k [B][H][N][d] (dt), ksum [B][H][N/64][d] (sum_dt).
+ *   block_table [B][N/64] int32: k is the page pool [npages][H][64][d] and
+ *     ksum the page summaries [npages][H][d]; the block's page is
+ *     block_table[b][C - 1]. An entry outside [0, npages) skips the row and
+ *     is reported by sas_device_status (kernel k_summary_last).
+ *   lens [B] int32 device, 1 <= lens[b] <= N; N a multiple of 64.
+ *   sum_dt SAS_F32 or SAS_BF16 (the fp32 mean rounded to nearest even).
+ */
+sas_status sas_block_summary_last(const void* k, sas_dtype dt, int B, int H, int N, int d,
+                                  const int32_t* lens, void* ksum, sas_dtype sum_dt,
+                                  const int32_t* block_table, int npages, sas_stream_t stream);
+
+/*
  * One decode step from and to host memory: enqueues on `stream` the copy of
  * q_host ([B][Hq][d], dt; page-locked for the copy to be asynchronous) into
  * q_dev and the sas_decode step. When o_host is page-locked host memory

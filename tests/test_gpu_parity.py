@@ -550,3 +550,71 @@ def test_decode_host_buffers_match_device_call():
     sas.sas_decode_host(qh, qd, kc, vc, lens, ks, 15, od, oh)
     torch.cuda.synchronize()
     assert torch.equal(oh, o_ref)
+
+
+# ------------------------------------------------------------------ summary upkeep
+def _last_block_expect(got, ref, sum_dtype):
+    """got, ref: one block's summaries (fp64); bf16 storage allows the one-ulp
+    rounding difference of test_block_summary_bf16."""
+    if sum_dtype == torch.bfloat16:
+        r = O.round_bf16(ref)
+        return bool(np.all(np.abs(got - r) <= _bf16_ulp(r) * 1.0001))
+    return maxerr(got, ref) < 1e-5
+
+
+@pytest.mark.parametrize("sum_dtype", [torch.float32, torch.bfloat16])
+def test_summary_last_contiguous(sum_dtype):
+    """Only each row's last complete block (C - 1, C = (n - 1) // 64) is
+    rewritten; rows with C = 0 and every other block keep their contents."""
+    B, H, N, d = 4, 2, 1024, 128
+    k = inputs.gen_prefill(B, H, H, N, d, "bf16", seed=14)["k"]
+    lens = torch.tensor([1, 65, 129, 1000], dtype=torch.int32)  # C = 0, 1, 2, 15
+    ks = torch.full((B, H, N // 64, d), 7.0, dtype=sum_dtype, device=DEV)
+    sas.sas_block_summary_last(dev(k), dev(lens), ks)
+    torch.cuda.synchronize()
+    ref, got = O.block_summary(k), np64(ks)
+    for b, n in enumerate(lens.tolist()):
+        C = (n - 1) // 64
+        for m in range(N // 64):
+            if m == C - 1:
+                assert _last_block_expect(got[b, :, m], ref[b, :, m], sum_dtype)
+            else:
+                assert (got[b, :, m] == 7.0).all()
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg
+
+
+def test_summary_last_paged_and_bad_entry():
+    """Paged: the page of block C - 1 gets the summary; a block-table entry
+    out of range skips its row and is reported, then cleared."""
+    B, H, N, d = 3, 2, 1024, 128
+    x = inputs.gen_decode(B, 2 * H, H, N, d, [700, 1024, 64], "bf16", seed=74)
+    kc, vc, lens = x["kc"], x["vc"], x["lens"]
+    kpool, _, bt = _to_pages(kc, vc, lens, seed=75)
+    ks = torch.full((kpool.shape[0], H, d), 7.0, dtype=torch.float32, device=DEV)
+    sas.sas_block_summary_last(dev(kpool), dev(lens), ks, block_table=dev(torch.from_numpy(bt)))
+    torch.cuda.synchronize()
+    ref, got = O.block_summary(kc), np64(ks)
+    touched = set()
+    for b, n in enumerate(lens.tolist()):
+        C = (n - 1) // 64
+        if C > 0:
+            p = int(bt[b, C - 1])
+            touched.add(p)
+            assert maxerr(got[p], ref[b, :, C - 1]) < 1e-5
+    for p in range(kpool.shape[0]):
+        if p not in touched:
+            assert (got[p] == 7.0).all()
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg
+    bad = bt.copy()
+    bad[1, (1024 - 1) // 64 - 1] = kpool.shape[0]  # one past the pool
+    ks2 = torch.full_like(ks, 7.0)
+    sas.sas_block_summary_last(dev(kpool), dev(lens), ks2, block_table=dev(torch.from_numpy(bad)))
+    st, msg = sas.sas_device_status(clear=True)
+    assert st != 0 and "k_summary_last" in msg
+    got2 = np64(ks2)
+    assert maxerr(got2[int(bt[0, (700 - 1) // 64 - 1])], ref[0, :, (700 - 1) // 64 - 1]) < 1e-5
+    assert (got2[int(bt[1, (1024 - 1) // 64 - 1])] == 7.0).all()
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg

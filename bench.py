@@ -113,7 +113,7 @@ class ClockSampler:
         except Exception:
             rows = []
         win = [x for t, x in rows if t0 - 0.15 <= t <= t1 + 0.15] or \
-              [x for t, x in rows if t >= t0][:1] or rows[-1:]
+              [x for t, x in rows if t >= t0][:1] or [x for _, x in rows[-1:]]
         if not win:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]

@@ -508,10 +508,11 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
   }
   __syncthreads();
-  // The head of this CTA's list is likely among the kept blocks: its K/V
-  // starts towards L2 now, under the exchange and the merge (the CTA that
-  // attends a block after the merge may be another one).
-  if (tid < min(my_len, (topk + CS - 1) / CS + 1)) {
+  // The head of this CTA's list (its first ceil(k/CS) keys, the share a
+  // CTA holds when the kept blocks spread evenly) is likely among the kept
+  // blocks: its K/V starts towards L2 now, under the exchange and the merge
+  // (the CTA that attends a block after the merge may be another one).
+  if (tid < min(my_len, (topk + CS - 1) / CS)) {
     const int blk = key_block(mylist[tid]);
     if (blk >= 0 && blk < nblk) {
       bulk_prefetch_l2(kv_tile(kc, blk), TILE * sizeof(T));

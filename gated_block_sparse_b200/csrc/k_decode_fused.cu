@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   __shared__ int loc_cnt;
   __shared__ unsigned long long red8[FD_WARPS];
   __shared__ float cw[FD_MAXCS];                      // combine weights of the CS states
-  __shared__ float fw[FD_WARPS * 8], fm[8], fl[8];    // fold weights per (head, warp)
+  __shared__ float2 mlw[8 * FD_WARPS];               // (m, l) per (head, warp) for the fold
 
   const int r = blockIdx.y, b = blockIdx.z;
   const int Hq = Hkv * G;
@@ -709,46 +709,20 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     }
   }
 
-  // ---- 5. fold the warp states per head; push head h's state into CTA h
+  // ---- 5. fold the warp states per head; push head h's state into CTA h.
+  // Every thread of the fold takes (head, 4 columns) and derives the 8 warp
+  // weights itself from the warps' (m, l).
   __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
-  float* wst = reinterpret_cast<float*>(U);  // [warp][head][D + 2]: acc, m, l
+  float* wst = reinterpret_cast<float*>(U);  // [warp][head][D] acc
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    float* w = wst + (size_t)(wid * G + h) * (D + 2);
+    float* w = wst + (size_t)(wid * G + h) * D;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) w[lane * CPL + c] = acc[h][c];
-    if (lane == 0) {
-      w[D] = m_w[h];
-      w[D + 1] = l_w[h];
-    }
   }
-  __syncthreads();
-  if (wid == 0) {  // fold weights: lane = (head within a group of 4, warp)
-    for (int h0 = 0; h0 < G; h0 += 4) {
-      const int h = h0 + (lane >> 3), w = lane & 7;
-      float m = -INFINITY, l = 0.f;
-      if (h < G) {
-        const float* ws = wst + (size_t)(w * G + h) * (D + 2);
-        l = ws[D + 1];
-        if (l > 0.f) m = ws[D];
-      }
-      float M = m;
-      M = fmaxf(M, __shfl_xor_sync(FULL, M, 1));
-      M = fmaxf(M, __shfl_xor_sync(FULL, M, 2));
-      M = fmaxf(M, __shfl_xor_sync(FULL, M, 4));
-      const float f = l > 0.f ? __expf(m - M) : 0.f;
-      float Ls = l * f;
-      Ls += __shfl_xor_sync(FULL, Ls, 1);
-      Ls += __shfl_xor_sync(FULL, Ls, 2);
-      Ls += __shfl_xor_sync(FULL, Ls, 4);
-      if (h < G) {
-        fw[h * 8 + w] = f;
-        if (w == 0) {
-          fm[h] = M;
-          fl[h] = Ls;
-        }
-      }
-    }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) mlw[h * FD_WARPS + wid] = make_float2(m_w[h], l_w[h]);
   }
   __syncthreads();
   {
@@ -757,18 +731,26 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const uint32_t sbar = smem_u32(state_bar);
     for (int e = tid; e < G * (D / 4); e += FD_THREADS) {
       const int h = e / (D / 4), c4 = (e % (D / 4)) * 4;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      float2 ml[FD_WARPS];
+      float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < FD_WARPS; ++w) {
-        const float* ws = wst + (size_t)(w * G + h) * (D + 2) + c4;
-        const float f = fw[h * 8 + w];
-        a0 += ws[0] * f;
-        a1 += ws[1] * f;
-        a2 += ws[2] * f;
-        a3 += ws[3] * f;
+        ml[w] = mlw[h * FD_WARPS + w];
+        if (ml[w].y > 0.f) M = fmaxf(M, ml[w].x);
+      }
+      float Ls = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int w = 0; w < FD_WARPS; ++w) {
+        const float f = ml[w].y > 0.f ? __expf(ml[w].x - M) : 0.f;
+        const float4 x = *reinterpret_cast<const float4*>(wst + (size_t)(w * G + h) * D + c4);
+        Ls += ml[w].y * f;
+        a0 += x.x * f;
+        a1 += x.y * f;
+        a2 += x.z * f;
+        a3 += x.w * f;
       }
       st_async_f32x4(mapa(cst_r + 4u * c4, h), a0, a1, a2, a3, mapa(sbar, h));
-      if (c4 == 0) st_async_f32x2(mapa(cml_r, h), fm[h], fl[h], mapa(sbar, h));
+      if (c4 == 0) st_async_f32x2(mapa(cml_r, h), M, Ls, mapa(sbar, h));
     }
   }
   cluster_arrive_relaxed();  // pairs with the wait at exit; carries no data

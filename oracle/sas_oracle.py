@@ -22,7 +22,7 @@ Plain, slow and written to be checked by eye against the pages:
   inference the continuous bias may be dropped and plain softmax attention
   runs over the Top-K blocks and the current block (`gated=0`).
 
-Readings where the pages leave a step open (each listed in the design doc):
+Readings where the pages leave a step open:
 * block size b = 64 (section 3.1); the selector is parameter-free:
   s_m = scale * qbar . kbar_m, kbar_m = mean of block m's 64 keys,
   qbar = mean of the kv group's query heads (and, in prefill, of the query

@@ -477,3 +477,123 @@ def select_backward(q, k, idx, cnt, dlogg, Hkv: int, scale: float | None = None,
     if return_ds:
         return dq, dk, ds_rows
     return dq, dk
+
+
+# --------------------------------------------------------------------------
+# Per-token selection in prefill (section 2.4: the fused kernel masks the
+# blocks a query did not select by that query's gate threshold, and skips a
+# key tile that no query of the tile selected). Every query token i of kv
+# group r selects its own blocks: qbar_i = mean of the group's G heads at
+# token i, C_i = i // 64 visible history blocks, the same gate and Top-K
+# rule as above. Layouts: idx/logg/dlogg [B][Hkv][N][k], cnt [B][Hkv][N].
+# --------------------------------------------------------------------------
+def select_prefill_tokens(q, ksum, Hkv: int, topk: int, scale: float | None = None):
+    """Per (b, kv group r, query token i): scores, gate and Top-K over the
+    C_i = i // 64 history blocks. Returns idx, cnt, logg and the scores
+    {(b, r, i): s}."""
+    q = _f64(q)
+    ksum = _f64(ksum)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    scale = _scale(d, scale)
+    idx = np.full((B, Hkv, N, topk), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hkv, N), dtype=np.int32)
+    logg = np.zeros((B, Hkv, N, topk))
+    scores = {}
+    for b in range(B):
+        for r in range(Hkv):
+            for i in range(N):
+                qbar = q[b, r * G:(r + 1) * G, i].mean(axis=0)
+                C = i // BLOCK
+                s = scale * (ksum[b, r, :C] @ qbar)
+                chosen, lg, _ = gate_and_topk(s, topk)
+                kk = chosen.shape[0]
+                idx[b, r, i, :kk] = chosen
+                cnt[b, r, i] = kk
+                logg[b, r, i, :kk] = lg
+                scores[(b, r, i)] = s
+    return idx, cnt, logg, scores
+
+
+def _token_keys(i, sel, sel_logg):
+    """Key positions of query token i and their bias: each selected history
+    block's 64 tokens (bias log g_m), then the current block's tokens up to
+    and including i (bias 0, causal)."""
+    pos, bias = [], []
+    for m, lg in zip(sel, sel_logg):
+        pos.append(np.arange(m * BLOCK, (m + 1) * BLOCK))
+        bias.append(np.full(BLOCK, float(lg)))
+    cur = np.arange((i // BLOCK) * BLOCK, i + 1)
+    pos.append(cur)
+    bias.append(np.zeros(cur.shape[0]))
+    return np.concatenate(pos), np.concatenate(bias)
+
+
+def _one_row(qi, kS, vS, bias, scale, dot=None, o_for_D=None):
+    """One query row over its key set: z = scale k.q + bias, p = softmax(z),
+    o = p V, lse = log sum e^z; with dot, the backward of L = dO . o:
+    D = dO . o, dz = p (V dO - D), dq = scale dz K, dK = scale dz q^T,
+    dV = p dO^T (o_for_D: the stored output used in D, if given)."""
+    z = scale * (kS @ qi) + bias
+    mx = z.max()
+    e = np.exp(z - mx)
+    ssum = e.sum()
+    p = e / ssum
+    o = p @ vS
+    lse = mx + np.log(ssum)
+    if dot is None:
+        return o, lse
+    D = dot @ (o if o_for_D is None else o_for_D)
+    dz = p * (vS @ dot - D)
+    return o, lse, scale * (dz @ kS), scale * np.outer(dz, qi), np.outer(p, dot), dz
+
+
+def attn_fwd_tokens(q, k, v, idx, cnt, logg, scale: float | None = None):
+    """o and lse of every head's rows, each query token over its own kept
+    blocks (bias log g) and the causal part of its current block."""
+    q, k, v, logg = _f64(q), _f64(k), _f64(v), _f64(logg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    G = Hq // k.shape[1]
+    scale = _scale(d, scale)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            r = h // G
+            for i in range(N):
+                kk = int(cnt[b, r, i])
+                pos, bias = _token_keys(i, idx[b, r, i, :kk], logg[b, r, i, :kk])
+                o[b, h, i], lse[b, h, i] = _one_row(q[b, h, i], k[b, r, pos], v[b, r, pos],
+                                                    bias, scale)
+    return o, lse
+
+
+def attn_bwd_tokens(q, k, v, do, idx, cnt, logg, scale: float | None = None, o_stored=None):
+    """Gradients of L = sum(dO * o) with o from attn_fwd_tokens; dlogg[b, r,
+    i, slot] sums dz over the group's heads and the slot's 64 keys of row i.
+    o_stored: the forward output as stored, used in D (optional)."""
+    q, k, v, do, logg = _f64(q), _f64(k), _f64(v), _f64(do), _f64(logg)
+    if o_stored is not None:
+        o_stored = _f64(o_stored)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    G = Hq // k.shape[1]
+    scale = _scale(d, scale)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dlogg = np.zeros(logg.shape)
+    for b in range(B):
+        for h in range(Hq):
+            r = h // G
+            for i in range(N):
+                kk = int(cnt[b, r, i])
+                pos, bias = _token_keys(i, idx[b, r, i, :kk], logg[b, r, i, :kk])
+                _, _, dqi, dkS, dvS, dz = _one_row(
+                    q[b, h, i], k[b, r, pos], v[b, r, pos], bias, scale, dot=do[b, h, i],
+                    o_for_D=None if o_stored is None else o_stored[b, h, i])
+                dq[b, h, i] = dqi
+                np.add.at(dk[b, r], pos, dkS)
+                np.add.at(dv[b, r], pos, dvS)
+                for slot in range(kk):
+                    dlogg[b, r, i, slot] += dz[slot * BLOCK:(slot + 1) * BLOCK].sum()
+    return dq, dk, dv, dlogg

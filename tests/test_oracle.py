@@ -16,7 +16,10 @@ normalised over the wrong set) fails at least one of them:
 * the paper's eq. 5 form of the gate gradient (SAS close reading,
   liuzhao09.github.io, section 2.2): dL/dg_m = sum_{i in B_m} p~_i/g_m do.(v_i - o);
 * gate invariants: sum g = 1, shift invariance (section 2.2), Top-K of s equals
-  Top-K of g (order preservation, MSA notes, papercache, Top-K kernel section).
+  Top-K of g (order preservation, MSA notes, papercache, Top-K kernel section);
+* per-token selection (section 2.4, the fused kernel's per-query threshold):
+  reduction to the per-block oracle when every query block's rows are equal,
+  the dense N x N masked logit matrix, and central finite differences.
 """
 import numpy as np
 import pytest
@@ -513,3 +516,101 @@ def test_round_bf16_matches_library_conversion():
     got = O.round_bf16(xs.astype(np.float64))
     assert np.array_equal(got, want)
     assert got[-5] == 1.0 and got[-4] == 1.0 + 2 * 2.0 ** -7 and got[-3] == -2.0
+
+
+# ------------------------------------------------------------------ per-token selection
+def _tok_case(N, d, Hq, Hkv, topk, seed, const_blocks=False):
+    B = 1
+    q, k, v, do = (rnd((B, Hq, N, d), seed), rnd((B, Hkv, N, d), seed + 1),
+                   rnd((B, Hkv, N, d), seed + 2), rnd((B, Hq, N, d), seed + 3))
+    if const_blocks:  # every query block's rows repeat its first row, per head
+        for t in range(-(-N // BLOCK)):
+            q[:, :, t * BLOCK:(t + 1) * BLOCK] = q[:, :, t * BLOCK:t * BLOCK + 1]
+    return q, k, v, do
+
+
+def test_tokens_equal_blocks_when_queries_are_constant_in_each_block():
+    """With q constant across each 64-token query block, every token's own
+    selection is its block's selection; outputs and gradients match the
+    per-block oracle, and the per-block d(log g) is the sum over the block's
+    tokens."""
+    N, d, Hq, Hkv, topk = 300, 16, 4, 2, 2
+    q, k, v, do = _tok_case(N, d, Hq, Hkv, topk, 900, const_blocks=True)
+    ks = O.block_summary(k)
+    bi, bc, bl, _ = O.select_prefill(q, ks, Hkv, topk)
+    ti, tc, tl, _ = O.select_prefill_tokens(q, ks, Hkv, topk)
+    for i in range(N):
+        t = i // BLOCK
+        assert np.array_equal(ti[:, :, i], bi[:, :, t]) and np.array_equal(tc[:, :, i], bc[:, :, t])
+        assert np.allclose(tl[:, :, i], bl[:, :, t], rtol=0, atol=1e-12)
+    ob, lb = O.attn_fwd(q, k, v, bi, bc, bl)
+    ot, lt = O.attn_fwd_tokens(q, k, v, ti, tc, tl)
+    assert np.abs(ob - ot).max() < 1e-12 and np.abs(lb - lt).max() < 1e-12
+    gb = O.attn_bwd(q, k, v, do, bi, bc, bl)
+    gt = O.attn_bwd_tokens(q, k, v, do, ti, tc, tl)
+    for a, b_ in zip(gb[:3], gt[:3]):
+        assert np.abs(a - b_).max() < 1e-10
+    summed = np.zeros_like(gb[3])
+    for i in range(N):
+        summed[:, :, i // BLOCK] += gt[3][:, :, i]
+    assert np.abs(summed - gb[3]).max() < 1e-10
+
+
+def test_tokens_forward_against_dense_masked_matrix():
+    """Brute force: the whole N x N logit matrix per head with the bias and
+    mask each row's selection implies, a softmax per row."""
+    N, d, Hq, Hkv, topk = 260, 8, 4, 2, 2
+    q, k, v, _ = _tok_case(N, d, Hq, Hkv, topk, 910)
+    idx, cnt, logg, _ = O.select_prefill_tokens(q, O.block_summary(k), Hkv, topk)
+    o, lse = O.attn_fwd_tokens(q, k, v, idx, cnt, logg)
+    G = Hq // Hkv
+    scale = 1.0 / np.sqrt(d)
+    blk = np.arange(N) // BLOCK
+    for h in range(Hq):
+        r = h // G
+        bias = np.full((N, N), -np.inf)
+        for i in range(N):
+            for slot in range(int(cnt[0, r, i])):
+                bias[i, blk == idx[0, r, i, slot]] = logg[0, r, i, slot]
+            cur = (blk == i // BLOCK) & (np.arange(N) <= i)
+            bias[i, cur] = 0.0
+        z = scale * (q[0, h] @ k[0, r].T) + bias
+        zmax = z.max(axis=1, keepdims=True)
+        p = np.exp(z - zmax)
+        assert np.abs(p / p.sum(axis=1, keepdims=True) @ v[0, r] - o[0, h]).max() < 1e-12
+        assert np.abs(zmax[:, 0] + np.log(p.sum(axis=1)) - lse[0, h]).max() < 1e-12
+
+
+def test_tokens_backward_central_finite_differences():
+    """dq, dk, dv and d(log g) of L = sum(dO * o) against central differences
+    (the selection held fixed; log g perturbed as an input)."""
+    N, d, Hq, Hkv, topk = 140, 4, 2, 1, 1
+    q, k, v, do = _tok_case(N, d, Hq, Hkv, topk, 920)
+    idx, cnt, logg, _ = O.select_prefill_tokens(q, O.block_summary(k), Hkv, topk)
+    dq, dk, dv, dlogg = O.attn_bwd_tokens(q, k, v, do, idx, cnt, logg)
+
+    def loss(q_, k_, v_, lg_):
+        return float((O.attn_fwd_tokens(q_, k_, v_, idx, cnt, lg_)[0] * do).sum())
+
+    eps = 1e-6
+    rng = np.random.Generator(np.random.PCG64(921))
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv), ("logg", logg, dlogg)):
+        flat = np.flatnonzero(cnt[..., None].repeat(topk, -1) > 0) if name == "logg" else None
+        for _ in range(4):
+            if name == "logg":
+                e = np.unravel_index(int(rng.choice(flat)), arr.shape)
+            else:
+                e = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            hi, lo = arr.copy(), arr.copy()
+            hi[e] += eps
+            lo[e] -= eps
+            args = {"q": (q, k, v, logg), "k": (q, k, v, logg), "v": (q, k, v, logg),
+                    "logg": (q, k, v, logg)}[name]
+            pos = list(args)
+            slot = ["q", "k", "v", "logg"].index(name)
+            pos[slot] = hi
+            up = loss(*pos)
+            pos[slot] = lo
+            dn = loss(*pos)
+            num = (up - dn) / (2 * eps)
+            assert abs(num - grad[e]) < 1e-6 * max(1.0, abs(num)), (name, e, num, grad[e])

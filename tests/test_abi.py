@@ -105,6 +105,17 @@ def test_rejects_bad_summary_dtype(lib):
                            FAKE, None, None)
     assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
 
+def test_summary_upkeep_argument_checks(lib):
+    st = lib.sas_block_summary_last(FAKE, 1, 1, 8, 1000, 128, FAKE, FAKE, 0, None, 0, None)
+    assert st == 1 and b"multiple of 64" in lib.sas_last_error_message()
+    st = lib.sas_block_summary_last(FAKE, 1, 1, 8, 1024, 128, FAKE, FAKE, 0, FAKE, 0, None)
+    assert st == 1 and b"npages" in lib.sas_last_error_message()
+    st = lib.sas_block_summary_last(FAKE, 1, 1, 8, 1024, 128, FAKE, FAKE, 3, None, 0, None)
+    assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
+    st = lib.sas_block_summary_last(FAKE, 1, 1, 8, 1024, 96, FAKE, FAKE, 0, None, 0, None)
+    assert st == 2  # head dim 96 is not supported
+    assert lib.sas_block_summary_last(None, 1, 0, 8, 1024, 128, None, None, 0, None, 0, None) == 0
+
 def test_empty_inputs_are_noops(lib):
     # B = 0 or N = 0: nothing to do, no pointer needed, no launch
     assert lib.sas_attn_fwd(None, None, None, 1, 0, 4, 4, 128, 64, None, None, None, 2, 0.0, None,

@@ -597,3 +597,41 @@ def attn_bwd_tokens(q, k, v, do, idx, cnt, logg, scale: float | None = None, o_s
                 for slot in range(kk):
                     dlogg[b, r, i, slot] += dz[slot * BLOCK:(slot + 1) * BLOCK].sum()
     return dq, dk, dv, dlogg
+
+
+def select_backward_tokens(q, k, idx, cnt, dlogg, Hkv: int, scale: float | None = None):
+    """Eq. 8 (sparse scope) for per-token selection: for each (b, r, token i)
+    with C = i // 64, kept set I_i and g = softmax(s_i) over m < C,
+        ds_m = dlogg[slot of m] [m in I_i] - g_m sum_{l in I_i} dlogg[slot of l];
+    with s_m = scale qbar_i . kbar_m (qbar_i the mean of the group's G heads
+    at token i), every head of the group gets scale sum_m ds_m kbar_m / G at
+    token i, and block m's 64 keys get scale ds_m qbar_i / 64 each.
+    Returns (dq_sel [B][Hq][N][d], dk_sel [B][Hkv][N][d]) in float64."""
+    q, k, dlogg = _f64(q), _f64(k), _f64(dlogg)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    scale = _scale(d, scale)
+    ksum = block_summary(k)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    for b in range(B):
+        for r in range(Hkv):
+            dkbar = np.zeros((ksum.shape[2], d))
+            for i in range(N):
+                C = i // BLOCK
+                if C == 0:
+                    continue
+                qbar = q[b, r * G:(r + 1) * G, i].mean(axis=0)
+                s = scale * (ksum[b, r, :C] @ qbar)
+                g = np.exp(s - s.max())
+                g = g / g.sum()
+                kk = int(cnt[b, r, i])
+                ds = -g * dlogg[b, r, i, :kk].sum()
+                for j in range(kk):
+                    ds[int(idx[b, r, i, j])] += dlogg[b, r, i, j]
+                dq[b, r * G:(r + 1) * G, i] += scale * (ds @ ksum[b, r, :C]) / G
+                dkbar[:C] += scale * np.outer(ds, qbar)
+            for m in range(dkbar.shape[0]):
+                dk[b, r, m * BLOCK:(m + 1) * BLOCK] += dkbar[m] / BLOCK
+    return dq, dk

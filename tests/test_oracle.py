@@ -614,3 +614,48 @@ def test_tokens_backward_central_finite_differences():
             dn = loss(*pos)
             num = (up - dn) / (2 * eps)
             assert abs(num - grad[e]) < 1e-6 * max(1.0, abs(num)), (name, e, num, grad[e])
+
+
+def _tokens_gated_loss(q, k, v, do, idx, cnt, Hkv):
+    """L(q, k) = sum(dO * o) with the per-token selection held fixed and each
+    token's gate recomputed from q and k (summaries, scores, log g)."""
+    ks = O.block_summary(k)
+    B, Hq, N, d = q.shape
+    G = Hq // Hkv
+    logg = np.zeros(idx.shape)
+    for b in range(B):
+        for r in range(Hkv):
+            for i in range(BLOCK, N):
+                s = (ks[b, r, :i // BLOCK] @ q[b, r * G:(r + 1) * G, i].mean(axis=0)) / np.sqrt(d)
+                _, _, logg_all = O.gate_and_topk(s, 1)
+                for j in range(int(cnt[b, r, i])):
+                    logg[b, r, i, j] = logg_all[idx[b, r, i, j]]
+    o, _ = O.attn_fwd_tokens(q, k, v, idx, cnt, logg)
+    return (o * do).sum(), logg
+
+
+def test_tokens_selector_backward_central_finite_differences():
+    """Per-token attention backward + per-token selector backward = the
+    numerical gradient of the loss with the selection fixed."""
+    N, d, Hq, Hkv, topk = 200, 8, 4, 2, 2
+    q, k, v, do = _tok_case(N, d, Hq, Hkv, topk, 930)
+    idx, cnt, logg, _ = O.select_prefill_tokens(q, O.block_summary(k), Hkv, topk)
+    _, logg0 = _tokens_gated_loss(q, k, v, do, idx, cnt, Hkv)
+    assert np.abs(logg0 - logg).max() < 1e-12
+    dq_a, dk_a, _, dlogg = O.attn_bwd_tokens(q, k, v, do, idx, cnt, logg)
+    dq_s, dk_s = O.select_backward_tokens(q, k, idx, cnt, dlogg, Hkv)
+    grads = {"q": dq_a + dq_s, "k": dk_a + dk_s}
+    h = 1e-5
+    misses = 0
+    for name, ix in (("q", (0, 1, 150, 3)), ("q", (0, 3, 70, 0)), ("q", (0, 2, 199, 5)),
+                     ("k", (0, 0, 10, 5)), ("k", (0, 1, 100, 2)), ("k", (0, 1, 70, 7))):
+        args = dict(q=q, k=k)
+        xp, xm = args[name].copy(), args[name].copy()
+        xp[ix] += h
+        xm[ix] -= h
+        lp, _ = _tokens_gated_loss(**{**args, name: xp}, v=v, do=do, idx=idx, cnt=cnt, Hkv=Hkv)
+        lm, _ = _tokens_gated_loss(**{**args, name: xm}, v=v, do=do, idx=idx, cnt=cnt, Hkv=Hkv)
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - grads[name][ix]) <= 1e-7 * max(1.0, abs(fd)), (name, ix, fd, grads[name][ix])
+        misses += abs(fd - (dq_a if name == "q" else dk_a)[ix]) > 1e-6 * max(1.0, abs(fd))
+    assert misses >= 3  # the selector's share is visible

@@ -185,6 +185,25 @@ def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: 
 
 
 # ----------------------------------------------------------------- decode
+def decode_bytes(c: dict, lens, summary: str = "f32") -> tuple[int, int, int]:
+    """Algorithmic bytes of one decode step: (selection, attention, whole step).
+
+    Selection reads each row's C summaries (C = (n-1)//64; 4 bytes per
+    element, 2 with bf16 summaries) and q; attention reads the kk = min(k, C)
+    kept blocks' and the current block's n-64C tokens of K and V, q, and
+    writes o; the fused step reads q once.
+    """
+    C = [(int(n) - 1) // 64 for n in lens]
+    kk = [min(c["topk"], x) for x in C]
+    ncur = [int(n) - 64 * x for n, x in zip(lens, C)]
+    d, Hkv, es = c["d"], c["Hkv"], 2 if c["dtype"] == "bf16" else 4
+    ses = 2 if summary == "bf16" else 4
+    qb = c["B"] * c["Hq"] * d * es
+    sel = sum(Hkv * x * d * ses for x in C) + qb
+    att = sum(Hkv * (k * 64 + nc) * d * es * 2 for k, nc in zip(kk, ncur)) + 2 * qb
+    return sel, att, sel + att - qb
+
+
 class DecodeWorkload:
     def __init__(self, name: str, summary: str = "f32"):
         from gated_block_sparse_b200 import inputs
@@ -193,18 +212,9 @@ class DecodeWorkload:
         self.c = inputs.CONFIGS[name]
         self.host = inputs.gen_config(name)
         c = self.c
-        lens = self.host["lens"].numpy()
         self.rows = c["B"] * c["Hkv"]
-        self.C = [(int(n) - 1) // 64 for n in lens]
-        kk = [min(c["topk"], C) for C in self.C]
-        ncur = [int(n) - 64 * C for n, C in zip(lens, self.C)]
-        d, Hkv, es = c["d"], c["Hkv"], 2 if c["dtype"] == "bf16" else 4
-        ses = 2 if summary == "bf16" else 4  # bytes per stored summary element
-        # algorithmic bytes per step, by kernel
-        self.sel_bytes = sum(Hkv * C * d * ses for C in self.C) + c["B"] * c["Hq"] * d * es
-        self.att_bytes = (sum(Hkv * (k * 64 + nc) * d * es * 2 for k, nc in zip(kk, ncur))
-                          + 2 * c["B"] * c["Hq"] * d * es)
-        self.step_bytes = self.sel_bytes + self.att_bytes - c["B"] * c["Hq"] * d * es  # q once
+        self.sel_bytes, self.att_bytes, self.step_bytes = decode_bytes(
+            c, self.host["lens"].numpy(), summary)
 
     def describe(self):
         from gated_block_sparse_b200 import inputs

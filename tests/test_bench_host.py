@@ -53,3 +53,23 @@ def test_clock_summary_without_samples():
     c = _sampler(b, [])
     got = c.summary(0.0, 1.0)
     assert got["sm_mhz"] is None and got["reasons"] == ["no nvidia-smi samples"]
+
+
+def test_decode_byte_accounting_matches_the_stated_figures():
+    """c2: 4,194,304 B of kept K/V (15 blocks + a full current block, 8 kv
+    heads), 4,190,208 B of fp32 summaries (1023 blocks), q and o 8 KB each;
+    c5: 16,777,216 B of K/V and 33,550,336 B of summaries (half with bf16)."""
+    from gated_block_sparse_b200 import inputs
+    b = _bench()
+    c2 = inputs.CONFIGS["c2"]
+    sel, att, step = b.decode_bytes(c2, [65536])
+    assert sel == 4190208 + 8192 and att == 4194304 + 2 * 8192 and step == 8400896
+    c5 = inputs.CONFIGS["c5"]
+    sel, att, step = b.decode_bytes(c5, [524288])
+    assert sel - 8192 == 33550336 and att - 16384 == 16777216
+    sel16, _, step16 = b.decode_bytes(c5, [524288], "bf16")
+    assert sel16 - 8192 == 33550336 // 2 and step - step16 == 33550336 // 2
+    # a ragged row: C = 1, kk = 1, current block of 1 token
+    c = dict(c2, B=1)
+    sel, att, step = b.decode_bytes(c, [65])
+    assert att == 8 * (64 + 1) * 128 * 2 * 2 + 2 * 8192 and sel == 8 * 1 * 128 * 4 + 8192

@@ -215,12 +215,16 @@ sas_status sas_decode_attend(const void* q, const void* kc, const void* vc, sas_
                              sas_stream_t stream);
 
 /*
- * Summaries in bf16 (cheaper long-context selection: the summary scan is the
- * length-dependent part of a decode step, and bf16 halves its bytes).
+ * Summaries in bf16, for cheaper long-context selection (SAS close reading,
+ * liuzhao09.github.io, section 2.4: the selector still scans every history
+ * block summary, so at very long contexts ranking, not attention I/O, sets
+ * the decode cost; bf16 halves the bytes of that scan).
  * sas_block_summary_ex writes the summaries in sum_dt: SAS_F32 as
  * sas_block_summary, or SAS_BF16, the fp32 mean rounded to nearest even.
  * sas_decode_ex is sas_decode reading summaries of type sum_dt; the scores
- * are computed from the stored (rounded) summaries.
+ * are computed from the stored (rounded) summaries. Same arguments, layouts
+ * and errors as sas_block_summary / sas_decode otherwise; sum_dt outside
+ * {SAS_F32, SAS_BF16} is SAS_ERR_INVALID_ARG.
  */
 sas_status sas_block_summary_ex(const void* k, sas_dtype dt, int B, int H, int N, int d,
                                 const int32_t* lens, void* ksum, sas_dtype sum_dt,

@@ -24,14 +24,15 @@
  *     soon as it is enqueued.
  *   - Layouts are dense row-major ("HND"): q, o, dO, dq [B][Hq][N][d];
  *     k, v, dk, dv [B][Hkv][N][d]; decode q/o [B][Hq][d]; caches
- *     [B][Hkv][Lmax][d]; block summaries [B][Hkv][N/64][d] fp32.
+ *     [B][Hkv][Lmax][d]; block summaries [B][Hkv][N/64][d] fp32 (bf16 too
+ *     through the *_ex and sas_block_summary_last calls).
  *     Selection rows: prefill idx/logg/dlogg [B][Hkv][T][topk] and cnt
  *     [B][Hkv][T] with T = ceil(N/64); decode idx [B][Hkv][topk].
  *     idx lists the kept history blocks in ascending order, padded with -1;
  *     cnt = min(topk, C).
  *   - Element type of q/k/v/o/dO/dq/dk/dv/caches: SAS_BF16 or SAS_F32, the
- *     same for all of them in one call. Scores, gates, lse and summaries are
- *     fp32; accumulation is fp32.
+ *     same for all of them in one call. Scores, gates and lse are fp32,
+ *     summaries fp32 unless a call says otherwise; accumulation is fp32.
  *   - Supported: d in {64, 128}; block size 64 (fixed); Hq % Hkv == 0;
  *     Hq/Hkv <= 8; 1 <= topk <= 128 (topk = 0 is accepted where stated);
  *     every pointer 16-byte aligned. Other shapes return SAS_ERR_UNSUPPORTED.

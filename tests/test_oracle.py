@@ -181,6 +181,58 @@ def test_prefill_selection_against_enumeration():
                 assert np.allclose(logg[0, r, t, :cnt[0, r, t]], np.log(g[want]), atol=1e-13)
 
 
+def test_prefill_query_pooling_closed_form():
+    """The selector's query mean, pinned by construction rather than by
+    re-slicing: q is zero except one token of one head, and every key of
+    block m equals (m + 1) e_{m mod d}. Then qbar of row (r, t) is that
+    token's vector / (G n_t) for the group holding the head and the block
+    holding the token (n_t = the block's token count, 58 for the ragged last
+    block here), and zero elsewhere, so every score has a closed form: a slip
+    in the head range, the token range or the divisor changes some score."""
+    B, Hq, Hkv, N, d = 1, 6, 3, 250, 4  # G = 2; T = 4 blocks, the last one 58 tokens
+    G, T = Hq // Hkv, 4
+    k = np.zeros((B, Hkv, N, d))
+    for m in range(T):
+        k[0, :, m * 64:min(N, (m + 1) * 64), m % d] = m + 1.0
+    ks = O.block_summary(k)
+    for h, i0, j, c in ((3, 200, 1, 5.0), (4, 249, 2, -3.0), (0, 64, 0, 2.0), (5, 130, 3, 7.0)):
+        q = np.zeros((B, Hq, N, d))
+        q[0, h, i0, j] = c
+        _, _, _, scores = O.select_prefill(q, ks, Hkv, 2)
+        t0, r0 = i0 // 64, h // G
+        n_t0 = min(64, N - 64 * t0)
+        for (b, r, t), srow in scores.items():
+            assert len(srow) == t
+            for m in range(t):
+                want = 0.0
+                if r == r0 and t == t0 and m % d == j:
+                    want = (c / (G * n_t0)) * (m + 1.0) / np.sqrt(d)
+                assert abs(srow[m] - want) < 1e-15, (h, i0, r, t, m, srow[m], want)
+
+
+def test_decode_query_pooling_closed_form():
+    """Decode: q nonzero in one head only; qbar = that head's vector / G for
+    its group and zero for the others (closed-form scores as above)."""
+    B, Hq, Hkv, L, d = 2, 8, 2, 512, 4  # G = 4
+    G = Hq // Hkv
+    kc = np.zeros((B, Hkv, L, d))
+    for m in range(L // 64):
+        kc[:, :, m * 64:(m + 1) * 64, m % d] = m + 1.0
+    ks = O.block_summary(kc)
+    lens = [512, 300]
+    for b0, h, j, c in ((0, 5, 2, 4.0), (1, 2, 3, -1.5)):
+        q = np.zeros((B, Hq, d))
+        q[b0, h, j] = c
+        _, _, _, scores = O.select_decode(q, ks, lens, Hkv, 3)
+        for (b, r), srow in scores.items():
+            C = (lens[b] - 1) // 64
+            assert len(srow) == C
+            for m in range(C):
+                want = (c / G) * (m + 1.0) / np.sqrt(d) if (b == b0 and r == h // G
+                                                             and m % d == j) else 0.0
+                assert abs(srow[m] - want) < 1e-15
+
+
 def _dense_torch_loss(q, k, v, do, idx, cnt, logg_t, scale):
     """Independent dense formulation in torch ops (mask + bias from a block
     map), differentiated by autograd; logg_t is a leaf [B][Hkv][T][k]."""

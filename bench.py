@@ -1,29 +1,39 @@
 #!/usr/bin/env python
 """Benchmark of the SAS gated block-sparse attention hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c4|c5|c3|c1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config all|c1|c2|c3|c4|c5]
                     [--impl ours|reference]
 
-Prints ONE JSON line (rank 0). A step is one pass of the hot path over one
-batch of the named synthetic workload:
-  decode configs (c2 default, c4, c5): block selection over the summaries
-    (scores, gate, Top-K) and split-K attention over the kept blocks plus the
-    current block, for every sequence and kv group; the summaries are built
-    when blocks complete, outside the step. Metric: GB/s of algorithmic bytes
-    (summaries scanned + kept K/V read + q/o).
-  prefill configs (c3, c1): summaries, selection, gated sparse forward and
-    backward. Metric: TFLOP/s of algorithmic FLOPs (kept block pairs, causal
-    pairs exact on the diagonal block, forward 4d and backward 10d per pair).
+Prints ONE JSON line (rank 0). The default (--config all) measures every
+workload the metric is quoted on, each with the same K timed steps:
+  c5  long-context decode (512K, batch 1, top-k 63): the headline record;
+  c4  batched decode (batch 8, ragged 96K-128K, top-k 31);
+  c2  decode (64K, batch 1, top-k 15), also through a paged cache;
+  c5 with bf16 block summaries (the cheaper long-context selection);
+  c3  prefill training step (N = 16384, GQA 32/8, top-k 31): summaries,
+      selection, gated sparse forward and backward, selector backward.
+The line's top level is the c5 record; "records" holds one full record per
+workload (roofline, cpu_baseline, e2e, clocks, launches).
 
-Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs and
-bracketed by CUDA events on the launching stream (barrier + synchronize on
-both sides, max over ranks). Decode steps rotate over L copies of the layer's
-cache and summaries so that the bytes touched between reuses exceed 3x L2.
+A decode step is block selection over the summaries (scores, gate, Top-K)
+and split-K attention over the kept blocks plus the current block, for every
+sequence and kv group; the summaries are cache state, built when blocks
+complete, outside the step. Metric: GB/s of algorithmic bytes (summaries
+scanned + kept K/V read + q/o). A prefill step's metric is TFLOP/s of
+algorithmic FLOPs (kept block pairs, causal pairs exact on the diagonal
+block, forward 4d and backward 10d per pair).
+
+Timing: W warm-up steps and one untimed replay of the timed graphs, then
+exactly K steps replayed from CUDA graphs and bracketed by CUDA events on the
+launching stream (barrier + synchronize on both sides, max over ranks).
+Decode steps rotate over L copies of the layer's cache and summaries so that
+the bytes touched between reuses exceed 3x L2; prefill inputs exceed L2.
 With N > 1 every rank runs its own replica (independent sequences, no
 data-path collective): weak scaling.
 
---impl reference times the fp64 CPU oracle on the host cores, on bounded
-samples of the same workload.
+cpu_baseline: the fp64 oracle on the host, on bounded samples of the same
+workload, once on one core and once on all cores (a spawn process pool over
+independent rows or query blocks). --impl reference times that oracle alone.
 """
 from __future__ import annotations
 
@@ -33,6 +43,7 @@ import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -45,6 +56,10 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn decode GB/s vs HBM peak; prefill fwd+bwd TFLOP/s vs bf16 peak"
 DEFAULT_STEPS = {"c1": 200, "c2": 100000, "c3": 200, "c4": 4000, "c5": 20000}
 DEFAULT_WARMUP = {"c1": 10, "c2": 1000, "c3": 3, "c4": 100, "c5": 500}
+# (record name, config, options) of the default run; the first is the headline
+ALL_RECORDS = (("c5", "c5", {}), ("c5_bf16_summaries", "c5", {"summary": "bf16"}),
+               ("c4", "c4", {}), ("c2", "c2", {}), ("c2_paged", "c2", {"paged": True}),
+               ("c3", "c3", {}))
 
 
 # ----------------------------------------------------------------- helpers
@@ -65,16 +80,31 @@ def source_sha(name: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, source: str):
+def recorded_traffic(kernel: str, source: str, workload: str | None = None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel; else None."""
+    on the current source of the kernel (and on this workload when the
+    record names one); else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    rec = json.load(open(p)).get(kernel)
+    recs = json.load(open(p))
+    rec = recs.get(f"{kernel}@{workload}") if workload else None
+    rec = rec or recs.get(kernel)
     if not rec or rec.get("source_sha") != source_sha(source):
         return None
+    if workload and rec.get("workload", workload) != workload:
+        return None
     return rec.get("dram_bytes_per_launch")
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 class ClockSampler:
@@ -124,11 +154,6 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(win)}
 
 
-def dist_setup(n_gpus: int):
-    from gated_block_sparse_b200 import dist as D
-    return D.setup()
-
-
 def barrier(world):
     from gated_block_sparse_b200 import dist as D
     D.barrier(world)
@@ -142,8 +167,10 @@ def max_over_ranks(world, x: float) -> float:
 def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: int = 512,
                  clocks: ClockSampler | None = None):
     """Capture fn_step(i) for i in [0, chunk) into a graph (plus a tail graph)
-    and time exactly n_steps steps after `warmup` untimed ones. Returns
-    (ms total, max over ranks; clock summary)."""
+    and time exactly n_steps steps after `warmup` untimed ones and one
+    untimed replay of every graph the timed schedule uses (so the timed
+    region holds no first launch of a graph). Returns (ms total, max over
+    ranks; clock summary)."""
     import torch
     chunk = max(1, min(chunk, n_steps))
     graphs = {}
@@ -166,9 +193,9 @@ def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: 
 
     with torch.cuda.stream(stream):
         run(max(3, warmup))
-        graph_of(chunk)
+        graph_of(chunk).replay()
         if n_steps % chunk:
-            graph_of(n_steps % chunk)
+            graph_of(n_steps % chunk).replay()
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
@@ -182,6 +209,22 @@ def timed_graphs(fn_step, n_steps: int, warmup: int, world: int, stream, chunk: 
         barrier(world)
     ms = max_over_ranks(world, start.elapsed_time(end))
     return ms, (clocks.summary(t0, t1) if clocks else None)
+
+
+def event_ms(fn, n: int, stream) -> float:
+    """Device time of n eager calls of fn on `stream` (ms, after 3 warm-ups)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+    return a.elapsed_time(b)
 
 
 # ----------------------------------------------------------------- decode
@@ -205,12 +248,12 @@ def decode_bytes(c: dict, lens, summary: str = "f32") -> tuple[int, int, int]:
 
 
 class DecodeWorkload:
-    def __init__(self, name: str, summary: str = "f32"):
+    def __init__(self, name: str, summary: str = "f32", host=None):
         from gated_block_sparse_b200 import inputs
         self.name = name
         self.summary = summary
         self.c = inputs.CONFIGS[name]
-        self.host = inputs.gen_config(name)
+        self.host = inputs.gen_config(name) if host is None else host
         c = self.c
         self.rows = c["B"] * c["Hkv"]
         self.sel_bytes, self.att_bytes, self.step_bytes = decode_bytes(
@@ -224,10 +267,11 @@ class DecodeWorkload:
                 "context": c["Lmax"] if c["lens"][0] == c["lens"][1] else list(c["lens"]),
                 "topk": c["topk"], "gated": c["gated"], "block": 64,
                 "summaries": "bf16" if self.summary == "bf16" else "fp32",
-                "bytes_per_step": self.step_bytes}
+                "bytes_per_step": self.step_bytes, "selected_kv_bytes_per_step": self.att_bytes}
 
 
-def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
+def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
+                      paged: bool = False, layers: int = 0) -> dict:
     import torch
 
     from gated_block_sparse_b200 import sas
@@ -238,8 +282,8 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     lens = h["lens"].to(dev)
     kc0, vc0 = h["kc"].to(dev), h["vc"].to(dev)
     bf16_sum = w.summary == "bf16"
-    if bf16_sum and args.paged:
-        raise SystemExit("--summary bf16 reads contiguous caches only")
+    if bf16_sum and paged:
+        raise SystemExit("bf16 summaries read contiguous caches only")
     ks0 = (sas.sas_block_summary_ex(kc0, torch.bfloat16) if bf16_sum
            else sas.sas_block_summary(kc0))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -247,8 +291,8 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     free = torch.cuda.mem_get_info(dev)[0]
     L = max(2, math.ceil(3 * l2 / w.step_bytes))
     L = min(L, max(2, int(0.6 * free // per_layer)))
-    if args.layers:
-        L = args.layers
+    if layers:
+        L = layers
     kcs, vcs, kss = [kc0], [vc0], [ks0]
     for _ in range(L - 1):
         kcs.append(kc0.clone())
@@ -256,7 +300,7 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
         kss.append(ks0.clone())
     topk, Hkv = c["topk"], c["Hkv"]
     bt = None
-    if args.paged:  # the same caches scattered into 64-token pages, random page order
+    if paged:  # the same caches scattered into 64-token pages, random page order
         B_, _, Lmax_, d_ = kc0.shape
         nblk = Lmax_ // 64
         perm = torch.randperm(B_ * nblk, generator=torch.Generator().manual_seed(12345)).to(dev)
@@ -271,11 +315,8 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
             kcs[j], vcs[j] = pages(kcs[j]), pages(vcs[j])
             kss[j] = sas.sas_block_summary(kcs[j]).view(B_ * nblk, Hkv, d_)
     o = torch.empty_like(q)
-    ws = torch.empty(sas.sas_decode_workspace_size(c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk),
-                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    K, W = args.steps, args.warmup
 
     def decode(j, qq, out):
         if bt is not None:
@@ -284,8 +325,7 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
         elif bf16_sum:
             sas.sas_decode_ex(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out)
         else:
-            sas.sas_decode(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out,
-                           ws=ws)
+            sas.sas_decode(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out)
 
     def step(i):
         decode(i % L, q, o)
@@ -301,16 +341,23 @@ def bench_decode_ours(args, world, rank, local, w: DecodeWorkload) -> dict:
     # the step is one launch of the cluster kernel: its duration is the step's
     kt = ms / K * 1e-3
     ach = w.step_bytes / kt / 1e9
+    ach_sel = w.att_bytes / kt / 1e9
+    variant = "paged" if bt is not None else ("bf16_summaries" if bf16_sum else None)
     roof = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(ach, 1),
             "peak": peaks["hbm"], "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
-            "traffic": recorded_traffic("k_decode_fused", "k_decode_fused.cu"),
+            "traffic": (None if variant else
+                        recorded_traffic("k_decode_fused", "k_decode_fused.cu", w.name)),
             "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
             "algorithmic_bytes_per_launch": w.step_bytes, "launch_us": round(kt * 1e6, 3),
-            "selected_kv_bytes_per_launch": w.att_bytes, "split_path": split}
-    if bt is not None or bf16_sum:
-        roof["traffic"] = None  # the ncu record is of contiguous caches with fp32 summaries
-    return finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode,
-                         ms, clk, roof, l2, bt is not None or bf16_sum, bt is not None)
+            "selected_kv_bytes_per_launch": w.att_bytes,
+            "achieved_selected_kv": round(ach_sel, 1),
+            "frac_selected_kv": round(ach_sel / peaks["hbm"], 4),
+            "split_path": split}
+    rec = finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode,
+                        ms, clk, roof, l2, variant)
+    del kcs, vcs, kss, kc0, vc0, ks0
+    torch.cuda.empty_cache()
+    return rec
 
 
 def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o):
@@ -323,7 +370,6 @@ def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
     att_ws = torch.empty(max(16, sas.load_library().sas_decode_attend_workspace_size(
         c["B"], c["Hq"], Hkv, c["Lmax"], c["d"], topk)), dtype=torch.uint8, device=dev)
     sel_out = [(torch.empty_like(a), torch.empty_like(b), torch.empty_like(cc)) for a, b, cc in sel]
-    Kk = min(K, 20000)
 
     def sel_step(i):
         j = i % L
@@ -333,9 +379,9 @@ def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
         j = i % L
         sas.sas_decode_attend(q, kcs[j], vcs[j], lens, *sel[j], gated=c["gated"], out=o, ws=att_ws)
 
-    ms_sel, _ = timed_graphs(sel_step, Kk, 10, world, stream)
-    ms_att, _ = timed_graphs(att_step, Kk, 10, world, stream)
-    t_sel, t_att = ms_sel / Kk * 1e-3, ms_att / Kk * 1e-3
+    ms_sel, _ = timed_graphs(sel_step, K, 10, world, stream)
+    ms_att, _ = timed_graphs(att_step, K, 10, world, stream)
+    t_sel, t_att = ms_sel / K * 1e-3, ms_att / K * 1e-3
     return {"k_select_decode": {"us": round(t_sel * 1e6, 3),
                                 "GBps": round(w.sel_bytes / t_sel / 1e9, 1)},
             "k_decode_attend": {"us": round(t_att * 1e6, 3),
@@ -343,7 +389,7 @@ def split_path_timing(sas, c, w, q, lens, kcs, vcs, kss, L, K, world, stream, o)
 
 
 def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, decode, ms, clk,
-                  roof, l2, torch_copies, paged) -> dict:
+                  roof, l2, variant) -> dict:
     import torch
 
     from gated_block_sparse_b200 import dist as D
@@ -352,15 +398,15 @@ def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, 
     qh.copy_(q.cpu())
     oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     qd = torch.empty_like(q)
-    E = min(K, 2000)
+    E = max(K, 200)
 
     def e2e_step(i):
         j = i % L
-        if torch_copies:  # host copies through torch around the call
+        if variant:  # host copies through torch around the call
             qd.copy_(qh, non_blocking=True)
             decode(j, qd, o)
             oh.copy_(o, non_blocking=True)
-        else:  # one C call: copy in, decode step, copy out
+        else:  # one C call: copy in, decode step, o written into pinned host memory
             sas.sas_decode_host(qh, qd, kcs[j], vcs[j], lens, kss[j], c["topk"], o, oh,
                                 gated=c["gated"])
 
@@ -370,65 +416,46 @@ def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, 
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
         e0.record(stream)
         for i in range(E):
             e2e_step(i)
+        h1 = time.perf_counter()
         e1.record(stream)
         torch.cuda.synchronize()
     ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
+    # where an end-to-end step's time goes: the host-side call alone (enqueue
+    # time per step, measured above around the loop), the q copy alone and the
+    # kernel alone (the device-timed step)
+    copy_ms = event_ms(lambda: qd.copy_(qh, non_blocking=True), E, stream)
     nb = q.numel() * q.element_size()
-    api = ("sas_decode_paged with torch copies" if paged
-           else "sas_decode_ex with torch copies" if torch_copies
-           else "sas_decode_host (copy in, then the step writing o into pinned host memory)")
+    api = ({"paged": "sas_decode_paged with torch copies",
+            "bf16_summaries": "sas_decode_ex with torch copies"}.get(variant) or
+           "sas_decode_host (copy in, then the step writing o into pinned host memory)")
     value = D.whole_job_rate(w.step_bytes * K, world, ms) / 1e9
+    cfg = {**w.describe(), "parallelism": f"replicas x{world}",
+           "cache": ("paged: 64-token pages in a random page order" if variant == "paged"
+                     else "contiguous [B][Hkv][Lmax][d]"),
+           "l2": f"rotating {L} layer copies of cache + summaries "
+                 f"({w.step_bytes * L / 1e6:.0f} MB touched per rotation, L2 {l2 / 1e6:.0f} MB)"}
     return {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if c["dtype"] == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) with planted relevant blocks)",
-        "config": {**w.describe(), "parallelism": f"replicas x{world}",
-                   "cache": ("paged: 64-token pages in a random page order" if paged
-                             else "contiguous [B][Hkv][Lmax][d]"),
-                   "l2": f"rotating {L} layer copies of cache + summaries "
-                         f"({w.step_bytes * L / 1e6:.0f} MB touched per rotation, L2 {l2 / 1e6:.0f} MB)"},
+        "config": cfg,
         "roofline": roof,
         "e2e": {"value": round(D.whole_job_rate(w.step_bytes * E, world, ms_e2e) / 1e9, 2),
                 "unit": "GB/s", "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb,
-                "path": f"pinned host q -> {api} via the Python binding -> pinned host o"},
+                "path": f"pinned host q -> {api} via the Python binding -> pinned host o",
+                "split_us_per_step": {"end_to_end": round(ms_e2e / E * 1e3, 3),
+                                      "host_call": round((h1 - h0) / E * 1e6, 3),
+                                      "q_copy_in": round(copy_ms / E * 1e3, 3),
+                                      "kernel": round(ms / K * 1e3, 3)},
+                "steps": E},
         "gpu_launches": K,
         "clocks": clk,
     }
-
-
-def one_thread():
-    """Limit numpy's BLAS to one thread (the oracle baseline runs on 1 core)."""
-    from threadpoolctl import threadpool_limits
-    return threadpool_limits(limits=1)
-
-
-def cpu_baseline_decode(name: str, seconds: float, w: "DecodeWorkload | None" = None,
-                        summary: str = "f32") -> dict:
-    """The fp64 oracle on whole decode steps of the workload, for ~`seconds`."""
-    from oracle import sas_oracle as O
-    w = DecodeWorkload(name, summary) if w is None else w
-    c = w.c
-    h = w.host
-    with one_thread():
-        ks = O.block_summary(h["kc"])  # summaries are built outside the step, as on the GPU
-        if w.summary == "bf16":
-            ks = O.round_bf16(ks)
-        lens = h["lens"].numpy()
-        n, t0 = 0, time.perf_counter()
-        while True:
-            O.decode(h["q"], h["kc"], h["vc"], lens, ks, c["Hkv"], c["topk"], gated=c["gated"])
-            n += 1
-            el = time.perf_counter() - t0
-            if el >= seconds:
-                break
-    return {"value": round(w.step_bytes * n / el / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle", "steps": n, "seconds": round(el, 2),
-            "sample": f"{n} whole decode steps of {name} (all {w.rows} rows), fp64 numpy oracle, "
-                      f"1 BLAS thread; summaries precomputed as on the GPU"}
 
 
 # ----------------------------------------------------------------- prefill
@@ -445,15 +472,14 @@ def prefill_flops(idx_cnt, N: int, Hq: int, Hkv: int, d: int):
     return 4 * d * pairs, 10 * d * pairs
 
 
-def bench_prefill_ours(args, world, rank, local) -> dict:
+def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=None) -> dict:
     import torch
 
     from gated_block_sparse_b200 import dist as D
     from gated_block_sparse_b200 import inputs, sas
-    name = args.config
     c = inputs.CONFIGS[name]
     dev = torch.device("cuda", local if world > 1 else 0)
-    h = inputs.gen_config(name)
+    h = inputs.gen_config(name) if host is None else host
     q, k, v, do = (h[n].to(dev) for n in ("q", "k", "v", "do"))
     topk, Hkv = c["topk"], c["Hkv"]
     B, Hq, N, d = q.shape
@@ -482,7 +508,6 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
         # the gradient through the selector (eq. 8), added into dq and dk
         sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
 
-    K, W = args.steps, args.warmup
     ms, clk = timed_graphs(step, K, W, world, stream, chunk=8, clocks=clocks)
     clocks.stop()
 
@@ -495,10 +520,11 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
     def sbw_step(i):
         sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
 
-    ms_f, _ = timed_graphs(fwd_step, max(3, K), 2, world, stream, chunk=8)
-    ms_b, _ = timed_graphs(bwd_step, max(3, K), 2, world, stream, chunk=8)
-    ms_s, _ = timed_graphs(sbw_step, max(3, K), 2, world, stream, chunk=8)
-    tf, tb = ms_f / max(3, K) * 1e-3, ms_b / max(3, K) * 1e-3
+    Kp = max(3, K)
+    ms_f, _ = timed_graphs(fwd_step, Kp, 2, world, stream, chunk=8)
+    ms_b, _ = timed_graphs(bwd_step, Kp, 2, world, stream, chunk=8)
+    ms_s, _ = timed_graphs(sbw_step, Kp, 2, world, stream, chunk=8)
+    tf, tb = ms_f / Kp * 1e-3, ms_b / Kp * 1e-3
     peaks = measured_peaks()
     tensor = c["dtype"] == "bf16" and d == 128 and (Hq // Hkv) % 2 == 0
     if tensor:  # tcgen05 kernels, timed alone: the burst bf16 peak
@@ -516,37 +542,53 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
     ach = kf / kt / 1e12
     roof = {"bound": bound, "kernel": kern, "achieved": round(ach, 2), "peak": round(peak, 1),
             "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-            "traffic": recorded_traffic(kern, srcs[i]), "peak_source": psrc,
+            "traffic": recorded_traffic(kern, srcs[i], name), "peak_source": psrc,
             "algorithmic_flops_per_launch": kf, "launch_ms": round(kt * 1e3, 4),
             "fwd_ms": round(tf * 1e3, 4), "bwd_ms": round(tb * 1e3, 4),
             "fwd_tflops": round(f_fwd / tf / 1e12, 2), "bwd_tflops": round(f_bwd / tb / 1e12, 2),
-            "select_bwd_ms": round(ms_s / max(3, K), 4)}
+            "fwd_frac": round(f_fwd / tf / 1e12 / peak, 4),
+            "bwd_frac": round(f_bwd / tb / 1e12 / peak, 4),
+            "fwd_plus_bwd_frac": round((f_fwd + f_bwd) / (tf + tb) / 1e12 / peak, 4),
+            "select_bwd_ms": round(ms_s / Kp, 4)}
 
     # end to end: pinned host inputs in, gradients out
     pin = {n: torch.empty(h[n].shape, dtype=h[n].dtype, pin_memory=True) for n in ("q", "k", "v", "do")}
     for n in pin:
         pin[n].copy_(h[n])
     outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o,) + tuple(grads)]
-    E = max(2, min(K, 5))
+    E = max(3, min(K, 10))
+
+    def copy_in():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        do.copy_(pin["do"], non_blocking=True)
+
+    def copy_out():
+        for dst, src in zip(outs, (o,) + tuple(grads)):
+            dst.copy_(src, non_blocking=True)
+
     with torch.cuda.stream(stream):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            copy_in()
+            step(0)
+            copy_out()
         torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(E):
-            q.copy_(pin["q"], non_blocking=True)
-            k.copy_(pin["k"], non_blocking=True)
-            v.copy_(pin["v"], non_blocking=True)
-            do.copy_(pin["do"], non_blocking=True)
+            copy_in()
             step(0)
-            for dst, src in zip(outs, (o,) + tuple(grads)):
-                dst.copy_(src, non_blocking=True)
+            copy_out()
         e1.record(stream)
         torch.cuda.synchronize()
     ms_e2e = max_over_ranks(world, e0.elapsed_time(e1))
+    ms_in = event_ms(copy_in, E, stream)
+    ms_out = event_ms(copy_out, E, stream)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in outs)
     total = f_fwd + f_bwd
-    return {
+    rec = {
         "metric": METRIC, "value": round(D.whole_job_rate(total * K, world, ms) / 1e12, 4),
         "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -557,25 +599,132 @@ def bench_prefill_ours(args, world, rank, local) -> dict:
                    "l2": f"inputs larger than L2 (q+k+v+dO = {h2d / 1e6:.0f} MB)"},
         "roofline": roof,
         "e2e": {"value": round(total * E * world / (ms_e2e * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host q, k, v, dO -> the step's five library calls -> pinned host "
+                        "o, dq, dk, dv, dlogg",
+                "split_ms_per_step": {"end_to_end": round(ms_e2e / E, 4),
+                                      "copy_in": round(ms_in / E, 4),
+                                      "copy_out": round(ms_out / E, 4),
+                                      "step": round(ms / K, 4)},
+                "steps": E},
         # summary, query means, selection, forward, backward, 2 conversions,
         # selector backward (query means, rows, columns)
         "gpu_launches": 10 * K,
         "clocks": clk,
     }
+    del q, k, v, do, grads, o, lse
+    torch.cuda.empty_cache()
+    return rec
 
 
-def cpu_baseline_prefill(name: str, seconds: float) -> dict:
-    """The oracle's forward+backward on whole query blocks of the workload."""
-    import numpy as np
+# ----------------------------------------------------------------- oracle baselines
+# The oracle (fp64 numpy, oracle/) timed on the host cores on bounded samples.
+# One-core runs limit BLAS to one thread; all-core runs use a spawn process
+# pool (one BLAS thread each) over independent decode rows or prefill query
+# blocks, sharing the input tensors through shared memory.
+def _one_thread():
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
 
+
+def _decode_rows_worker(args):
+    """Decode rows (b, r) of one workload, round-robin, for `seconds`; each
+    row is one oracle decode step of a single-row problem. Returns (rows
+    done, seconds)."""
+    from oracle import sas_oracle as O
+    rows, seconds, topk, gated, G = args
+    with _one_thread():
+        n, t0 = 0, time.perf_counter()
+        while True:
+            q, kc, vc, lens, ks = rows[n % len(rows)]
+            O.decode(q, kc, vc, lens, ks, 1, topk, gated=gated)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return n, el
+
+
+def _prefill_units_worker(args):
+    """Prefill (kv group, query block) units, forward + backward of the
+    group's heads, for `seconds`. Returns (FLOPs done, units done, seconds)."""
+    from oracle import sas_oracle as O
+    units, seconds, d = args
+    with _one_thread():
+        flops, n, t0 = 0, 0, time.perf_counter()
+        while True:
+            q, k, v, do, idx, cnt, logg, t, G, N = units[n % len(units)]
+            O.query_block(q, k, v, do, idx, cnt, logg, 0, 0, t)
+            nr = min(64, N - 64 * t)
+            flops += 14 * d * (int(cnt[0, 0, t]) * G * nr * 64 + G * nr * (nr + 1) // 2)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return flops, n, el
+
+
+def _pool_map(fn, tasks):
+    import torch.multiprocessing as tmp
+    with tmp.get_context("spawn").Pool(len(tasks)) as pool:
+        return pool.map(fn, tasks)
+
+
+def cpu_baseline_decode(w: DecodeWorkload, seconds: float, all_cores: bool = True) -> dict:
+    """The fp64 oracle on whole decode steps of the workload (one core), and
+    on all cores over its independent rows."""
+    from oracle import sas_oracle as O
+    c = w.c
+    h = w.host
+    with _one_thread():
+        ks = O.block_summary(h["kc"], lens=h["lens"].numpy())  # cache state, as on the GPU
+        if w.summary == "bf16":
+            ks = O.round_bf16(ks)
+        lens = h["lens"].numpy()
+        n, t0 = 0, time.perf_counter()
+        while True:
+            O.decode(h["q"], h["kc"], h["vc"], lens, ks, c["Hkv"], c["topk"], gated=c["gated"])
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    one = w.step_bytes * n / el / 1e9
+    res = {"value": round(one, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "steps": n, "seconds": round(el, 2),
+           "sample": f"{n} whole decode steps of {w.name} (all {w.rows} rows), fp64 numpy "
+                     f"oracle, 1 BLAS thread; summaries precomputed as on the GPU",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    ncpu = os.cpu_count() or 1
+    if all_cores and ncpu > 1:
+        G = c["Hq"] // c["Hkv"]
+        rows = []
+        for b in range(c["B"]):
+            for r in range(c["Hkv"]):
+                rows.append((h["q"][b:b + 1, r * G:(r + 1) * G].clone(),
+                             h["kc"][b:b + 1, r:r + 1].clone(), h["vc"][b:b + 1, r:r + 1].clone(),
+                             lens[b:b + 1].copy(), ks[b:b + 1, r:r + 1].copy()))
+        P = min(ncpu, len(rows))
+        tasks = [(rows[j::P], seconds, c["topk"], c["gated"], G) for j in range(P)]
+        out = _pool_map(_decode_rows_worker, tasks)
+        done = sum(x[0] for x in out)
+        span = max(x[1] for x in out)
+        rate = done / w.rows / span * w.step_bytes / 1e9
+        res["all_cores"] = {"value": round(rate, 4), "unit": "GB/s", "cores": P,
+                            "rows": done, "seconds": round(span, 2),
+                            "sample": f"{P} processes (spawn, 1 BLAS thread each) each running "
+                                      f"its share of the {w.rows} rows for {seconds:g} s; rate = "
+                                      f"rows done / rows per step / slowest process's time"}
+    return res
+
+
+def cpu_baseline_prefill(name: str, seconds: float, host=None, all_cores: bool = True) -> dict:
+    """The oracle's forward+backward on whole query blocks of the workload
+    (one core), and on all cores over (kv group, query block) units."""
     from gated_block_sparse_b200 import inputs
     from oracle import sas_oracle as O
     c = inputs.CONFIGS[name]
-    h = inputs.gen_config(name)
+    h = inputs.gen_config(name) if host is None else host
     N, d = c["N"], c["d"]
     G = c["Hq"] // c["Hkv"]
-    with one_thread():
+    with _one_thread():
         ks = O.block_summary(h["k"])
         idx, cnt, logg, _ = O.select_prefill(h["q"], ks, c["Hkv"], c["topk"])
         T = idx.shape[2]
@@ -591,21 +740,77 @@ def cpu_baseline_prefill(name: str, seconds: float) -> dict:
             if time.perf_counter() - t0 >= seconds:
                 break
         el = time.perf_counter() - t0
-    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "seconds": round(el, 2),
-            "sample": f"{n} of {len(order)} (sequence, kv group, query block) units of {name} "
-                      "(forward + backward, all heads of the group), fp64 numpy oracle, 1 BLAS thread"}
+    res = {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+           "seconds": round(el, 2),
+           "sample": f"{n} of {len(order)} (sequence, kv group, query block) units of {name} "
+                     "(forward + backward, all heads of the group, latest query blocks first), "
+                     "fp64 numpy oracle, 1 BLAS thread",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    ncpu = os.cpu_count() or 1
+    if all_cores and ncpu > 1 and c["B"] == 1:
+        P = ncpu
+        units = []
+        for t in range(T - 1, -1, -1):
+            for r in range(c["Hkv"]):
+                units.append((r, t))
+        groups = {}
+        for r in range(c["Hkv"]):
+            groups[r] = (h["q"][:, r * G:(r + 1) * G].clone(), h["k"][:, r:r + 1].clone(),
+                         h["v"][:, r:r + 1].clone(), h["do"][:, r * G:(r + 1) * G].clone(),
+                         idx[:, r:r + 1].copy(), cnt[:, r:r + 1].copy(), logg[:, r:r + 1].copy())
+        share = [[groups[r] + (t, G, N) for (r, t) in units[j::P][:64]] for j in range(P)]
+        share = [s for s in share if s]
+        out = _pool_map(_prefill_units_worker, [(s, seconds, d) for s in share])
+        fl = sum(x[0] for x in out)
+        span = max(x[2] for x in out)
+        res["all_cores"] = {"value": round(fl / span / 1e12, 6), "unit": "TFLOP/s",
+                            "cores": len(share), "units": sum(x[1] for x in out),
+                            "seconds": round(span, 2),
+                            "sample": f"{len(share)} processes (spawn, 1 BLAS thread each), each "
+                                      f"cycling over up to 64 of the latest (kv group, query "
+                                      f"block) units for {seconds:g} s; rate = FLOPs done / "
+                                      f"slowest process's time"}
+    return res
 
 
 # ----------------------------------------------------------------- main
+def run_one(name: str, cfg: str, opts: dict, K: int, W: int, world: int, rank: int, local: int,
+            cpu_seconds: float, hosts: dict, baselines: dict) -> dict:
+    from gated_block_sparse_b200 import inputs
+    c = inputs.CONFIGS[cfg]
+    if cfg not in hosts:
+        hosts.clear()  # one workload's inputs on the host at a time
+        hosts[cfg] = inputs.gen_config(cfg)
+    if c["kind"] == "decode":
+        w = DecodeWorkload(cfg, opts.get("summary", "f32"), host=hosts[cfg])
+        rec = bench_decode_ours(K, W, world, local, w, paged=opts.get("paged", False),
+                                layers=opts.get("layers", 0))
+        if rank == 0:
+            key = (cfg, w.summary)
+            if key not in baselines:
+                baselines[key] = cpu_baseline_decode(w, cpu_seconds)
+            rec["cpu_baseline"] = baselines[key]
+    else:
+        rec = bench_prefill_ours(cfg, K, W, world, local, host=hosts[cfg])
+        if rank == 0:
+            rec["cpu_baseline"] = cpu_baseline_prefill(cfg, cpu_seconds, host=hosts[cfg])
+    if opts.get("paged"):
+        rec["config"]["variant"] = "paged KV cache (sas_decode_paged)"
+    if opts.get("summary") == "bf16":
+        rec["config"]["variant"] = "bf16 block summaries (sas_decode_ex)"
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--config", default="all", choices=["all", "c1", "c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=None,
+                    help="oracle baseline sample per config and core setting "
+                         "(default 4 s with --config all, 10 s otherwise)")
     ap.add_argument("--paged", action="store_true",
                     help="decode: read the caches through 64-token pages (sas_decode_paged)")
     ap.add_argument("--summary", default="f32", choices=["f32", "bf16"],
@@ -613,40 +818,50 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="decode: number of rotated layer copies (default: enough for 3x L2)")
     args = ap.parse_args()
-    args.steps = args.steps or DEFAULT_STEPS[args.config]
-    args.warmup = max(3, args.warmup if args.warmup is not None else DEFAULT_WARMUP[args.config])
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    decode = args.config in ("c2", "c4", "c5")
+    cpu_s = args.cpu_seconds or (4.0 if args.config == "all" else 10.0)
+
+    if args.config == "all":
+        plan = ALL_RECORDS
+    else:
+        opts = {"paged": args.paged, "summary": args.summary, "layers": args.layers}
+        plan = ((args.config, args.config, opts),)
 
     if args.impl == "reference":
         if rank != 0:
             return
-        base = (cpu_baseline_decode(args.config, args.cpu_seconds, summary=args.summary) if decode
-                else cpu_baseline_prefill(args.config, args.cpu_seconds))
         from gated_block_sparse_b200 import inputs
+        name, cfg, opts = plan[0]
+        if inputs.CONFIGS[cfg]["kind"] == "decode":
+            base = cpu_baseline_decode(DecodeWorkload(cfg, opts.get("summary", "f32")), cpu_s)
+        else:
+            base = cpu_baseline_prefill(cfg, cpu_s)
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
             "n_gpus": args.gpus, "steps": base.get("steps"), "warmup": 0,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded, same generator)",
-            "config": {"workload": f"{args.config}: {inputs.DESCRIPTIONS[args.config]}"},
+            "config": {"workload": f"{cfg}: {inputs.DESCRIPTIONS[cfg]}"},
             "cpu_baseline": base,
             "e2e": {"value": base["value"], "unit": base["unit"], "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}))
         return
 
-    world, rank, local = dist_setup(args.gpus)
-    if decode:
-        w = DecodeWorkload(args.config, args.summary)
-        res = bench_decode_ours(args, world, rank, local, w)
-    else:
-        res = bench_prefill_ours(args, world, rank, local)
-    if rank == 0:
-        res["cpu_baseline"] = (cpu_baseline_decode(args.config, args.cpu_seconds, w) if decode
-                               else cpu_baseline_prefill(args.config, args.cpu_seconds))
-        print(json.dumps(res))
     from gated_block_sparse_b200 import dist as D
+    world, rank, local = D.setup()
+    records, hosts, baselines = {}, {}, {}
+    for name, cfg, opts in plan:
+        K = args.steps or DEFAULT_STEPS[cfg]
+        W = max(3, args.warmup if args.warmup is not None else DEFAULT_WARMUP[cfg])
+        records[name] = run_one(name, cfg, opts, K, W, world, rank, local, cpu_s, hosts, baselines)
+    if rank == 0:
+        head = dict(records[plan[0][0]])
+        if len(plan) > 1:
+            head["records"] = records
+            head["config"] = dict(head["config"], headline=plan[0][0],
+                                  records=[n for n, _, _ in plan])
+        print(json.dumps(head))
     D.teardown(world)
 
 

@@ -140,8 +140,8 @@ size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk,
 
 sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
                       int N, int d, int topk, sas_mode mode, const int32_t* lens, float scale,
-                      int32_t* idx, int32_t* cnt, float* logg, void* ws, size_t ws_bytes,
-                      sas_stream_t stream) {
+                      int32_t* idx, int32_t* cnt, float* logg, float* scores_out, void* ws,
+                      size_t ws_bytes, sas_stream_t stream) {
   g_last_error.clear();
   sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
   if (s != SAS_OK) return s;
@@ -154,6 +154,8 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
     REQUIRE_PTR(logg);
   }
   if (N / 64 > 0) REQUIRE_PTR(ksum);
+  if (scores_out)
+    REQUIRE(aligned16(scores_out), SAS_ERR_INVALID_ARG, "scores_out must be 16-byte aligned");
   const size_t need = sas_select_workspace_size(B, Hq, Hkv, N, d, topk, mode);
   REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
   REQUIRE_PTR(ws);
@@ -163,7 +165,7 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
     REQUIRE(lens == nullptr, SAS_ERR_INVALID_ARG, "lens must be NULL in prefill mode");
     REQUIRE((N + 63) / 64 - 1 <= 256 * 64, SAS_ERR_UNSUPPORTED, "prefill N too long for selection");
     return cuda_status(sas::launch_select_prefill(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
-                                                  sc, idx, cnt, logg, ws, st),
+                                                  sc, idx, cnt, logg, scores_out, ws, st),
                        "sas_select launch");
   }
   REQUIRE_PTR(lens);
@@ -175,7 +177,8 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
   cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)B * Hkv, st);
   if (e != cudaSuccess) return cuda_status(e, "sas_select memset");
   return cuda_status(sas::launch_select_decode(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
-                                               lens, sc, idx, cnt, logg, p, counters, rest, st),
+                                               lens, sc, idx, cnt, logg, scores_out, p, counters,
+                                               rest, st),
                      "sas_select launch");
 }
 
@@ -419,10 +422,12 @@ sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, cons
   // the combining CTAs then write o straight into it, with no separate copy.
   void* o_out = nullptr;
   cudaPointerAttributes at;
-  if (cudaPointerGetAttributes(&at, o_host) == cudaSuccess && at.type == cudaMemoryTypeHost &&
-      at.devicePointer != nullptr && aligned16(at.devicePointer))
+  const cudaError_t pa = cudaPointerGetAttributes(&at, o_host);
+  if (pa != cudaSuccess)
+    cudaGetLastError();  // clears that query's own error: a pageable o_host is not a failure
+  else if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr &&
+           aligned16(at.devicePointer))
     o_out = at.devicePointer;
-  cudaGetLastError();  // a pageable pointer is not an error here
   e = sas::launch_decode_fused(q_dev, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, ksum,
                                topk, gated, resolve_scale(scale, d), o_out ? o_out : o_dev,
                                idx_out, st);

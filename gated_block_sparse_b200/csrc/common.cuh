@@ -444,10 +444,12 @@ __host__ __device__ inline int ceil_log2(int k) {
 
 // ---------------------------------------------------------------- PDL
 // Programmatic dependent launch: a kernel launched with the programmatic
-// stream serialization attribute may start before its predecessor ends.
-// grid_dep_wait() blocks until every CTA of the predecessor has triggered
-// (grid_dep_launch) or exited; only the predecessor's writes made before its
-// trigger are guaranteed visible after it.
+// stream serialization attribute may be scheduled before its predecessor
+// ends, once every CTA of the predecessor has called grid_dep_launch() or
+// exited (without a call, at the predecessor's completion). The trigger only
+// decides that early scheduling. grid_dep_wait() blocks until the predecessor
+// grids have completed and their memory operations are visible, so every
+// write of the predecessor, before or after its trigger, is seen after it.
 __device__ __forceinline__ void grid_dep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

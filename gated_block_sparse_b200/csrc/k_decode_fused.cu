@@ -16,14 +16,16 @@
 //      selection, is copied by the CTA that owns it as soon as the ring is
 //      free, under the selection;
 //   2. reduces its range to (max, sum exp) and a best-first list of
-//      min(k, n) candidates (the keys at or above the k-th key of a strided
-//      sample, ranked among themselves), and stores both into its slot of
-//      every CTA of the cluster with asynchronous remote stores that
-//      complete on the receiver's mbarrier;
+//      min(k, n) candidates (rank counting for short ranges, per-warp
+//      register bitonic sorts and a bitonic merge tree for ranges up to 512,
+//      and beyond that the keys at or above the k-th key of a strided sample,
+//      ranked among themselves), and stores both into its slot of every CTA
+//      of the cluster with asynchronous remote stores that complete on the
+//      receiver's mbarrier;
 //   3. once all lists have landed, every CTA computes the gate's LSE and the
-//      same Top-K: the keys above a pruning threshold are ranked among
-//      themselves, giving the kept blocks in score order (CTA 0 also writes
-//      them in ascending block order to idx_out);
+//      same Top-K with a tree of bitonic merges of the CS sorted lists,
+//      giving the kept blocks in score order (CTA 0 also writes them in
+//      ascending block order to idx_out);
 //   4. streams the K/V blocks of its share of the units (the current block
 //      first, then kept blocks in score order) through a ring that reuses
 //      the summary ring.

@@ -53,9 +53,10 @@ __device__ __forceinline__ float block_reduce_sum(float v, float* red) {
 // s[j] = scale * qbar . ksum_row[m0 + j] for j < n. Warp-per-block with the
 // d dimension split over the lanes (D/32 floats each), four blocks in flight
 // per warp. A -0 score is stored as +0 so that exact ties compare equal.
+// gs (nullable): the row's raw-score output, written at gs[m0 + j] as well.
 template <int D>
 __device__ void score_chunk(const float* __restrict__ ks_row, int m0, int n,
-                            const float* qbar_s, float scale, float* sc) {
+                            const float* qbar_s, float scale, float* sc, float* gs) {
   constexpr int PER = D / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nw = blockDim.x >> 5;
@@ -86,7 +87,11 @@ __device__ void score_chunk(const float* __restrict__ ks_row, int m0, int n,
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int j = base + u * nw;
-        if (j < n) sc[j] = part[u] * scale + 0.0f;
+        if (j < n) {
+          const float sj = part[u] * scale + 0.0f;
+          sc[j] = sj;
+          if (gs != nullptr) gs[m0 + j] = sj;
+        }
       }
     }
   }
@@ -163,7 +168,8 @@ __global__ void __launch_bounds__(256) k_qbar_prefill(const T* __restrict__ q, i
 template <int D>
 __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
     const float* __restrict__ qbar, const float* __restrict__ ksum, int Hkv, int nblk, int topk,
-    float scale, int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg) {
+    float scale, int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg,
+    float* __restrict__ scores) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z, T_ = gridDim.x;
   const int C = t;
@@ -183,10 +189,13 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_prefill(
   for (int i = threadIdx.x; i < D; i += blockDim.x) q_s[i] = qrow[i];
   __syncthreads();
   const float* ks_row = ksum + ((size_t)b * Hkv + r) * nblk * D;
+  float* gs = scores != nullptr ? scores + row * T_ : nullptr;  // [T] of this row
+  if (gs != nullptr)
+    for (int m = C + threadIdx.x; m < T_; m += blockDim.x) gs[m] = -INFINITY;
   float run_m = -FLT_MAX, run_s = 0.f;
   for (int c = 0; c < nchunk; ++c) {
     const int m0 = c * SEL_CHUNK_MAX, n = min(SEL_CHUNK_MAX, C - m0);
-    score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
+    score_chunk<D>(ks_row, m0, n, q_s, scale, sc, gs);
     __syncthreads();
     if (topk > 0) chunk_topk(sc, m0, n, topk, la + ((size_t)c << lg));
     float lm = -FLT_MAX;
@@ -241,7 +250,8 @@ cudaError_t launch_qbar_prefill(const void* q, int bf16, int B, int Hq, int Hkv,
 
 cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
                                   int Hkv, int N, int d, int topk, float scale, int32_t* idx,
-                                  int32_t* cnt, float* logg, void* ws, cudaStream_t st) {
+                                  int32_t* cnt, float* logg, float* scores, void* ws,
+                                  cudaStream_t st) {
   const int T_ = (N + SAS_BLOCK - 1) / SAS_BLOCK;
   if (B == 0 || T_ == 0) return cudaSuccess;
   float* qbar = static_cast<float*>(ws);
@@ -260,11 +270,11 @@ cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, in
   if (d == 128) {
     ensure_smem(k_select_prefill<128>, smem);
     k_select_prefill<128><<<grid, SEL_THREADS, smem, st>>>(qbar, ksum, Hkv, nblk, topk, scale,
-                                                           idx, cnt, logg);
+                                                           idx, cnt, logg, scores);
   } else {
     ensure_smem(k_select_prefill<64>, smem);
     k_select_prefill<64><<<grid, SEL_THREADS, smem, st>>>(qbar, ksum, Hkv, nblk, topk, scale,
-                                                          idx, cnt, logg);
+                                                          idx, cnt, logg, scores);
   }
   return cudaGetLastError();
 }
@@ -310,8 +320,8 @@ cudaError_t launch_select_prefill_static(const void* q, int bf16, const float* k
   float* qbar = nullptr;
   cudaError_t e = static_qbar_address(&qbar);
   if (e != cudaSuccess) return e;
-  return launch_select_prefill(q, bf16, ksum, B, Hq, Hkv, N, d, topk, scale, idx, cnt, logg, qbar,
-                               st);
+  return launch_select_prefill(q, bf16, ksum, B, Hq, Hkv, N, d, topk, scale, idx, cnt, logg,
+                               nullptr, qbar, st);
 }
 
 // ------------------------------------------------------------------ decode
@@ -372,7 +382,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
     const T* __restrict__ q, const float* __restrict__ ksum, int Hq, int Hkv, int nblk,
     const int32_t* __restrict__ lens, int topk, float scale, int chunk, DecodeSelectWs w,
-    int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg) {
+    int32_t* __restrict__ idx, int32_t* __restrict__ cnt, float* __restrict__ logg,
+    float* __restrict__ scores) {
   __shared__ __align__(16) float q_s[D];
   __shared__ float sc[DEC_CHUNK_MAX];
   __shared__ float red[32];
@@ -383,6 +394,10 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   const int nchunk = gridDim.x;
   const int G = Hq / Hkv;
   const int row = b * Hkv + r;
+  // A programmatic dependent (the decode attention) may be scheduled now and
+  // load what does not depend on this grid; it waits for this grid's
+  // completion, with every write visible, before it reads the selection.
+  grid_dep_launch();
   const int n_tok = min(max(lens[b], 1), nblk * SAS_BLOCK);  // 1 <= n <= Lmax
   const int C = (n_tok - 1) / SAS_BLOCK;
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
@@ -393,7 +408,11 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   __syncthreads();
   const int m0 = c * chunk, n = max(0, min(chunk, C - m0));
   const float* ks_row = ksum + (size_t)row * nblk * D;
-  score_chunk<D>(ks_row, m0, n, q_s, scale, sc);
+  float* gs = scores != nullptr ? scores + (size_t)row * nblk : nullptr;  // [nblk] of this row
+  if (gs != nullptr)
+    for (int m = max(C, m0) + threadIdx.x; m < min(m0 + chunk, nblk); m += blockDim.x)
+      gs[m] = -INFINITY;
+  score_chunk<D>(ks_row, m0, n, q_s, scale, sc, gs);
   __syncthreads();
   const size_t rc = (size_t)row * nchunk + c;
   if (topk > 0) chunk_topk(sc, m0, n, topk, w.lk + rc * topk);
@@ -413,10 +432,6 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
   __syncthreads();
   if (threadIdx.x == 0) is_last = (atomicAdd(w.counter + row, 1) == nchunk - 1);
   __syncthreads();
-  // No explicit launch trigger: a programmatic dependent (the decode attention)
-  // is only guaranteed to see writes made before the trigger, and the merge
-  // below writes the selection it consumes. The implicit trigger at grid exit
-  // comes after every write.
   if (!is_last) return;
   __threadfence();
   // Stage the row's partials in shared memory with one parallel pass of L2
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(SEL_THREADS) k_select_decode(
 cudaError_t launch_select_decode(const void* q, int bf16, const float* ksum, int B, int Hq,
                                  int Hkv, int Lmax, int d, int topk, const int32_t* lens,
                                  float scale, int32_t* idx, int32_t* cnt, float* logg,
-                                 const SelectPlan& plan, int* counters, void* ws,
+                                 float* scores, const SelectPlan& plan, int* counters, void* ws,
                                  cudaStream_t st) {
   if (B == 0) return cudaSuccess;
   DecodeSelectWs w = carve_decode_select(counters, ws, plan);
@@ -476,7 +491,8 @@ const size_t smem = decode_merge_smem(plan.nchunk, topk);
     ensure_smem(k_select_decode<T, D>, smem);                                                \
     k_select_decode<T, D><<<grid, SEL_THREADS, smem, st>>>(static_cast<const T*>(q), ksum,   \
                                                            Hq, Hkv, nblk, lens, topk, scale, \
-                                                           plan.chunk, w, idx, cnt, logg);   \
+                                                           plan.chunk, w, idx, cnt, logg,    \
+                                                           scores);                          \
   } while (0)
   if (bf16) {
     if (d == 128) SAS_SELD(__nv_bfloat16, 128); else SAS_SELD(__nv_bfloat16, 64);

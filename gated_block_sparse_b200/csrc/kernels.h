@@ -41,9 +41,11 @@ struct SelectPlan {
 SelectPlan plan_decode_select(int B, int Hkv, int Lmax, int topk);
 size_t decode_select_ws_bytes(const SelectPlan& p);
 
+// scores (nullable): raw selector scores [B][Hkv][T][T], -inf at m >= t.
 cudaError_t launch_select_prefill(const void* q, int bf16, const float* ksum, int B, int Hq,
                                   int Hkv, int N, int d, int topk, float scale, int32_t* idx,
-                                  int32_t* cnt, float* logg, void* ws, cudaStream_t st);
+                                  int32_t* cnt, float* logg, float* scores, void* ws,
+                                  cudaStream_t st);
 size_t select_prefill_ws_bytes(int B, int Hkv, int N, int d);
 // Query means of the prefill selector, qbar [B][Hkv][T][d] fp32.
 cudaError_t launch_qbar_prefill(const void* q, int bf16, int B, int Hq, int Hkv, int N, int d,
@@ -67,10 +69,11 @@ cudaError_t launch_select_prefill_static(const void* q, int bf16, const float* k
 
 // Decode selection. `counters` holds one int per row and must be zero on
 // entry (the kernel leaves it zero); `ws` holds the plan's partials.
+// scores (nullable): raw selector scores [B][Hkv][Lmax/64], -inf at m >= C.
 cudaError_t launch_select_decode(const void* q, int bf16, const float* ksum, int B, int Hq,
                                  int Hkv, int Lmax, int d, int topk, const int32_t* lens,
                                  float scale, int32_t* idx, int32_t* cnt, float* logg,
-                                 const SelectPlan& plan, int* counters, void* ws,
+                                 float* scores, const SelectPlan& plan, int* counters, void* ws,
                                  cudaStream_t st);
 
 // ---- decode attention

@@ -28,7 +28,8 @@ SIGNATURES = {
     "sas_version": (_I, []),
     "sas_block_summary": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sas_select_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
-    "sas_select": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F, _P, _P, _P, _P, _Z, _P]),
+    "sas_select": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F, _P, _P, _P, _P, _P, _Z,
+                        _P]),
     "sas_select_prefill_noalloc_capacity": (_Z, []),
     "sas_select_prefill_noalloc": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "sas_attn_fwd_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
@@ -130,12 +131,14 @@ def sas_block_summary(k: torch.Tensor, lens: torch.Tensor | None = None,
 
 def sas_select(q: torch.Tensor, ksum: torch.Tensor, Hkv: int, topk: int, mode: str = "prefill",
                lens: torch.Tensor | None = None, scale: float = 0.0, out=None, ws=None,
-               stream=None):
+               stream=None, scores_out: torch.Tensor | None = None):
     """Scores, gate and Top-K. Returns (idx int32, cnt int32, logg fp32).
 
     prefill: q [B][Hq][N][d] -> idx/logg [B][Hkv][T][topk], cnt [B][Hkv][T].
     decode:  q [B][Hq][d], N = Lmax = 64 * ksum.shape[2] -> idx/logg
              [B][Hkv][topk], cnt [B][Hkv].
+    scores_out (optional, fp32): receives the raw scores, [B][Hkv][T][T]
+    (prefill) or [B][Hkv][N/64] (decode), -inf past each row's C blocks.
     """
     lib = load_library()
     if mode == "prefill":
@@ -159,8 +162,8 @@ def sas_select(q: torch.Tensor, ksum: torch.Tensor, Hkv: int, topk: int, mode: s
     w = _ws(need, q.device, ws)
     _check("sas_select", lib.sas_select(
         _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, m, _ptr(lens), float(scale),
-        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None, _ptr(w),
-        w.numel(), _stream(stream)))
+        _ptr(idx) if topk else None, _ptr(cnt), _ptr(logg) if topk else None,
+        _ptr(scores_out), _ptr(w), w.numel(), _stream(stream)))
     return idx, cnt, logg
 
 
@@ -235,10 +238,11 @@ def sas_decode(q, kc, vc, lens, ksum, topk: int, gated: int = 1, scale: float = 
     if out is None:
         out = torch.empty_like(q)
     need = lib.sas_decode_workspace_size(B, Hq, Hkv, Lmax, d, topk)
-    w = _ws(need, q.device, ws)
+    w = _ws(need, q.device, ws) if need else None  # the one-launch step needs none
     _check("sas_decode", lib.sas_decode(
         _ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, Lmax, d, _ptr(lens), _ptr(ksum), topk,
-        int(gated), float(scale), _ptr(out), _ptr(idx_out), _ptr(w), w.numel(), _stream(stream)))
+        int(gated), float(scale), _ptr(out), _ptr(idx_out), _ptr(w), 0 if w is None else w.numel(),
+        _stream(stream)))
     return out
 
 

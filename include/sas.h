@@ -105,14 +105,18 @@ sas_status sas_block_summary(const void* k, sas_dtype dt, int B, int H, int N, i
  *     [B][Hkv]. lens [B] int32 device, 1 <= lens[b] <= N.
  *   ksum  [B][Hkv][N/64][d] fp32 (from sas_block_summary)
  *   logg  log g of each kept block (padding slots 0)
+ *   scores_out  fp32 or NULL: the raw selector scores s_m of every row,
+ *     prefill [B][Hkv][T][T] (row (b, r, t), column m) and decode
+ *     [B][Hkv][N/64]; entries m >= C hold -inf. Written only when non-NULL
+ *     (16-byte aligned); nothing on the attention path reads them.
  *   topk >= 0; topk = 0 gives cnt = 0.
  * Workspace: sas_select_workspace_size().
  */
 size_t sas_select_workspace_size(int B, int Hq, int Hkv, int N, int d, int topk, sas_mode mode);
 sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int Hq, int Hkv,
                       int N, int d, int topk, sas_mode mode, const int32_t* lens, float scale,
-                      int32_t* idx, int32_t* cnt, float* logg, void* ws, size_t ws_bytes,
-                      sas_stream_t stream);
+                      int32_t* idx, int32_t* cnt, float* logg, float* scores_out, void* ws,
+                      size_t ws_bytes, sas_stream_t stream);
 
 /*
  * Prefill selection that allocates nothing and takes no workspace. The paper
@@ -121,7 +125,8 @@ sas_status sas_select(const void* q, sas_dtype dt, const float* ksum, int B, int
  * host runtime that hands a kernel library only its input and output
  * buffers and forbids device allocation after start-up (cudaMalloc can
  * synchronise the device and has no latency bound).
- *   Same arguments, layouts and results as sas_select in SAS_PREFILL mode.
+ *   Same arguments, layouts and results as sas_select in SAS_PREFILL mode
+ *   (without scores_out).
  *   Its scratch (the fp32 query summary of every (b, kv group, query block),
  *   B*Hkv*ceil(N/64)*d*4 bytes) lives in a fixed device array inside the
  *   library of sas_select_prefill_noalloc_capacity() bytes (4 MiB), which

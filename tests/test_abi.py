@@ -77,11 +77,15 @@ def test_rejects_null_and_misaligned_pointers(lib):
 
 def test_rejects_topk_and_workspace(lib):
     st = lib.sas_select(FAKE, 1, FAKE, 1, 4, 4, 128, 64, 129, 0, None, 0.0, FAKE, FAKE, FAKE,
-                        FAKE, 1 << 20, None)
+                        None, FAKE, 1 << 20, None)
     assert st == 2
     st = lib.sas_select(FAKE, 1, FAKE, 1, 4, 4, 128, 64, 2, 0, None, 0.0, FAKE, FAKE, FAKE,
-                        FAKE, 16, None)
+                        None, FAKE, 16, None)
     assert st == 1 and b"workspace too small" in lib.sas_last_error_message()
+    # the optional raw-score output, when given, must be aligned like every other buffer
+    st = lib.sas_select(FAKE, 1, FAKE, 1, 4, 4, 128, 64, 2, 0, None, 0.0, FAKE, FAKE, FAKE,
+                        FAKE + 4, FAKE, 1 << 20, None)
+    assert st == 1 and b"scores_out" in lib.sas_last_error_message()
 
 
 def test_rejects_bad_decode_shapes(lib):

@@ -154,6 +154,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(win)}
 
 
+_SAMPLER: ClockSampler | None = None
+
+
+def clock_sampler(gpu_index: int) -> ClockSampler:
+    """One sampler for the whole run, started before the first workload, so
+    that a short timed region still has samples around it."""
+    global _SAMPLER
+    if _SAMPLER is None:
+        _SAMPLER = ClockSampler(gpu_index)
+        time.sleep(0.5)
+    return _SAMPLER
+
+
 def barrier(world):
     from gated_block_sparse_b200 import dist as D
     D.barrier(world)
@@ -316,7 +329,7 @@ def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
             kss[j] = sas.sas_block_summary(kcs[j]).view(B_ * nblk, Hkv, d_)
     o = torch.empty_like(q)
     stream = torch.cuda.Stream(dev)
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks = clock_sampler(dev.index if dev.index is not None else 0)
 
     def decode(j, qq, out):
         if bt is not None:
@@ -331,7 +344,6 @@ def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
         decode(i % L, q, o)
 
     ms, clk = timed_graphs(step, K, W, world, stream, clocks=clocks)
-    clocks.stop()
 
     # split path (contiguous caches, fp32 summaries): selection alone, attention alone
     split = None
@@ -498,7 +510,7 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
     sbw_ws = torch.empty(max(16, lib.sas_select_bwd_workspace_size(B, Hq, Hkv, N, d)),
                          dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks = clock_sampler(dev.index if dev.index is not None else 0)
 
     def step(i):
         sas.sas_block_summary(k, out=ks)
@@ -509,7 +521,6 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
         sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
 
     ms, clk = timed_graphs(step, K, W, world, stream, chunk=8, clocks=clocks)
-    clocks.stop()
 
     def fwd_step(i):
         sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
@@ -850,6 +861,7 @@ def main():
 
     from gated_block_sparse_b200 import dist as D
     world, rank, local = D.setup()
+    clock_sampler(local if world > 1 else 0)
     records, hosts, baselines = {}, {}, {}
     for name, cfg, opts in plan:
         K = args.steps or DEFAULT_STEPS[cfg]
@@ -862,6 +874,8 @@ def main():
             head["config"] = dict(head["config"], headline=plan[0][0],
                                   records=[n for n, _, _ in plan])
         print(json.dumps(head))
+    if _SAMPLER is not None:
+        _SAMPLER.stop()
     D.teardown(world)
 
 

@@ -60,6 +60,8 @@ constexpr int FD_WARPS = FD_THREADS / 32;
 constexpr int FD_NS = 4;      // summary ring slots
 constexpr int FD_MAXKV = 4;   // K/V ring slots at most
 constexpr int FD_MAXCS = 16;  // cluster size at most
+constexpr int FD_BIG_REGION = 192 * 1024;  // ring region with one CTA per SM
+constexpr size_t FD_SMEM_MAX = 226 * 1024; // dynamic shared memory per CTA at most
 constexpr unsigned FULL = 0xffffffffu;
 
 struct FdSmem {  // byte offsets into dynamic shared memory
@@ -75,8 +77,10 @@ __host__ __device__ inline size_t fd_al(size_t x) { return (x + 127) & ~(size_t)
 // during the scan; then K/V slot 0 (the current block) followed by the list
 // scratch (warp lists, sample, survivors, merge buffer) during selection;
 // K/V slots 0 .. nkv-1 afterwards; the per-warp states at the end.
+// ub_min: the region's size at least (0: two K/V slots, sized for two CTAs
+// per SM; larger when the grid leaves one CTA per SM, for deeper rings).
 __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int kq, int CS,
-                                             int ses) {
+                                             int ses, size_t ub_min = 0) {
   FdSmem L;
   const size_t kvslot = (size_t)2 * SAS_BLOCK * D * es;
   L.wl = kvslot;
@@ -84,6 +88,7 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int k
   L.samp = fd_al(L.wb + (size_t)FD_WARPS * kq * 8);
   L.surv = L.samp + 256 * 8;
   size_t ub = 2 * kvslot;
+  if (ub < ub_min) ub = ub_min;
   if (ub < L.surv + 512 * 8) ub = L.surv + 512 * 8;
   const size_t comb = (size_t)FD_WARPS * G * (D + 2) * 4;
   if (ub < comb) ub = comb;
@@ -162,6 +167,37 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float x0, float x1, f
       : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
 }
 
+// One stage of a transposing warp reduction over CNT values per lane: lanes
+// with bit `o` set keep the upper half of the values, the others the lower
+// half, and each adds its partner's copy of the half it keeps.
+template <int CNT>
+__device__ __forceinline__ void tr_stage(float* v, int lane, int o) {
+  constexpr int H = CNT / 2;
+  const bool up = (lane & o) != 0;
+#pragma unroll
+  for (int i = 0; i < H; ++i) {
+    const float send = up ? v[i] : v[i + H];
+    const float keep = up ? v[i + H] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+
+// Sums NV (8, 16 or 32) values over the warp's 32 lanes at once: lane l
+// returns the total of value index l * NV / 32 (NV - 1 shuffles in all;
+// with NV < 32 several lanes return the same total).
+template <int NV>
+__device__ __forceinline__ float transpose_sum(float (&v)[NV], int lane) {
+  static_assert(NV == 8 || NV == 16 || NV == 32, "8, 16 or 32 values");
+  tr_stage<NV>(v, lane, 16);
+  tr_stage<NV / 2>(v, lane, 8);
+  tr_stage<NV / 4>(v, lane, 4);
+  if constexpr (NV >= 16) tr_stage<NV / 8>(v, lane, 2);
+  else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+  if constexpr (NV == 32) tr_stage<2>(v, lane, 1);
+  else v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+  return v[0];
+}
+
 // Combines two (max, sum exp) pairs; an empty pair is (-FLT_MAX, 0).
 __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
   const float M = fmaxf(m, m2);
@@ -180,11 +216,10 @@ template <typename T, int D, int G, bool PAGED, typename S>
 __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
     const S* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
-    int gated, float scale, int per_max, T* __restrict__ o, int32_t* __restrict__ idx_out,
-    const int32_t* __restrict__ bt, int npages) {
+    int gated, float scale, int per_max, int ub_min, T* __restrict__ o,
+    int32_t* __restrict__ idx_out, const int32_t* __restrict__ bt, int npages) {
   constexpr int TILE = SAS_BLOCK * D;
   constexpr int VEC = Vec16<T>::N;     // elements per 16-byte vector
-  constexpr int NCHK = D / (4 * VEC);  // 16-byte chunks of a key row per lane (4 lanes per key)
   constexpr int CPL = D / 32;          // output columns per lane
   constexpr int PER = D / 32;          // summary elements per lane
   extern __shared__ __align__(128) unsigned char sm[];
@@ -193,7 +228,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   const int crank = (int)cluster.block_rank();
   const int lg = ceil_log2(topk > 0 ? topk : 1);
   const int kq = 1 << lg;  // list stride (power of two)
-  const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S));
+  const FdSmem L = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S), ub_min);
   unsigned char* U = sm + L.u;
   const size_t kvslot = (size_t)2 * TILE * sizeof(T);
   S* ring = reinterpret_cast<S*>(U);
@@ -601,108 +636,106 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       idx_out[row * topk + pos] = mi;
     }
   }
-  float m_w[G], l_w[G], acc[G][CPL];
+  // Each warp takes 8 keys of every unit (keys wid*8 .. wid*8+7) and keeps
+  // its own online-softmax state per head. Lane l holds columns
+  // [l*CPL, l*CPL + CPL) of q and of the accumulators of every head. The
+  // q.k partial sums of the warp's 8 keys x GP heads (one pass per group of
+  // at most 4 heads) are summed over the lanes by a transposing reduction:
+  // each shuffle stage halves the values a lane carries, so 8*GP sums cost
+  // fewer than 8*GP shuffles and lane l ends with the sum of key l/4 and
+  // head (l%4)/(4/GP) of the pass (lanes holding the same pair agree).
+  constexpr int GP = G < 4 ? G : 4;  // heads per pass
+  constexpr int HP = G / GP;         // passes
+  constexpr int NV = 8 * GP;         // partial sums per lane per pass
+  float qr[G][CPL], acc[G][CPL], m_p[HP], l_p[HP];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    m_w[h] = -INFINITY;
-    l_w[h] = 0.f;
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+    for (int c = 0; c < CPL; ++c) {
+      qr[h][c] = q_s[h * D + lane * CPL + c];
+      acc[h][c] = 0.f;
+    }
   }
-  const int key = wid * 8 + (lane >> 2);  // this lane's key of the unit (4 lanes per key)
-  const int qq = lane & 3;                // and its quarter of each 16-byte chunk group
+#pragma unroll
+  for (int p = 0; p < HP; ++p) {
+    m_p[p] = -INFINITY;
+    l_p[p] = 0.f;
+  }
+  const int jj = lane >> 2;                                  // this lane's key of the 8
+  const int hp = (lane & 3) / (4 / GP);                      // and head within a pass
+  const bool uniq = (lane & (4 / GP - 1)) == 0;              // first lane holding the pair
+  float* pw = zp + wid * (2 * 8 * G);                        // [8 keys][G] p of this warp
+  float* aw = pw + 8 * G;                                    // [G] rescale factors
   for (int i = 0; i < nu; ++i) {
     const int slot = i % NKV;
     const int u = unit_of(i);
     const bool cur = (u == kk);
     const float bias = (!cur && gated) ? key_score(fin[u]) - lse : 0.f;
     mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
-    const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot);
+    const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot) + (size_t)wid * 8 * D;
     const T* vt = kt + TILE;
-    float dot[G], dot1[G];
+    const bool masked = cur && (wid * 8 + jj >= ncur);
 #pragma unroll
-    for (int h = 0; h < G; ++h) dot[h] = dot1[h] = 0.f;
+    for (int p = 0; p < HP; ++p) {
+      float part[NV];
 #pragma unroll
-    for (int c = 0; c < NCHK; ++c) {
-      const int d0 = c * 4 * VEC + qq * VEC;
-      float kv[VEC];
-      Vec16<T>::load(kt + (size_t)key * D + d0, kv);
+      for (int k8 = 0; k8 < 8; ++k8) {
+        float kv[CPL];
+        loadn<CPL>(kt + (size_t)k8 * D + lane * CPL, kv);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+        for (int g = 0; g < GP; ++g) {
+          float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < VEC; e += 4) {
-          const float4 qv = *reinterpret_cast<const float4*>(q_s + h * D + d0 + e);
-          fma2(dot[h], dot1[h], kv[e], kv[e + 1], qv.x, qv.y);
-          fma2(dot[h], dot1[h], kv[e + 2], kv[e + 3], qv.z, qv.w);
+          for (int c = 0; c < CPL; ++c) a = fmaf(qr[p * GP + g][c], kv[c], a);
+          part[k8 * GP + g] = a;
         }
       }
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h) dot[h] += dot1[h];
-    // z of this lane's key (the four lanes of a key hold the same value);
-    // the warp's 8 keys meet in shared memory, read back by broadcast.
-    float* zw = zp + wid * (2 * 8 * G);  // [8 keys][G] z, then [8 keys][G] p
-    float* pw = zw + 8 * G;
-    float z[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float d2 = dot[h] + __shfl_xor_sync(FULL, dot[h], 1);
-      d2 += __shfl_xor_sync(FULL, d2, 2);
-      z[h] = (cur && key >= ncur) ? -INFINITY : d2 * scale + bias;
-    }
-    const int kl = lane >> 2;
-    if (qq == 0) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) zw[kl * G + h] = z[h];
-    }
-    __syncwarp();
-    float zmax[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) zmax[h] = -INFINITY;
-#pragma unroll
-    for (int k8 = 0; k8 < 8; ++k8) {
-      float zz[G];
-      loadg<G>(zw + k8 * G, zz);
-#pragma unroll
-      for (int h = 0; h < G; ++h) zmax[h] = fmaxf(zmax[h], zz[h]);
-    }
-    float alpha[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mn = fmaxf(m_w[h], zmax[h]);
-      float p;
+      const float dot = transpose_sum<NV>(part, lane);
+      const float z = masked ? -INFINITY : dot * scale + bias;
+      float zmax = z;
+      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 4));
+      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 8));
+      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 16));
+      const float mn = fmaxf(m_p[p], zmax);
+      float pr, alpha;
       if (mn == -INFINITY) {  // every key seen so far is masked
-        p = 0.f;
-        alpha[h] = 1.f;
+        pr = 0.f;
+        alpha = 1.f;
       } else {
-        p = __expf(z[h] - mn);
-        alpha[h] = __expf(m_w[h] - mn);
+        pr = __expf(z - mn);
+        alpha = __expf(m_p[p] - mn);
       }
-      m_w[h] = mn;
-      if (qq == 0) pw[kl * G + h] = p;
+      m_p[p] = mn;
+      float ps = pr;
+      ps += __shfl_xor_sync(FULL, ps, 4);
+      ps += __shfl_xor_sync(FULL, ps, 8);
+      ps += __shfl_xor_sync(FULL, ps, 16);
+      l_p[p] = l_p[p] * alpha + ps;
+      const int h = p * GP + hp;
+      if (uniq) {
+        pw[jj * G + h] = pr;
+        if (jj == 0) aw[h] = alpha;
+      }
     }
     __syncwarp();
+    {
+      float al[G];
+      loadg<G>(aw, al);
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+      for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[h][c] *= alpha[h];
-    float psum[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) psum[h] = 0.f;
+        for (int c = 0; c < CPL; ++c) acc[h][c] *= al[h];
+    }
 #pragma unroll
     for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys
       float pk[G], v[CPL];
       loadg<G>(pw + k8 * G, pk);
-      loadn<CPL>(vt + (size_t)(wid * 8 + k8) * D + lane * CPL, v);
+      loadn<CPL>(vt + (size_t)k8 * D + lane * CPL, v);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        psum[h] += pk[h];
+      for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk[h], pk[h], v[c], v[c + 1]);
-      }
     }
-#pragma unroll
-    for (int h = 0; h < G; ++h) l_w[h] = l_w[h] * alpha[h] + psum[h];
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
     if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
@@ -722,9 +755,9 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
 #pragma unroll
     for (int c = 0; c < CPL; ++c) w[lane * CPL + c] = acc[h][c];
   }
-  if (lane == 0) {
+  if (lane < 4 && uniq) {  // the lanes of key 0 hold every head's (m, l) once
 #pragma unroll
-    for (int h = 0; h < G; ++h) mlw[h * FD_WARPS + wid] = make_float2(m_w[h], l_w[h]);
+    for (int p = 0; p < HP; ++p) mlw[(p * GP + hp) * FD_WARPS + wid] = make_float2(m_p[p], l_p[p]);
   }
   __syncthreads();
   {
@@ -783,15 +816,18 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
 namespace {
 
 struct FdPick {
-  int dev, rows, nblk, kq, CS;
+  int dev, rows, nblk, kq, CS, ub;
 };
 
-// Cluster size for a shape: the largest of 16, 8, 4, 2, 1 (and >= G, since
-// CTA h combines head h) whose clusters of all rows are co-resident on the
-// GPU; if none is, the largest that launches. Cached per shape, so repeated
-// launches make no occupancy queries.
+// Cluster size and ring region for a shape. Candidates: cluster sizes 16,
+// 8, 4, 2, 1 (>= G, since CTA h combines head h), each first with a large
+// ring region (when the grid leaves at most one CTA per SM: deeper summary
+// and K/V rings) and then with the small one (two CTAs per SM). The first
+// whose clusters of all rows are co-resident on the GPU wins; if none is,
+// the first that launches. Cached per shape, so repeated launches make no
+// occupancy queries.
 template <typename T, int D, int G, bool PAGED, typename S>
-cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
+cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out, int& ub_out) {
   static std::mutex mu;
   static FdPick cache[32];
   static int ncache = 0;
@@ -805,54 +841,65 @@ cudaError_t pick_cluster(int B, int Hkv, int nblk, int kq, int& CS_out) {
       if (cache[i].dev == dev && cache[i].rows == rows && cache[i].nblk == nblk &&
           cache[i].kq == kq) {
         CS_out = cache[i].CS;
+        ub_out = cache[i].ub;
         return cudaSuccess;
       }
   }
+  int nsm = 0;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   auto kern = k_decode_fused<T, D, G, PAGED, S>;
-  int best = 0, first = 0;
+  int best = 0, best_ub = 0, first = 0, first_ub = 0;
   const int cands[5] = {16, 8, 4, 2, 1};
-  for (int ci = 0; ci < 5; ++ci) {
+  for (int ci = 0; ci < 5 && !best; ++ci) {
     const int CS = cands[ci];
     if (CS < G) break;
-    const size_t smem =
-        fd_layout(D, G, (int)sizeof(T), (nblk + CS - 1) / CS, kq, CS, (int)sizeof(S)).total;
-    if (smem > 227 * 1024) continue;
-    if (ensure_smem(kern, smem) != cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    if (CS > 8 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CS, Hkv, B);
-    cfg.blockDim = dim3(FD_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int ncl = 0;
-    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    if (ncl < 1) continue;
-    if (!first) first = CS;
-    if (ncl >= rows) {
-      best = CS;
-      break;
+    for (int big = (rows * CS <= nsm) ? 1 : 0; big >= 0 && !best; --big) {
+      const int ub = big ? FD_BIG_REGION : 0;
+      const size_t smem =
+          fd_layout(D, G, (int)sizeof(T), (nblk + CS - 1) / CS, kq, CS, (int)sizeof(S), ub).total;
+      if (smem > FD_SMEM_MAX) continue;
+      if (ensure_smem(kern, smem) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      if (CS > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                         1) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(CS, Hkv, B);
+      cfg.blockDim = dim3(FD_THREADS);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = CS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      if (ncl < 1) continue;
+      if (!first) {
+        first = CS;
+        first_ub = ub;
+      }
+      if (ncl >= rows) {
+        best = CS;
+        best_ub = ub;
+      }
     }
   }
   CS_out = best ? best : first;
+  ub_out = best ? best_ub : first_ub;
   if (!CS_out) return cudaErrorInvalidConfiguration;
   std::lock_guard<std::mutex> lock(mu);
-  if (ncache < 32) cache[ncache++] = FdPick{dev, rows, nblk, kq, CS_out};
+  if (ncache < 32) cache[ncache++] = FdPick{dev, rows, nblk, kq, CS_out, ub_out};
   return cudaSuccess;
 }
 
@@ -864,11 +911,12 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   auto kern = k_decode_fused<T, D, G, PAGED, S>;
   const int nblk = Lmax / SAS_BLOCK;
   const int kq = 1 << ceil_log2(topk > 0 ? topk : 1);
-  int CS = 0;
-  cudaError_t e = pick_cluster<T, D, G, PAGED, S>(B, Hkv, nblk, kq, CS);
+  int CS = 0, ub = 0;
+  cudaError_t e = pick_cluster<T, D, G, PAGED, S>(B, Hkv, nblk, kq, CS, ub);
   if (e != cudaSuccess) return e;
   const int per_max = (nblk + CS - 1) / CS;
-  const size_t smem = fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S)).total;
+  const size_t smem =
+      fd_layout(D, G, (int)sizeof(T), per_max, kq, CS, (int)sizeof(S), ub).total;
   e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -887,8 +935,8 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
                             static_cast<const T*>(vc), static_cast<const S*>(ksum), Hkv, Lmax,
-                            lens, topk, gated, scale,
-                            per_max, static_cast<T*>(o), idx_out, bt, npages);
+                            lens, topk, gated, scale, per_max, ub, static_cast<T*>(o), idx_out,
+                            bt, npages);
 }
 
 template <typename T, int D>

@@ -496,6 +496,131 @@ sas_status sas_select_bwd(const void* q, sas_dtype dt, const float* ksum, int B,
                      "sas_select_bwd launch");
 }
 
+// ---------------------------------------------------------------- per-token selection
+sas_status sas_select_tokens(const void* q, sas_dtype dt, const float* ksum, int B, int Hq,
+                             int Hkv, int N, int d, int topk, float scale, int32_t* idx,
+                             int32_t* cnt, float* logg, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE(N <= sas::tokens_max_n(), SAS_ERR_UNSUPPORTED,
+          "per-token selection supports N <= %d (got %d)", sas::tokens_max_n(), N);
+  if (B == 0 || N == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(cnt);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  if (N > 64) REQUIRE_PTR(ksum);
+  return cuda_status(sas::launch_select_tokens(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d, topk,
+                                               resolve_scale(scale, d), idx, cnt, logg,
+                                               (cudaStream_t)stream),
+                     "sas_select_tokens launch");
+}
+
+sas_status sas_attn_fwd_tokens(const void* q, const void* k, const void* v, sas_dtype dt, int B,
+                               int Hq, int Hkv, int N, int d, const int32_t* idx,
+                               const int32_t* cnt, const float* logg, int topk, float scale,
+                               void* o, float* lse, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE(N <= sas::tokens_max_n(), SAS_ERR_UNSUPPORTED,
+          "per-token attention supports N <= %d (got %d)", sas::tokens_max_n(), N);
+  if (B == 0 || N == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(cnt);
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(lse);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+  }
+  return cuda_status(sas::launch_attn_fwd_tokens(q, k, v, dt == SAS_BF16, B, Hq, Hkv, N, d, idx,
+                                                 cnt, logg, topk, resolve_scale(scale, d), o,
+                                                 lse, (cudaStream_t)stream),
+                     "sas_attn_fwd_tokens launch");
+}
+
+size_t sas_attn_bwd_tokens_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  (void)Hq;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return 0;
+  return a16(sas::attn_bwd_tokens_ws_bytes(B, Hkv, N, d));
+}
+
+sas_status sas_attn_bwd_tokens(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, sas_dtype dt, int B, int Hq, int Hkv, int N,
+                               int d, const float* lse, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* dq, void* dk,
+                               void* dv, float* dlogg, void* ws, size_t ws_bytes,
+                               sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE(N <= sas::tokens_max_n(), SAS_ERR_UNSUPPORTED,
+          "per-token attention supports N <= %d (got %d)", sas::tokens_max_n(), N);
+  if (B == 0 || N == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(lse);
+  REQUIRE_PTR(cnt);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  REQUIRE_PTR(ws);
+  if (topk > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(logg);
+    REQUIRE_PTR(dlogg);
+  }
+  const size_t need = sas_attn_bwd_tokens_workspace_size(B, Hq, Hkv, N, d);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)",
+          ws_bytes, need);
+  return cuda_status(sas::launch_attn_bwd_tokens(q, k, v, o, dout, dt == SAS_BF16, B, Hq, Hkv, N,
+                                                 d, lse, idx, cnt, logg, topk,
+                                                 resolve_scale(scale, d), dq, dk, dv, dlogg, ws,
+                                                 (cudaStream_t)stream),
+                     "sas_attn_bwd_tokens launch");
+}
+
+size_t sas_select_bwd_tokens_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  (void)Hq;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return 0;
+  return a16(sas::select_bwd_tokens_ws_bytes(B, Hkv, N, d));
+}
+
+sas_status sas_select_bwd_tokens(const void* q, sas_dtype dt, const float* ksum, int B, int Hq,
+                                 int Hkv, int N, int d, int topk, float scale, const int32_t* idx,
+                                 const int32_t* cnt, const float* dlogg, void* dq, void* dk,
+                                 void* ws, size_t ws_bytes, sas_stream_t stream) {
+  g_last_error.clear();
+  sas_status s = check_common(dt, B, Hq, Hkv, N, d, topk);
+  if (s != SAS_OK) return s;
+  REQUIRE(N <= sas::tokens_max_n(), SAS_ERR_UNSUPPORTED,
+          "per-token selector backward supports N <= %d (got %d)", sas::tokens_max_n(), N);
+  if (B == 0 || N < 128 || topk == 0) return SAS_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(ksum);
+  REQUIRE_PTR(idx);
+  REQUIRE_PTR(cnt);
+  REQUIRE_PTR(dlogg);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  const size_t need = sas_select_bwd_tokens_workspace_size(B, Hq, Hkv, N, d);
+  REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small: %zu < %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  return cuda_status(sas::launch_select_bwd_tokens(q, dt == SAS_BF16, ksum, B, Hq, Hkv, N, d,
+                                                   topk, resolve_scale(scale, d), idx, cnt,
+                                                   dlogg, dq, dk, ws, (cudaStream_t)stream),
+                     "sas_select_bwd_tokens launch");
+}
+
 // ---------------------------------------------------------------- device status
 sas_status sas_device_status(int clear, sas_stream_t stream) {
   g_last_error.clear();
@@ -511,6 +636,7 @@ sas_status sas_device_status(int clear, sas_stream_t stream) {
       {"k_attn_simt", sas::attn_simt_error_word},
       {"k_wait_selftest", sas::selftest_error_word},
       {"k_summary_last", sas::summary_error_word},
+      {"k_attn_*_tokens", sas::tokens_error_word},
   };
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "sas_device_status synchronize");

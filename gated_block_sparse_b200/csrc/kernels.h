@@ -30,6 +30,32 @@ cudaError_t launch_summary_last(const void* k, int bf16, int B, int H, int N, in
                                 cudaStream_t st);
 uint32_t* summary_error_word();
 
+// Per-token selection prefill (k_tokens.cu): selection rows per query token,
+// idx/logg [B][Hkv][N][topk], cnt [B][Hkv][N]; N <= tokens_max_n().
+int tokens_max_n();
+cudaError_t launch_select_tokens(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                 int Hkv, int N, int d, int topk, float scale, int32_t* idx,
+                                 int32_t* cnt, float* logg, cudaStream_t st);
+cudaError_t launch_attn_fwd_tokens(const void* q, const void* k, const void* v, int bf16, int B,
+                                   int Hq, int Hkv, int N, int d, const int32_t* idx,
+                                   const int32_t* cnt, const float* logg, int topk, float scale,
+                                   void* o, float* lse, cudaStream_t st);
+size_t attn_bwd_tokens_ws_bytes(int B, int Hkv, int N, int d);
+cudaError_t launch_attn_bwd_tokens(const void* q, const void* k, const void* v, const void* o,
+                                   const void* dout, int bf16, int B, int Hq, int Hkv, int N,
+                                   int d, const float* lse, const int32_t* idx,
+                                   const int32_t* cnt, const float* logg, int topk, float scale,
+                                   void* dq, void* dk, void* dv, float* dlogg, void* ws,
+                                   cudaStream_t st);
+// Selector backward for per-token rows (eq. 8), added into dq and dk; ws
+// holds the fp32 block-summary gradients [B][Hkv][N/64][d].
+size_t select_bwd_tokens_ws_bytes(int B, int Hkv, int N, int d);
+cudaError_t launch_select_bwd_tokens(const void* q, int bf16, const float* ksum, int B, int Hq,
+                                     int Hkv, int N, int d, int topk, float scale,
+                                     const int32_t* idx, const int32_t* cnt, const float* dlogg,
+                                     void* dq, void* dk, void* ws, cudaStream_t st);
+uint32_t* tokens_error_word();
+
 // ---- selection
 // Shared layout of one row's per-chunk partial results (decode scratch).
 struct SelectPlan {

@@ -261,6 +261,50 @@ sas_status sas_block_summary_last(const void* k, sas_dtype dt, int B, int H, int
                                   const int32_t* block_table, int npages, sas_stream_t stream);
 
 /*
+ * Per-token selection prefill (SAS close reading, section 2.4: the fused
+ * kernel masks, per query, the blocks below that query's gate threshold and
+ * skips key tiles no query selected). Each query token i of kv group r has
+ * its own row: qbar_i = the mean of the group's heads at token i, C_i = i/64
+ * history blocks, s_m = scale * qbar_i . ksum_m, log g = s - LSE(s), Top-K
+ * with ties to the lower block index; every head of the group attends over
+ * its token's set and the causal part of the token's own block.
+ *   Selection rows: idx/logg [B][Hkv][N][topk] (ascending, -1 / 0 padding),
+ *   cnt [B][Hkv][N]; dlogg has the layout of logg.
+ *   sas_select_tokens: q [B][Hq][N][d] (dt), ksum [B][Hkv][N/64][d] fp32.
+ *   sas_attn_fwd_tokens / sas_attn_bwd_tokens: as sas_attn_fwd /
+ *   sas_attn_bwd with per-token rows; the backward's workspace is
+ *   sas_attn_bwd_tokens_workspace_size() bytes.
+ *   sas_select_bwd_tokens: the selector's gradient for per-token rows (eq. 8,
+ *   section 2.3, as sas_select_bwd): for token i of group r with C = i/64,
+ *   ds_m = dlogg[slot of m] [m in I_i] - g_m sum_{l in I_i} dlogg[slot of l];
+ *   each head of the group gets scale * sum_m ds_m ksum_m / G ADDED into dq
+ *   at token i, and each of block m's 64 keys gets
+ *   scale * sum_i ds_im qbar_i / 64 ADDED into dk. Its workspace is
+ *   sas_select_bwd_tokens_workspace_size() bytes (fp32 summary gradients).
+ *   N <= 32832 (512 history blocks per query block); larger N returns
+ *   SAS_ERR_UNSUPPORTED. CUDA-core kernels (fp32 arithmetic).
+ */
+sas_status sas_select_tokens(const void* q, sas_dtype dt, const float* ksum, int B, int Hq,
+                             int Hkv, int N, int d, int topk, float scale, int32_t* idx,
+                             int32_t* cnt, float* logg, sas_stream_t stream);
+sas_status sas_attn_fwd_tokens(const void* q, const void* k, const void* v, sas_dtype dt, int B,
+                               int Hq, int Hkv, int N, int d, const int32_t* idx,
+                               const int32_t* cnt, const float* logg, int topk, float scale,
+                               void* o, float* lse, sas_stream_t stream);
+size_t sas_attn_bwd_tokens_workspace_size(int B, int Hq, int Hkv, int N, int d);
+size_t sas_select_bwd_tokens_workspace_size(int B, int Hq, int Hkv, int N, int d);
+sas_status sas_select_bwd_tokens(const void* q, sas_dtype dt, const float* ksum, int B, int Hq,
+                                 int Hkv, int N, int d, int topk, float scale, const int32_t* idx,
+                                 const int32_t* cnt, const float* dlogg, void* dq, void* dk,
+                                 void* ws, size_t ws_bytes, sas_stream_t stream);
+sas_status sas_attn_bwd_tokens(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, sas_dtype dt, int B, int Hq, int Hkv, int N,
+                               int d, const float* lse, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* dq, void* dk,
+                               void* dv, float* dlogg, void* ws, size_t ws_bytes,
+                               sas_stream_t stream);
+
+/*
  * One decode step from and to host memory: enqueues on `stream` the copy of
  * q_host ([B][Hq][d], dt; page-locked for the copy to be asynchronous) into
  * q_dev and the sas_decode step. When o_host is page-locked host memory

@@ -416,19 +416,29 @@ sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, cons
   if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
   const size_t bytes = (size_t)B * Hq * d * (dt == SAS_BF16 ? 2 : 4);
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return cuda_status(e, "sas_decode_host copy in");
-  // A page-locked o_host is addressable from the device (unified addressing):
-  // the combining CTAs then write o straight into it, with no separate copy.
-  void* o_out = nullptr;
-  cudaPointerAttributes at;
-  const cudaError_t pa = cudaPointerGetAttributes(&at, o_host);
-  if (pa != cudaSuccess)
-    cudaGetLastError();  // clears that query's own error: a pageable o_host is not a failure
-  else if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr &&
-           aligned16(at.devicePointer))
-    o_out = at.devicePointer;
-  e = sas::launch_decode_fused(q_dev, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, ksum,
+  // Page-locked host buffers are addressable from the device (unified
+  // addressing): the step then reads q and writes o straight over the bus,
+  // with no separate copy; otherwise q is copied into q_dev first and o_dev
+  // is copied back. A failed query only means "not page-locked".
+  auto mapped = [](const void* p) -> const void* {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      cudaGetLastError();  // clears that query's own error
+      return nullptr;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr && aligned16(at.devicePointer))
+      return at.devicePointer;
+    return nullptr;
+  };
+  const void* q_in = mapped(q_host);
+  void* o_out = const_cast<void*>(mapped(o_host));
+  cudaError_t e = cudaSuccess;
+  if (!q_in) {
+    e = cudaMemcpyAsync(q_dev, q_host, bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_status(e, "sas_decode_host copy in");
+    q_in = q_dev;
+  }
+  e = sas::launch_decode_fused(q_in, kc, vc, dt == SAS_BF16, B, Hq, Hkv, Lmax, d, lens, ksum,
                                topk, gated, resolve_scale(scale, d), o_out ? o_out : o_dev,
                                idx_out, st);
   if (e != cudaSuccess) return cuda_status(e, "sas_decode_host launch");

@@ -305,14 +305,15 @@ sas_status sas_attn_bwd_tokens(const void* q, const void* k, const void* v, cons
                                sas_stream_t stream);
 
 /*
- * One decode step from and to host memory: enqueues on `stream` the copy of
- * q_host ([B][Hq][d], dt; page-locked for the copy to be asynchronous) into
- * q_dev and the sas_decode step. When o_host is page-locked host memory
- * (cudaHostAlloc / cudaMallocHost), the step writes o straight into it over
- * the bus and o_dev is not touched; otherwise it writes o_dev and a copy
- * into o_host follows. The caches, lens and summaries are device memory as
- * in sas_decode. Returns once the work is enqueued; o_host is valid after
- * the stream reaches that point.
+ * One decode step from and to host memory. When q_host is page-locked host
+ * memory (cudaHostAlloc / cudaMallocHost), the step reads q straight from
+ * it over the bus and q_dev is not touched; otherwise the copy of q_host
+ * ([B][Hq][d], dt) into q_dev is enqueued on `stream` first. Likewise, when
+ * o_host is page-locked the step writes o straight into it and o_dev is not
+ * touched; otherwise it writes o_dev and a copy into o_host follows. The
+ * caches, lens and summaries are device memory as in sas_decode. Returns
+ * once the work is enqueued; o_host is valid after the stream reaches that
+ * point, and q_host may be rewritten only after that point too.
  */
 sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, const void* vc,
                            sas_dtype dt, int B, int Hq, int Hkv, int Lmax, int d,

@@ -611,8 +611,9 @@ def test_decode_paged_matches_contiguous_and_oracle(gated):
 
 
 def test_decode_host_buffers_match_device_call():
-    """sas_decode_host (pinned host q in, pinned host o out, one C call) gives
-    the device call's output exactly."""
+    """sas_decode_host gives the device call's output exactly, with pinned
+    host q and o (read and written by the step over the bus) and with
+    pageable ones (copied through the device staging buffers)."""
     x = inputs.gen_decode(2, 32, 8, 4096, 128, [4096, 3000], "bf16", seed=73, planted=8)
     q, kc, vc, lens = x["q"], dev(x["kc"]), dev(x["vc"]), dev(x["lens"])
     ks = sas.sas_block_summary(kc)
@@ -624,6 +625,13 @@ def test_decode_host_buffers_match_device_call():
     sas.sas_decode_host(qh, qd, kc, vc, lens, ks, 15, od, oh)
     torch.cuda.synchronize()
     assert torch.equal(oh, o_ref)
+    # pageable host buffers: q is copied in through q_dev, o copied out of o_dev
+    qp = q.clone()
+    op = torch.empty(q.shape, dtype=q.dtype)
+    qd.zero_()
+    sas.sas_decode_host(qp, qd, kc, vc, lens, ks, 15, od, op)
+    torch.cuda.synchronize()
+    assert torch.equal(op, o_ref) and torch.equal(qd.cpu(), q)
 
 
 # ------------------------------------------------------------------ summary upkeep

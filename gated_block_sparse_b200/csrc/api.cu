@@ -549,6 +549,11 @@ sas_status sas_attn_fwd_tokens(const void* q, const void* k, const void* v, sas_
     REQUIRE_PTR(idx);
     REQUIRE_PTR(logg);
   }
+  if (sas::attn_fwd_tc_supported(dt == SAS_BF16, d, Hq, Hkv) && topk > 0)
+    return cuda_status(sas::launch_attn_fwd_tc_tokens(q, k, v, B, Hq, Hkv, N, idx, cnt, logg,
+                                                      topk, resolve_scale(scale, d), o, lse,
+                                                      (cudaStream_t)stream),
+                       "sas_attn_fwd_tokens launch");
   return cuda_status(sas::launch_attn_fwd_tokens(q, k, v, dt == SAS_BF16, B, Hq, Hkv, N, d, idx,
                                                  cnt, logg, topk, resolve_scale(scale, d), o,
                                                  lse, (cudaStream_t)stream),
@@ -592,6 +597,12 @@ sas_status sas_attn_bwd_tokens(const void* q, const void* k, const void* v, cons
   const size_t need = sas_attn_bwd_tokens_workspace_size(B, Hq, Hkv, N, d);
   REQUIRE(ws_bytes >= need, SAS_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)",
           ws_bytes, need);
+  if (sas::attn_fwd_tc_supported(dt == SAS_BF16, d, Hq, Hkv) && topk > 0)
+    return cuda_status(sas::launch_attn_bwd_tc_tokens(q, k, v, o, dout, B, Hq, Hkv, N, lse, idx,
+                                                      cnt, logg, topk, resolve_scale(scale, d),
+                                                      dq, dk, dv, dlogg, ws,
+                                                      (cudaStream_t)stream),
+                       "sas_attn_bwd_tokens launch");
   return cuda_status(sas::launch_attn_bwd_tokens(q, k, v, o, dout, dt == SAS_BF16, B, Hq, Hkv, N,
                                                  d, lse, idx, cnt, logg, topk,
                                                  resolve_scale(scale, d), dq, dk, dv, dlogg, ws,

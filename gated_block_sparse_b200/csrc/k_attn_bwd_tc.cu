@@ -36,6 +36,13 @@
 // unit) drain at about 20 bytes per cycle per SM, so the flush warps take
 // them off the gradient warps' path.
 // 512 TMEM columns and about 213 KB of shared memory: one CTA per SM.
+//
+// Per-token selection (TOK = true; section 2.4): units are the union of the
+// blocks the query block's tokens selected (a bitmask walked in ascending
+// order), then the current block; each gradient row adds its token's log g
+// where its token selected the unit's block and masks the unit otherwise,
+// and adds its logit gradients over the unit's keys into its token's slot of
+// dlogg ([B][Hkv][N][topk]).
 #include <cuda.h>
 #include <math.h>
 
@@ -67,7 +74,9 @@ constexpr uint32_t OFF_T = OFF_DS + PT_BYTES;         // fp32 [warp][2][8 keys][
 constexpr int FSLOT = 1;         // [32 keys][32 d] slices per flush warp
 constexpr uint32_t OFF_DL = OFF_T + NFW * FSLOT * 32 * 32 * 4;  // fp32 [unit][warp] d(log g) partials
 constexpr uint32_t OFF_BAR = OFF_DL + 129 * 8 * 4 + 64;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+constexpr uint32_t OFF_UM = OFF_BAR + 256;  // per-token mode: union bitmask and its count
+constexpr uint32_t SMEM_BYTES = OFF_UM + 128;
+constexpr int TOK_UMAX = 512;  // history blocks of a query block at most (per-token mode)
 constexpr float LOG2E = 1.4426950408889634f;
 
 enum Bar {
@@ -93,6 +102,7 @@ __device__ __forceinline__ void named_bar_softmax() {
 
 }  // namespace
 
+template <bool TOK>
 __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap domap,
@@ -112,16 +122,58 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
   const int r = blockIdx.y / pairs, hp = blockIdx.y % pairs, b = blockIdx.z;
   const int h0 = r * G + 2 * hp;
   const size_t srow = ((size_t)b * Hkv + r) * T_ + t;
-  const int kk = min(max(cnt[srow], 0), topk);
-  const int nunits = kk + 1;
-  const int32_t* idx_row = idx + srow * topk;
-  const float* logg_row = logg + srow * topk;
+  int kk = TOK ? 0 : min(max(cnt[srow], 0), topk);
+  const int32_t* idx_row = idx + (TOK ? 0 : srow * topk);
+  const float* logg_row = logg + (TOK ? 0 : srow * topk);
   if ((smem_u32(sm) & 1023u) != 0) {
     if (tid == 0) atomicOr(err, kErrBadIndex);
     return;
   }
+  const size_t tok0 = ((size_t)b * Hkv + r) * N + 64 * t;  // first token row of the block
+  const int words = (t + 31) / 32;
+  uint32_t* umask = reinterpret_cast<uint32_t*>(sm + OFF_UM);  // per-token: TOK_UMAX / 32 words
+  if constexpr (TOK) {
+    int& ucnt = *reinterpret_cast<int*>(sm + OFF_UM + TOK_UMAX / 8);
+    const int nr = min(64, N - 64 * t);
+    for (int w = tid; w < words; w += BT_THREADS) umask[w] = 0u;
+    __syncthreads();
+    for (int e = tid; e < nr * topk; e += BT_THREADS) {
+      const int i = e / topk, p = e - i * topk;
+      if (p < min(max(cnt[tok0 + i], 0), topk)) {
+        const int m = idx[(tok0 + i) * topk + p];
+        if (m >= 0 && m < t) atomicOr(&umask[m >> 5], 1u << (m & 31));
+        else atomicOr(err, kErrBadIndex);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int c = 0;
+      for (int w = lane; w < words; w += 32) c += __popc(umask[w]);
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) ucnt = c;
+    }
+    __syncthreads();
+    kk = ucnt;
+  }
+  const int nunits = kk + 1;
+  // per-token: smallest selected block >= from (ascending), -1 past the end
+  auto next_unit = [&](int from) -> int {
+    for (int w = from >> 5; w < words; ++w) {
+      const uint32_t word = umask[w] & (w == (from >> 5) ? (~0u << (from & 31)) : ~0u);
+      if (word) return w * 32 + __ffs(word) - 1;
+    }
+    return -1;
+  };
+  // block of unit j (units in order; per-token mode advances the cursor)
+  int ucur = -1;
   auto unit_block = [&](int j) -> int {
-    int blk = (j < kk) ? idx_row[j] : t;
+    int blk;
+    if constexpr (TOK) {
+      if (j < kk) ucur = next_unit(ucur + 1);
+      blk = (j < kk) ? ucur : t;
+    } else {
+      blk = (j < kk) ? idx_row[j] : t;
+    }
     if (blk < 0 || blk >= t) blk = t;
     return blk;
   };
@@ -157,7 +209,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
         const int s = j % NKV;
         if (j >= NKV) mbar_wait_data(&bars[B_KVE + s], ((j / NKV) - 1) & 1, err);
         const int blk = unit_block(j);
-        if (j < kk && blk != idx_row[j]) atomicOr(err, kErrBadIndex);
+        if (!TOK && j < kk && blk != idx_row[j]) atomicOr(err, kErrBadIndex);
         unsigned char* st = sm + OFF_KV + s * KV_STAGE;
         mbar_arrive_expect_tx(&bars[B_KVF + s], KV_STAGE);
         const int plane = b * Hkv + r;
@@ -308,9 +360,27 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     unsigned char* dsrow = sm + OFF_DS + row * 128;
     const int gtid = hc * 128 + row;  // 0..255 over the gradient warps
     float* dl_s = reinterpret_cast<float*>(sm + OFF_DL);
+    // per-token: this row's own list (ascending), walked as the units advance
+    const size_t trow = tok0 + (valid ? qr : 0);
+    const int tn = (TOK && valid) ? min(max(cnt[trow], 0), topk) : 0;
+    const int32_t* tidx = idx + trow * topk;
+    const float* tlog = logg + trow * topk;
+    int tp = 0;
     for (int j = 0; j < nunits; ++j) {
       const bool cur = (j == kk);
-      const float bias = cur ? 0.f : logg_row[j] * LOG2E;
+      float bias;
+      bool sel = !cur;
+      if constexpr (TOK) {
+        bias = 0.f;
+        if (!cur) {
+          const int blk = unit_block(j);
+          while (tp < tn && tidx[tp] < blk) ++tp;
+          sel = tp < tn && tidx[tp] == blk;
+          bias = sel ? tlog[tp] * LOG2E : -INFINITY;
+        }
+      } else {
+        bias = cur ? 0.f : logg_row[j] * LOG2E;
+      }
       mbar_wait_data(&bars[B_SF], j & 1, err);
       tc::fence_after_sync();
       float sv[32], dp[32];
@@ -354,7 +424,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PF]);
-      if (!cur) {  // this warp's part of d(log g) of the slot, summed at the end
+      if constexpr (TOK) {  // this row's part (its 32 keys) of its token's slot
+        if (sel) atomicAdd(dlogg + trow * topk + tp, dsum);
+      } else if (!cur) {  // this warp's part of d(log g) of the slot, summed at the end
         dsum = warp_sum(dsum);
         if (lane == 0) dl_s[j * NGW + warp] = dsum;
       }
@@ -362,7 +434,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_attn_bwd_tc(
     mbar_wait_data(&bars[B_MD], (nunits - 1) & 1, err);
     tc::fence_after_sync();
     named_bar_softmax();
-    for (int j = gtid; j < kk; j += 2 * 128) {  // d(log g): fixed-order sum over the warps
+    for (int j = gtid; j < (TOK ? 0 : kk); j += 2 * 128) {  // d(log g): fixed-order sum over the warps
       float a = 0.f;
 #pragma unroll
       for (int w = 0; w < NGW; ++w) a += dl_s[j * NGW + w];
@@ -409,19 +481,21 @@ __global__ void k_convert_tc(const float* __restrict__ src, TT* __restrict__ dst
     dst[i] = from_f<TT>(src[i]);
 }
 
-cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, int B, int Hq, int Hkv, int N,
-                               const float* lse, const int32_t* idx, const int32_t* cnt,
-                               const float* logg, int topk, float scale, void* dq, void* dk,
-                               void* dv, float* dlogg, void* ws, cudaStream_t st) {
+template <bool TOK>
+static cudaError_t launch_bwd_tc(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, int B, int Hq, int Hkv, int N,
+                                 const float* lse, const int32_t* idx, const int32_t* cnt,
+                                 const float* logg, int topk, float scale, void* dq, void* dk,
+                                 void* dv, float* dlogg, void* ws, cudaStream_t st) {
   const int T_ = (N + 63) / 64;
   if (B == 0 || T_ == 0) return cudaSuccess;
+  if (TOK && T_ - 1 > TOK_UMAX) return cudaErrorInvalidValue;
   const size_t nkv = (size_t)B * Hkv * N * D;
   float* dk_acc = static_cast<float*>(ws);
   float* dv_acc = dk_acc + nkv;
   cudaError_t e = cudaMemsetAsync(ws, 0, 2 * nkv * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(dlogg, 0, (size_t)B * Hkv * T_ * topk * sizeof(float), st);
+  e = cudaMemsetAsync(dlogg, 0, (size_t)B * Hkv * (TOK ? N : T_) * topk * sizeof(float), st);
   if (e != cudaSuccess) return e;
   CUtensorMap qm, km, vm, dom, dkm, dvm;
   if (!make_map(&qm, q, N, B * Hq) || !make_map(&km, k, N, B * Hkv) ||
@@ -429,10 +503,10 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
       !make_tma_map_f32_3d(&dkm, dk_acc, D, N, B * Hkv, 32, 32) ||
       !make_tma_map_f32_3d(&dvm, dv_acc, D, N, B * Hkv, 32, 32))
     return cudaErrorInvalidValue;
-  e = ensure_smem(k_attn_bwd_tc, SMEM_BYTES);
+  e = ensure_smem(k_attn_bwd_tc<TOK>, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(T_, Hkv * (Hq / Hkv / 2), B);
-  k_attn_bwd_tc<<<grid, BT_THREADS, SMEM_BYTES, st>>>(
+  k_attn_bwd_tc<TOK><<<grid, BT_THREADS, SMEM_BYTES, st>>>(
       qm, km, vm, dom, static_cast<const __nv_bfloat16*>(o),
       static_cast<const __nv_bfloat16*>(dout), dkm, dvm, lse, Hq, Hkv, N, idx, cnt, logg, topk,
       scale, static_cast<__nv_bfloat16*>(dq), dlogg);
@@ -442,6 +516,25 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
   k_convert_tc<__nv_bfloat16><<<cgrid, 256, 0, st>>>(dk_acc, static_cast<__nv_bfloat16*>(dk), nkv);
   k_convert_tc<__nv_bfloat16><<<cgrid, 256, 0, st>>>(dv_acc, static_cast<__nv_bfloat16*>(dv), nkv);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, int B, int Hq, int Hkv, int N,
+                               const float* lse, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* dq, void* dk,
+                               void* dv, float* dlogg, void* ws, cudaStream_t st) {
+  return launch_bwd_tc<false>(q, k, v, o, dout, B, Hq, Hkv, N, lse, idx, cnt, logg, topk, scale,
+                              dq, dk, dv, dlogg, ws, st);
+}
+
+cudaError_t launch_attn_bwd_tc_tokens(const void* q, const void* k, const void* v,
+                                      const void* o, const void* dout, int B, int Hq, int Hkv,
+                                      int N, const float* lse, const int32_t* idx,
+                                      const int32_t* cnt, const float* logg, int topk,
+                                      float scale, void* dq, void* dk, void* dv, float* dlogg,
+                                      void* ws, cudaStream_t st) {
+  return launch_bwd_tc<true>(q, k, v, o, dout, B, Hq, Hkv, N, lse, idx, cnt, logg, topk, scale,
+                             dq, dk, dv, dlogg, ws, st);
 }
 
 uint32_t* attn_bwd_tc_error_word() {

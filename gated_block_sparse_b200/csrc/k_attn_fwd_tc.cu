@@ -25,6 +25,16 @@
 // About 113 KB of shared memory and 256 TMEM columns per CTA, so two CTAs
 // share an SM and overlap one's softmax with the other's MMAs. Every wait is
 // bounded.
+//
+// Per-token selection (TOK = true; section 2.4: the fused kernel masks, per
+// query, the blocks below that query's gate threshold and skips a key tile no
+// query of the tile selected): every query token has its own selection row.
+// The CTA first builds the union of the blocks its 64 tokens selected
+// (ascending); the units are that union, then the current block. For a
+// history unit, row i adds its token's log g when its token selected the
+// unit's block and masks the whole unit (-inf) otherwise; each row finds that
+// by walking its own ascending list as the units advance. MMAs and softmax
+// are otherwise the same.
 #include <cuda.h>
 #include <math.h>
 
@@ -48,14 +58,17 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + Q_BYTES;
 constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+constexpr uint32_t OFF_UM = OFF_BAR + 128;  // per-token mode: union bitmask and its count
+constexpr uint32_t SMEM_BYTES = OFF_UM + 128;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy rescale threshold (log2 units)
+constexpr int TOK_UMAX = 512;         // history blocks of a query block at most (per-token mode)
 
 enum Bar { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 10, NBAR = 11 };
 
 }  // namespace
 
+template <bool TOK>
 __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
     const __grid_constant__ CUtensorMap vmap, int Hq, int Hkv, int N,
@@ -73,14 +86,54 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
   const int r = blockIdx.y / pairs, hp = blockIdx.y % pairs, b = blockIdx.z;
   const int h0 = r * G + 2 * hp;
   const size_t srow = ((size_t)b * Hkv + r) * T_ + t;
-  const int kk = min(max(cnt[srow], 0), topk);
-  const int nunits = kk + 1;  // kept history blocks, then the current block
-  const int32_t* idx_row = idx + srow * topk;
-  const float* logg_row = logg + srow * topk;
+  // per query block: kept history blocks; per token: the union of the
+  // tokens' blocks (built below); then the current block
+  int kk = TOK ? 0 : min(max(cnt[srow], 0), topk);
+  const int32_t* idx_row = idx + (TOK ? 0 : srow * topk);
+  const float* logg_row = logg + (TOK ? 0 : srow * topk);
   if ((smem_u32(sm) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
     if (tid == 0) atomicOr(err, kErrBadIndex);
     return;
   }
+  const size_t tok0 = ((size_t)b * Hkv + r) * N + 64 * t;  // first token row of the block
+  const int nr = min(64, N - 64 * t);
+  // the union as a bitmask over the t history blocks; each consumer walks it
+  // in ascending order with its own cursor (next_unit)
+  const uint32_t* umask_p = nullptr;
+  const int words = (t + 31) / 32;
+  if constexpr (TOK) {
+    uint32_t* umask = reinterpret_cast<uint32_t*>(sm + OFF_UM);  // TOK_UMAX / 32 words
+    int& ucnt = *reinterpret_cast<int*>(sm + OFF_UM + TOK_UMAX / 8);
+    umask_p = umask;
+    for (int w = tid; w < words; w += FT_THREADS) umask[w] = 0u;
+    __syncthreads();
+    for (int e = tid; e < nr * topk; e += FT_THREADS) {
+      const int i = e / topk, p = e - i * topk;
+      if (p < min(max(cnt[tok0 + i], 0), topk)) {
+        const int m = idx[(tok0 + i) * topk + p];
+        if (m >= 0 && m < t) atomicOr(&umask[m >> 5], 1u << (m & 31));
+        else atomicOr(err, kErrBadIndex);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {  // the number of units
+      int c = 0;
+      for (int w = lane; w < words; w += 32) c += __popc(umask[w]);
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) ucnt = c;
+    }
+    __syncthreads();
+    kk = ucnt;
+  }
+  // smallest selected block >= from (the union is ascending), -1 past the end
+  auto next_unit = [&](int from) -> int {
+    for (int w = from >> 5; w < words; ++w) {
+      const uint32_t word = umask_p[w] & (w == (from >> 5) ? (~0u << (from & 31)) : ~0u);
+      if (word) return w * 32 + __ffs(word) - 1;
+    }
+    return -1;
+  };
+  const int nunits = kk + 1;  // history units, then the current block
   if (tid == 0) {
     // S-empty (both buffers) and P-full take one arrival per softmax warp
     for (int i = 0; i < NBAR; ++i)
@@ -106,10 +159,12 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
         for (int h = 0; h < 2; ++h)
           tc::tma_load_3d(sm + OFF_Q + c * 16384 + h * 8192, &qmap, 64 * c, 64 * t,
                           b * Hq + h0 + h, &bars[B_Q]);
+      int ucur = -1;  // per-token: the previous unit's block
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
         if (j >= 2) mbar_wait_data(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
-        int blk = (j < kk) ? idx_row[j] : t;
+        if (TOK && j < kk) ucur = next_unit(ucur + 1);
+        int blk = (j < kk) ? (TOK ? ucur : idx_row[j]) : t;
         if (blk < 0 || blk >= t) {
           if (j < kk) atomicOr(err, kErrBadIndex);
           blk = t;
@@ -171,10 +226,28 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
     const float c1 = scale * LOG2E;
     float m = -1e30f, l = 0.f;
     unsigned char* prow = sm + OFF_P + row * 128;
+    // per-token selection: this row's own list (ascending), walked as the
+    // units advance; rows past the sequence end select nothing
+    const size_t trow = tok0 + (pos < N ? qr : 0);
+    const int tn = (TOK && pos < N) ? min(max(cnt[trow], 0), topk) : 0;
+    const int32_t* tidx = idx + trow * topk;
+    const float* tlog = logg + trow * topk;
+    int tp = 0, ucur = -1;
     for (int j = 0; j < nunits; ++j) {
       const int s = j & 1;
       const bool cur = (j == kk);
-      const float bias = cur ? 0.f : logg_row[j] * LOG2E;
+      float bias;
+      if constexpr (TOK) {
+        bias = 0.f;
+        if (!cur) {
+          ucur = next_unit(ucur + 1);
+          const int blk = ucur;
+          while (tp < tn && tidx[tp] < blk) ++tp;
+          bias = (tp < tn && tidx[tp] == blk) ? tlog[tp] * LOG2E : -INFINITY;
+        }
+      } else {
+        bias = cur ? 0.f : logg_row[j] * LOG2E;
+      }
       mbar_wait_data(&bars[B_SF + s], (j >> 1) & 1, err);
       tc::fence_after_sync();
       float z[64];
@@ -291,23 +364,38 @@ bool attn_fwd_tc_supported(int bf16, int d, int Hq, int Hkv) {
   return bf16 && d == 128 && G >= 2 && (G % 2) == 0;
 }
 
-cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq,
-                               int Hkv, int N, const int32_t* idx, const int32_t* cnt,
-                               const float* logg, int topk, float scale, void* o, float* lse,
-                               cudaStream_t st) {
+template <bool TOK>
+static cudaError_t launch_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq,
+                                 int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                                 const float* logg, int topk, float scale, void* o, float* lse,
+                                 cudaStream_t st) {
   const int T_ = (N + 63) / 64;
   if (B == 0 || T_ == 0) return cudaSuccess;
+  if (TOK && T_ - 1 > TOK_UMAX) return cudaErrorInvalidValue;
   CUtensorMap qm, km, vm;
   if (!make_map(&qm, q, N, B * Hq) || !make_map(&km, k, N, B * Hkv) ||
       !make_map(&vm, v, N, B * Hkv))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem(k_attn_fwd_tc, SMEM_BYTES);
+  cudaError_t e = ensure_smem(k_attn_fwd_tc<TOK>, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(T_, Hkv * (Hq / Hkv / 2), B);
-  k_attn_fwd_tc<<<grid, FT_THREADS, SMEM_BYTES, st>>>(qm, km, vm, Hq, Hkv, N, idx, cnt, logg,
-                                                       topk, scale,
-                                                       static_cast<__nv_bfloat16*>(o), lse);
+  k_attn_fwd_tc<TOK><<<grid, FT_THREADS, SMEM_BYTES, st>>>(
+      qm, km, vm, Hq, Hkv, N, idx, cnt, logg, topk, scale, static_cast<__nv_bfloat16*>(o), lse);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq,
+                               int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                               const float* logg, int topk, float scale, void* o, float* lse,
+                               cudaStream_t st) {
+  return launch_fwd_tc<false>(q, k, v, B, Hq, Hkv, N, idx, cnt, logg, topk, scale, o, lse, st);
+}
+
+cudaError_t launch_attn_fwd_tc_tokens(const void* q, const void* k, const void* v, int B, int Hq,
+                                      int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                                      const float* logg, int topk, float scale, void* o,
+                                      float* lse, cudaStream_t st) {
+  return launch_fwd_tc<true>(q, k, v, B, Hq, Hkv, N, idx, cnt, logg, topk, scale, o, lse, st);
 }
 
 uint32_t* attn_fwd_tc_error_word() {

@@ -144,6 +144,13 @@ cudaError_t launch_attn_fwd_tc(const void* q, const void* k, const void* v, int 
                                int Hkv, int N, const int32_t* idx, const int32_t* cnt,
                                const float* logg, int topk, float scale, void* o, float* lse,
                                cudaStream_t st);
+// The same kernel with per-token selection rows (idx/logg [B][Hkv][N][topk],
+// cnt [B][Hkv][N]): units are the union of the query block's tokens' blocks;
+// N <= 64 * 513.
+cudaError_t launch_attn_fwd_tc_tokens(const void* q, const void* k, const void* v, int B, int Hq,
+                                      int Hkv, int N, const int32_t* idx, const int32_t* cnt,
+                                      const float* logg, int topk, float scale, void* o,
+                                      float* lse, cudaStream_t st);
 uint32_t* attn_fwd_tc_error_word();
 // Tensor-core backward (same support as the forward); ws as attn_bwd_simt.
 cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, const void* o,
@@ -151,6 +158,14 @@ cudaError_t launch_attn_bwd_tc(const void* q, const void* k, const void* v, cons
                                const float* lse, const int32_t* idx, const int32_t* cnt,
                                const float* logg, int topk, float scale, void* dq, void* dk,
                                void* dv, float* dlogg, void* ws, cudaStream_t st);
+// The same kernel with per-token selection rows (layouts as the per-token
+// forward; dlogg [B][Hkv][N][topk]); ws as launch_attn_bwd_tc.
+cudaError_t launch_attn_bwd_tc_tokens(const void* q, const void* k, const void* v,
+                                      const void* o, const void* dout, int B, int Hq, int Hkv,
+                                      int N, const float* lse, const int32_t* idx,
+                                      const int32_t* cnt, const float* logg, int topk,
+                                      float scale, void* dq, void* dk, void* dv, float* dlogg,
+                                      void* ws, cudaStream_t st);
 uint32_t* attn_bwd_tc_error_word();
 
 // Self-test of the bounded wait (k_status.cu): one warp waits on a barrier

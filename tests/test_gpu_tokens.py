@@ -33,8 +33,9 @@ def _np(t):
 
 
 @pytest.mark.parametrize("dtype,Hq,Hkv,N,d,topk,seed", [
-    ("f32", 2, 2, 640, 64, 2, 31),
-    ("bf16", 8, 2, 1000, 128, 5, 32),
+    ("f32", 2, 2, 640, 64, 2, 31),       # CUDA-core kernels
+    ("bf16", 8, 2, 1000, 128, 5, 32),    # tensor-core kernels (bf16, d = 128, even group)
+    ("bf16", 4, 2, 2200, 128, 7, 37),    # tensor-core kernels, unions over two mask words
 ])
 def test_tokens_selection_forward_backward(dtype, Hq, Hkv, N, d, topk, seed):
     x = inputs.gen_prefill(1, Hq, Hkv, N, d, dtype, seed=seed, plant="ramp", q_shift=4.0)
@@ -68,24 +69,46 @@ def test_tokens_selection_forward_backward(dtype, Hq, Hkv, N, d, topk, seed):
     assert st == 0, msg
 
 
-def test_tokens_reduce_to_block_rows_when_rows_agree():
+@pytest.mark.parametrize("dtype,d,Hq,Hkv", [("f32", 64, 2, 1), ("bf16", 128, 4, 2)])
+def test_tokens_reduce_to_block_rows_when_rows_agree(dtype, d, Hq, Hkv):
     """Rows of a query block with equal queries select alike: the per-token
-    forward equals the per-block forward on the same (repeated) selection."""
-    N, d, Hq, Hkv, topk = 512, 64, 2, 1, 2
-    x = inputs.gen_prefill(1, Hq, Hkv, N, d, "f32", seed=34, plant="ramp", q_shift=4.0)
+    forward and backward equal the per-block ones on the same (repeated)
+    selection (fp32: CUDA-core kernels, within rounding; bf16, d = 128: the
+    tensor-core kernels, whose per-token units are then the block's own kept
+    blocks, bit for bit)."""
+    N, topk = 512, 2
+    x = inputs.gen_prefill(1, Hq, Hkv, N, d, dtype, seed=34, plant="ramp", q_shift=4.0)
     q = x["q"].clone()
     for t in range(N // 64):
         q[:, :, t * 64:(t + 1) * 64] = q[:, :, t * 64:t * 64 + 1]
-    q, k, v = q.to(DEV), x["k"].to(DEV), x["v"].to(DEV)
+    q, k, v, do = q.to(DEV), x["k"].to(DEV), x["v"].to(DEV), x["do"].to(DEV)
     ks = sas.sas_block_summary(k)
     bi, bc, bl = sas.sas_select(q, ks, Hkv, topk, "prefill")
     ti, tc, tl = sas.sas_select_tokens(q, ks, Hkv, topk)
-    ob, lb = sas.sas_attn_fwd(q, k, v, bi, bc, bl)
-    ot, lt = sas.sas_attn_fwd_tokens(q, k, v, ti, tc, tl)
     torch.cuda.synchronize()
     for i in range(N):
         assert torch.equal(ti[:, :, i], bi[:, :, i // 64])
-    assert float((ob - ot).abs().max()) < 1e-5 and float((lb - lt).abs().max()) < 1e-5
+    # the attention calls get the block rows repeated for their 64 tokens, so
+    # both see the same gates
+    ti, tc, tl = (x_.repeat_interleave(64, dim=2).contiguous() for x_ in (bi, bc, bl))
+    ob, lb = sas.sas_attn_fwd(q, k, v, bi, bc, bl)
+    ot, lt = sas.sas_attn_fwd_tokens(q, k, v, ti, tc, tl)
+    gb = sas.sas_attn_bwd(q, k, v, ob, do, lb, bi, bc, bl)
+    gt = sas.sas_attn_bwd_tokens(q, k, v, ob, do, lb, ti, tc, tl)
+    torch.cuda.synchronize()
+    if dtype == "bf16":  # dk, dv add fp32 partials in L2 in any order: half an ulp apart
+        assert torch.equal(ob, ot) and torch.equal(lb, lt) and torch.equal(gb[0], gt[0])
+        for a, b in zip(gb[1:3], gt[1:3]):
+            assert excess(_np(a), _np(b), 1e-6, True) <= 0
+    else:
+        assert float((ob - ot).abs().max()) < 1e-5 and float((lb - lt).abs().max()) < 1e-5
+        for a, b in zip(gb[:3], gt[:3]):
+            assert float((a - b).abs().max()) < 1e-5
+    # the block's dlogg slot is the sum of its tokens' slots
+    dl_tok = gt[3].view(1, Hkv, N // 64, 64, topk).sum(dim=3)
+    assert float((dl_tok - gb[3]).abs().max()) < 1e-3 * float(gb[3].abs().max()) + 1e-4
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg
 
 
 @pytest.mark.parametrize("dtype,Hq,Hkv,N,d,topk,seed", [

@@ -59,7 +59,7 @@ DEFAULT_WARMUP = {"c1": 10, "c2": 1000, "c3": 3, "c4": 100, "c5": 500}
 # (record name, config, options) of the default run; the first is the headline
 ALL_RECORDS = (("c5", "c5", {}), ("c5_bf16_summaries", "c5", {"summary": "bf16"}),
                ("c4", "c4", {}), ("c2", "c2", {}), ("c2_paged", "c2", {"paged": True}),
-               ("c3", "c3", {}))
+               ("c3", "c3", {}), ("c3_tokens", "c3", {"tokens": True}))
 
 
 # ----------------------------------------------------------------- helpers
@@ -505,7 +505,20 @@ def prefill_flops(idx_cnt, N: int, Hq: int, Hkv: int, d: int):
     return 4 * d * pairs, 10 * d * pairs
 
 
-def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=None) -> dict:
+def prefill_flops_tokens(cnt_tok, N: int, Hq: int, Hkv: int, d: int):
+    """Algorithmic FLOPs of one forward and one backward with per-token
+    selection rows: every token i of every head sees 64 keys of each of its
+    cnt_i kept blocks and the i % 64 + 1 causal keys of its own block."""
+    import numpy as np
+    cnt = np.asarray(cnt_tok)  # [B][Hkv][N]
+    G = Hq // Hkv
+    cur = (np.arange(N) % 64 + 1).astype(np.int64)
+    pairs = int(G * (64 * cnt.astype(np.int64).sum() + cnt.shape[0] * cnt.shape[1] * cur.sum()))
+    return 4 * d * pairs, 10 * d * pairs
+
+
+def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=None,
+                       tokens: bool = False) -> dict:
     import torch
 
     from gated_block_sparse_b200 import dist as D
@@ -517,24 +530,42 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
     topk, Hkv = c["topk"], c["Hkv"]
     B, Hq, N, d = q.shape
     ks = sas.sas_block_summary(k)
-    idx, cnt, logg = sas.sas_select(q, ks, Hkv, topk, "prefill")
-    o, lse = sas.sas_attn_fwd(q, k, v, idx, cnt, logg)
-    grads = sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg)
-    torch.cuda.synchronize()
-    f_fwd, f_bwd = prefill_flops(cnt.cpu().numpy(), N, Hq, Hkv, d)
     lib = sas.load_library()
     dt = 1 if c["dtype"] == "bf16" else 0
+    if tokens:  # per-token selection rows (each query token its own block set)
+        idx, cnt, logg = sas.sas_select_tokens(q, ks, Hkv, topk)
+        o, lse = sas.sas_attn_fwd_tokens(q, k, v, idx, cnt, logg)
+        bwd_ws = torch.empty(max(16, lib.sas_attn_bwd_tokens_workspace_size(B, Hq, Hkv, N, d)),
+                             dtype=torch.uint8, device=dev)
+        grads = sas.sas_attn_bwd_tokens(q, k, v, o, do, lse, idx, cnt, logg, ws=bwd_ws)
+        sbw_ws = torch.empty(max(16, lib.sas_select_bwd_tokens_workspace_size(B, Hq, Hkv, N, d)),
+                             dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        f_fwd, f_bwd = prefill_flops_tokens(cnt.cpu().numpy(), N, Hq, Hkv, d)
+    else:
+        idx, cnt, logg = sas.sas_select(q, ks, Hkv, topk, "prefill")
+        o, lse = sas.sas_attn_fwd(q, k, v, idx, cnt, logg)
+        grads = sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg)
+        torch.cuda.synchronize()
+        f_fwd, f_bwd = prefill_flops(cnt.cpu().numpy(), N, Hq, Hkv, d)
+        bwd_ws = torch.empty(max(16, lib.sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt)),
+                             dtype=torch.uint8, device=dev)
+        sbw_ws = torch.empty(max(16, lib.sas_select_bwd_workspace_size(B, Hq, Hkv, N, d)),
+                             dtype=torch.uint8, device=dev)
     sel_ws = torch.empty(max(16, lib.sas_select_workspace_size(B, Hq, Hkv, N, d, topk, 0)),
-                         dtype=torch.uint8, device=dev)
-    bwd_ws = torch.empty(max(16, lib.sas_attn_bwd_workspace_size(B, Hq, Hkv, N, d, topk, dt)),
-                         dtype=torch.uint8, device=dev)
-    sbw_ws = torch.empty(max(16, lib.sas_select_bwd_workspace_size(B, Hq, Hkv, N, d)),
                          dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(dev)
     clocks = clock_sampler(dev.index if dev.index is not None else 0)
 
     def step(i):
         sas.sas_block_summary(k, out=ks)
+        if tokens:
+            sas.sas_select_tokens(q, ks, Hkv, topk, out=(idx, cnt, logg))
+            sas.sas_attn_fwd_tokens(q, k, v, idx, cnt, logg, out=(o, lse))
+            sas.sas_attn_bwd_tokens(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+            sas.sas_select_bwd_tokens(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1],
+                                      ws=sbw_ws)
+            return
         sas.sas_select(q, ks, Hkv, topk, "prefill", out=(idx, cnt, logg), ws=sel_ws)
         sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
         sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
@@ -544,13 +575,23 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
     ms, clk = timed_graphs(step, K, W, world, stream, chunk=8, clocks=clocks)
 
     def fwd_step(i):
-        sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
+        if tokens:
+            sas.sas_attn_fwd_tokens(q, k, v, idx, cnt, logg, out=(o, lse))
+        else:
+            sas.sas_attn_fwd(q, k, v, idx, cnt, logg, out=(o, lse))
 
     def bwd_step(i):
-        sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+        if tokens:
+            sas.sas_attn_bwd_tokens(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
+        else:
+            sas.sas_attn_bwd(q, k, v, o, do, lse, idx, cnt, logg, out=grads, ws=bwd_ws)
 
     def sbw_step(i):
-        sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
+        if tokens:
+            sas.sas_select_bwd_tokens(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1],
+                                      ws=sbw_ws)
+        else:
+            sas.sas_select_bwd(q, ks, Hkv, idx, cnt, grads[3], grads[0], grads[1], ws=sbw_ws)
 
     Kp = max(3, K)
     ms_f, _ = timed_graphs(fwd_step, Kp, 2, world, stream, chunk=8)
@@ -625,7 +666,9 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
         "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if c["dtype"] == "bf16" else "f32", "data": "synthetic (seeded N(0,1), planted)",
-        "config": {"workload": f"{name}: {inputs.DESCRIPTIONS[name]}", "batch": B, "seq_len": N,
+        "config": {"workload": f"{name}: {inputs.DESCRIPTIONS[name]}"
+                               + (", per-token selection rows" if tokens else ""),
+                   "batch": B, "seq_len": N,
                    "q_heads": Hq, "kv_heads": Hkv, "head_dim": d, "topk": topk,
                    "flops_fwd": f_fwd, "flops_bwd": f_bwd, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (q+k+v+dO = {h2d / 1e6:.0f} MB)"},
@@ -639,9 +682,11 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
                                       "copy_out": round(ms_out / E, 4),
                                       "step": round(ms / K, 4)},
                 "steps": E},
-        # summary, query means, selection, forward, backward, 2 conversions,
-        # selector backward (query means, rows, columns)
-        "gpu_launches": 10 * K,
+        # block rows: summary, query means, selection, forward, backward, 2
+        # conversions, selector backward (query means, rows, columns); token
+        # rows: summary, selection, forward, backward, 2 conversions, selector
+        # backward (rows, spread)
+        "gpu_launches": (8 if tokens else 10) * K,
         "clocks": clk,
     }
     del q, k, v, do, grads, o, lse
@@ -805,6 +850,41 @@ def cpu_baseline_prefill(name: str, seconds: float, host=None, all_cores: bool =
     return res
 
 
+def cpu_baseline_prefill_tokens(name: str, seconds: float, host=None) -> dict:
+    """The per-token oracle (selection, forward, backward) on a prefix of the
+    workload: the first n tokens of every head (n grows by 64-token blocks
+    while a pass stays within the time), so the sample keeps the workload's
+    shapes and selection rule at shorter history."""
+    from gated_block_sparse_b200 import inputs
+    from oracle import sas_oracle as O
+    c = inputs.CONFIGS[name]
+    h = inputs.gen_config(name) if host is None else host
+    d, Hkv, topk = c["d"], c["Hkv"], c["topk"]
+    G = c["Hq"] // Hkv
+    n, flops, el, passes = 256, 0, 0.0, 0
+    with _one_thread():
+        while True:
+            x = {k_: h[k_][:, :, :n] for k_ in ("q", "k", "v", "do")}
+            t0 = time.perf_counter()
+            idx, cnt, logg, _ = O.select_prefill_tokens(x["q"], O.block_summary(x["k"]), Hkv, topk)
+            O.attn_fwd_tokens(x["q"], x["k"], x["v"], idx, cnt, logg)
+            O.attn_bwd_tokens(x["q"], x["k"], x["v"], x["do"], idx, cnt, logg)
+            dt_ = time.perf_counter() - t0
+            cur = sum(i % 64 + 1 for i in range(n))
+            flops += 14 * d * G * (64 * int(cnt.sum()) + Hkv * cur)
+            el += dt_
+            passes += 1
+            if el >= seconds or n >= c["N"]:
+                break
+            n = min(c["N"], 2 * n)
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "seconds": round(el, 2),
+            "sample": f"{passes} pass(es) over prefixes of {name}, from its first 256 tokens "
+                      f"(doubling) to its first {n} tokens of every head: per-token selection, "
+                      "forward and backward, fp64 numpy oracle, 1 BLAS thread",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+
+
 # ----------------------------------------------------------------- main
 def run_one(name: str, cfg: str, opts: dict, K: int, W: int, world: int, rank: int, local: int,
             cpu_seconds: float, hosts: dict, baselines: dict) -> dict:
@@ -822,6 +902,11 @@ def run_one(name: str, cfg: str, opts: dict, K: int, W: int, world: int, rank: i
             if key not in baselines:
                 baselines[key] = cpu_baseline_decode(w, cpu_seconds)
             rec["cpu_baseline"] = baselines[key]
+    elif opts.get("tokens"):
+        rec = bench_prefill_ours(cfg, K, W, world, local, host=hosts[cfg], tokens=True)
+        if rank == 0:
+            rec["cpu_baseline"] = cpu_baseline_prefill_tokens(cfg, cpu_seconds, host=hosts[cfg])
+        rec["config"]["variant"] = "per-token selection (sas_select_tokens, *_tokens)"
     else:
         rec = bench_prefill_ours(cfg, K, W, world, local, host=hosts[cfg])
         if rank == 0:
@@ -847,6 +932,8 @@ def main():
                     help="decode: read the caches through 64-token pages (sas_decode_paged)")
     ap.add_argument("--summary", default="f32", choices=["f32", "bf16"],
                     help="decode: store block summaries in fp32 or bf16 (sas_decode_ex)")
+    ap.add_argument("--tokens", action="store_true",
+                    help="prefill: per-token selection rows (sas_select_tokens, *_tokens)")
     ap.add_argument("--layers", type=int, default=0,
                     help="decode: number of rotated layer copies (default: enough for 3x L2)")
     args = ap.parse_args()
@@ -857,7 +944,8 @@ def main():
     if args.config == "all":
         plan = ALL_RECORDS
     else:
-        opts = {"paged": args.paged, "summary": args.summary, "layers": args.layers}
+        opts = {"paged": args.paged, "summary": args.summary, "layers": args.layers,
+                "tokens": args.tokens}
         plan = ((args.config, args.config, opts),)
 
     if args.impl == "reference":

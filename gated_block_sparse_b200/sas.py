@@ -305,45 +305,51 @@ def sas_block_summary_last(k, lens, ksum, block_table=None, npages: int = 0, str
     return ksum
 
 
-def sas_select_tokens(q, ksum, Hkv: int, topk: int, scale: float = 0.0, stream=None):
+def sas_select_tokens(q, ksum, Hkv: int, topk: int, scale: float = 0.0, out=None, stream=None):
     """Per-token selection rows: idx/logg [B][Hkv][N][topk], cnt [B][Hkv][N]."""
     lib = load_library()
     B, Hq, N, d = q.shape
-    idx = torch.empty((B, Hkv, N, topk), dtype=torch.int32, device=q.device)
-    cnt = torch.empty((B, Hkv, N), dtype=torch.int32, device=q.device)
-    logg = torch.empty((B, Hkv, N, topk), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = (torch.empty((B, Hkv, N, topk), dtype=torch.int32, device=q.device),
+               torch.empty((B, Hkv, N), dtype=torch.int32, device=q.device),
+               torch.empty((B, Hkv, N, topk), dtype=torch.float32, device=q.device))
+    idx, cnt, logg = out
     _check("sas_select_tokens", lib.sas_select_tokens(
         _ptr(q), _dt(q), _ptr(ksum), B, Hq, Hkv, N, d, topk, float(scale), _ptr(idx), _ptr(cnt),
         _ptr(logg), _stream(stream)))
     return idx, cnt, logg
 
 
-def sas_attn_fwd_tokens(q, k, v, idx, cnt, logg, scale: float = 0.0, stream=None):
+def sas_attn_fwd_tokens(q, k, v, idx, cnt, logg, scale: float = 0.0, out=None, stream=None):
     """Forward with per-token selection rows; returns (o, lse)."""
     lib = load_library()
     B, Hq, N, d = q.shape
     Hkv, topk = k.shape[1], idx.shape[-1]
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty((B, Hq, N), dtype=torch.float32, device=q.device))
+    o, lse = out
     _check("sas_attn_fwd_tokens", lib.sas_attn_fwd_tokens(
         _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, N, d, _ptr(idx), _ptr(cnt), _ptr(logg),
         topk, float(scale), _ptr(o), _ptr(lse), _stream(stream)))
     return o, lse
 
 
-def sas_attn_bwd_tokens(q, k, v, o, do, lse, idx, cnt, logg, scale: float = 0.0, stream=None):
+def sas_attn_bwd_tokens(q, k, v, o, do, lse, idx, cnt, logg, scale: float = 0.0, out=None,
+                        ws=None, stream=None):
     """Backward with per-token selection rows; returns (dq, dk, dv, dlogg)."""
     lib = load_library()
     B, Hq, N, d = q.shape
     Hkv, topk = k.shape[1], idx.shape[-1]
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dlogg = torch.empty((B, Hkv, N, topk), dtype=torch.float32, device=q.device)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+               torch.empty((B, Hkv, N, topk), dtype=torch.float32, device=q.device))
+    dq, dk, dv, dlogg = out
     nws = lib.sas_attn_bwd_tokens_workspace_size(B, Hq, Hkv, N, d)
-    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    w = _ws(nws, q.device, ws)
     _check("sas_attn_bwd_tokens", lib.sas_attn_bwd_tokens(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _dt(q), B, Hq, Hkv, N, d, _ptr(lse),
         _ptr(idx), _ptr(cnt), _ptr(logg), topk, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(dlogg), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(dlogg), _ptr(w), w.numel(), _stream(stream)))
     return dq, dk, dv, dlogg
 
 

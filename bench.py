@@ -615,7 +615,8 @@ def bench_prefill_ours(name: str, K: int, W: int, world: int, local: int, host=N
     ach = kf / kt / 1e12
     roof = {"bound": bound, "kernel": kern, "achieved": round(ach, 2), "peak": round(peak, 1),
             "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-            "traffic": recorded_traffic(kern, srcs[i], name), "peak_source": psrc,
+            "traffic": recorded_traffic(kern, srcs[i], name + ("_tokens" if tokens else "")),
+            "peak_source": psrc,
             "algorithmic_flops_per_launch": kf, "launch_ms": round(kt * 1e3, 4),
             "fwd_ms": round(tf * 1e3, 4), "bwd_ms": round(tb * 1e3, 4),
             "fwd_tflops": round(f_fwd / tf / 1e12, 2), "bwd_tflops": round(f_bwd / tb / 1e12, 2),

@@ -31,7 +31,12 @@
 //      the summary ring.
 //      Each warp takes 8 keys of every unit and keeps its own online-softmax
 //      state (m, l, acc) for every head of the group, so no CTA-wide barrier
-//      runs per unit;
+//      runs per unit. bf16 caches: the K/V tiles arrive by TMA as 64-column
+//      boxes with the 128-byte swizzle, and q.k and p.v are warp MMAs
+//      (mma.sync m16n8k16 / m16n8k8, fp32 accumulation) with the group's
+//      heads as the rows of the A operand and P reused as the A operand of
+//      p.v in the layout the q.k accumulator leaves it; fp32 caches: CUDA
+//      cores;
 //   5. folds the warp states into one per head and stores head h's state
 //      into CTA h (remote stores on CTA h's mbarrier); CTA h < G combines the
 //      CS states (exact LSE rescaling) and writes o.
@@ -41,11 +46,15 @@
 // keeps every CTA resident until all stores into it are done. No global
 // scratch, atomics or memsets; every wait is bounded.
 #include <cooperative_groups.h>
+#include <cuda.h>
 #include <float.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -65,7 +74,7 @@ constexpr size_t FD_SMEM_MAX = 226 * 1024; // dynamic shared memory per CTA at m
 constexpr unsigned FULL = 0xffffffffu;
 
 struct FdSmem {  // byte offsets into dynamic shared memory
-  size_t u, q, qbar, sc, mine, slen, stage, sstat, fin, cst, cml, zp, bars, total;
+  size_t u, q, qf, qbar, sc, mine, slen, stage, sstat, fin, cst, cml, zp, bars, total;
   size_t wl, wb, samp, surv;                  // list scratch inside region u, after K/V slot 0
   int nkv;                                    // K/V ring slots held by region u
   int subc;                                   // summaries per ring slot
@@ -98,6 +107,7 @@ __host__ __device__ inline FdSmem fd_layout(int D, int G, int es, int per, int k
   size_t o = 0;
   L.u = o; o += fd_al(ub);
   L.q = o; o += fd_al((size_t)G * D * 4);
+  L.qf = o; o += fd_al((size_t)(D / 16) * 2 * 32 * 4);  // q as warp-MMA A fragments (bf16)
   L.qbar = o; o += fd_al((size_t)D * 4);
   L.sc = o; o += fd_al((size_t)(per > 0 ? per : 1) * 4);
   L.mine = o; o += fd_al((size_t)kq * 8);
@@ -198,6 +208,44 @@ __device__ __forceinline__ float transpose_sum(float (&v)[NV], int lane) {
   return v[0];
 }
 
+// Warp MMAs on bf16 operands with fp32 accumulation (c += a b).
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// m16n8k8 with the A operand's rows 8..15 zero: c2, c3 (rows 8..15 of the
+// result) pass through unchanged, so every call can share one zero pair.
+__device__ __forceinline__ void mma_1688(float (&c)[2], float& z2, float& z3, uint32_t a0,
+                                         uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(z2), "+f"(z3)
+      : "r"(a0), "r"(0u), "r"(b0));
+}
+// Four transposed 8 x 8 bf16 matrices; lane l gives the address of row l % 8
+// of matrix l / 8.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Byte offset of element (row, col) of a bf16 [64][D] tile stored as
+// 64-column boxes of [64 rows][128 B] with the 128-byte swizzle (16-byte
+// chunk c of row r at chunk c ^ (r % 8)), as the tensor-map loads leave it.
+__device__ __forceinline__ uint32_t sw_off(int row, int col) {
+  return (uint32_t)((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                    (col & 7) * 2);
+}
+
 // Combines two (max, sum exp) pairs; an empty pair is (-FLT_MAX, 0).
 __device__ __forceinline__ void ms_merge(float& m, float& s, float m2, float s2) {
   const float M = fmaxf(m, m2);
@@ -217,12 +265,15 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
     const S* __restrict__ ksum, int Hkv, int Lmax, const int32_t* __restrict__ lens, int topk,
     int gated, float scale, int per_max, int ub_min, T* __restrict__ o,
-    int32_t* __restrict__ idx_out, const int32_t* __restrict__ bt, int npages) {
+    int32_t* __restrict__ idx_out, const int32_t* __restrict__ bt, int npages,
+    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+  // bf16 caches: K/V tiles by TMA (swizzled) and warp MMAs; fp32: bulk copies, CUDA cores
+  constexpr bool TMA_KV = std::is_same<T, __nv_bfloat16>::value;
   constexpr int TILE = SAS_BLOCK * D;
   constexpr int VEC = Vec16<T>::N;     // elements per 16-byte vector
   constexpr int CPL = D / 32;          // output columns per lane
   constexpr int PER = D / 32;          // summary elements per lane
-  extern __shared__ __align__(128) unsigned char sm[];
+  extern __shared__ __align__(1024) unsigned char sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = (int)cluster.num_blocks();
   const int crank = (int)cluster.block_rank();
@@ -267,6 +318,14 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   // scheduled now (it waits for this grid's completion before its own first
   // global read), and this grid reads nothing the previous one may still
   // write before that grid has completed.
+  if (TMA_KV && (smem_u32(sm) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
+    if (tid == 0) atomicOr(&g_decode_fused_err, kErrBadIndex);
+    return;  // every CTA of the launch sees the same alignment: no cluster barrier is left waiting
+  }
+  if (TMA_KV && tid == 0) {
+    tc::prefetch_map(&kmap);
+    tc::prefetch_map(&vmap);
+  }
   grid_dep_launch();
   grid_dep_wait();
   // the group's queries and the sequence length first: both loads in flight together
@@ -305,6 +364,29 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   auto kv_tile = [&](const T* base, int blk) -> const T* {
     if constexpr (PAGED) return base + ((size_t)page_of(blk) * Hkv + r) * TILE;
     else return base + kvrow + (size_t)blk * TILE;
+  };
+  // K and V of logical block blk into a K/V slot (2 * TILE elements), both
+  // completing on `bar`: TMA boxes (bf16) or two bulk copies (fp32)
+  auto issue_kv = [&](unsigned char* dst, int blk, uint64_t* bar) {
+    mbar_arrive_expect_tx(bar, (uint32_t)(2 * TILE * sizeof(T)));
+    if constexpr (TMA_KV) {
+      int plane, row0;
+      if constexpr (PAGED) {
+        plane = page_of(blk) * Hkv + r;
+        row0 = 0;
+      } else {
+        plane = b * Hkv + r;
+        row0 = SAS_BLOCK * blk;
+      }
+#pragma unroll
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tc::tma_load_3d(dst + bx * 8192, &kmap, 64 * bx, row0, plane, bar);
+        tc::tma_load_3d(dst + TILE * sizeof(T) + bx * 8192, &vmap, 64 * bx, row0, plane, bar);
+      }
+    } else {
+      bulk_g2s(dst, kv_tile(kc, blk), TILE * sizeof(T), bar);
+      bulk_g2s(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), bar);
+    }
   };
   // summaries [first, first + cnt) of this CTA's range into ring slot `slot`:
   // one bulk copy (contiguous), or one row copy per lane of warp 0 (paged)
@@ -446,11 +528,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
   // The ring is consumed (the scan's last barrier): K/V slot 0 takes the
   // current block, unit 0 of this CTA's order when it owns it; the copy
   // overlaps the selection below.
-  if (tid == 0 && own_cur) {
-    mbar_arrive_expect_tx(&full[0], (uint32_t)(2 * TILE * sizeof(T)));
-    bulk_g2s(U, kv_tile(kc, t), TILE * sizeof(T), &full[0]);
-    bulk_g2s(U + TILE * sizeof(T), kv_tile(vc, t), TILE * sizeof(T), &full[0]);
-  }
+  if (tid == 0 && own_cur) issue_kv(U, t, &full[0]);
 
   // ---- 2. this range's (max, sum exp) and best-first list
   {
@@ -614,10 +692,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       blk = t;
     }
     const int slot = i % NKV;
-    unsigned char* dst = U + (size_t)slot * kvslot;
-    mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * TILE * sizeof(T)));
-    bulk_g2s(dst, kv_tile(kc, blk), TILE * sizeof(T), &full[slot]);
-    bulk_g2s(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), &full[slot]);
+    issue_kv(U + (size_t)slot * kvslot, blk, &full[slot]);
   };
   if (tid == 0) {
     fence_proxy_async_smem();  // the list scratch written above becomes K/V slots
@@ -636,129 +711,229 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       idx_out[row * topk + pos] = mi;
     }
   }
-  // Each warp takes 8 keys of every unit (keys wid*8 .. wid*8+7) and keeps
-  // its own online-softmax state per head. Lane l holds columns
-  // [l*CPL, l*CPL + CPL) of q and of the accumulators of every head. The
-  // q.k partial sums of the warp's 8 keys x GP heads (one pass per group of
-  // at most 4 heads) are summed over the lanes by a transposing reduction:
-  // each shuffle stage halves the values a lane carries, so 8*GP sums cost
-  // fewer than 8*GP shuffles and lane l ends with the sum of key l/4 and
-  // head (l%4)/(4/GP) of the pass (lanes holding the same pair agree).
-  constexpr int GP = G < 4 ? G : 4;  // heads per pass
-  constexpr int HP = G / GP;         // passes
-  constexpr int NV = 8 * GP;         // partial sums per lane per pass
-  float qr[G][CPL], acc[G][CPL], m_p[HP], l_p[HP];
+  float* wst = reinterpret_cast<float*>(U);  // [warp][head][D] acc, once the units are done
+  if constexpr (TMA_KV) {
+    // Warp MMAs. Per unit, warp w takes keys 8w .. 8w+7: S = Q K^T as one
+    // m16n8k16 chain over d (A: the group's heads as rows 0..G-1 of 16, q in
+    // registers; B: K rows from the swizzled tile), leaving lane (g, t) =
+    // (lane / 4, lane % 4) with head g's scores of keys 8w + 2t and 8w + 2t + 1;
+    // the online softmax per head reduces over the four lanes of a head; P
+    // in bf16 is then the A operand of O += P V (m16n8k8 over the 8 keys, V
+    // by transposing ldmatrix), one per 8-column tile of O.
+    constexpr int KS = D / 16;  // k-steps of q.k
+    constexpr int NT = D / 8;   // 8-column tiles of O
+    const int g = lane >> 2, t4 = lane & 3;
+    // q as the A fragments of every k-step (lane-major in shared memory, read
+    // back conflict-free each unit): head g's columns 16ks + 2t4 (+1) and
+    // 16ks + 2t4 + 8 (+9); rows g >= G are zero
+    uint32_t* qf = reinterpret_cast<uint32_t*>(sm + L.qf);
+    if (wid == 0) {
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      qr[h][c] = q_s[h * D + lane * CPL + c];
-      acc[h][c] = 0.f;
-    }
-  }
-#pragma unroll
-  for (int p = 0; p < HP; ++p) {
-    m_p[p] = -INFINITY;
-    l_p[p] = 0.f;
-  }
-  const int jj = lane >> 2;                                  // this lane's key of the 8
-  const int hp = (lane & 3) / (4 / GP);                      // and head within a pass
-  const bool uniq = (lane & (4 / GP - 1)) == 0;              // first lane holding the pair
-  float* pw = zp + wid * (2 * 8 * G);                        // [8 keys][G] p of this warp
-  float* aw = pw + 8 * G;                                    // [G] rescale factors
-  for (int i = 0; i < nu; ++i) {
-    const int slot = i % NKV;
-    const int u = unit_of(i);
-    const bool cur = (u == kk);
-    const float bias = (!cur && gated) ? key_score(fin[u]) - lse : 0.f;
-    mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
-    const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot) + (size_t)wid * 8 * D;
-    const T* vt = kt + TILE;
-    const bool masked = cur && (wid * 8 + jj >= ncur);
-#pragma unroll
-    for (int p = 0; p < HP; ++p) {
-      float part[NV];
-#pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8) {
-        float kv[CPL];
-        loadn<CPL>(kt + (size_t)k8 * D + lane * CPL, kv);
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float a = 0.f;
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) a = fmaf(qr[p * GP + g][c], kv[c], a);
-          part[k8 * GP + g] = a;
-        }
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c = ks * 16 + 2 * t4;
+        qf[(2 * ks) * 32 + lane] = g < G ? pack_bf16(q_s[g * D + c], q_s[g * D + c + 1]) : 0u;
+        qf[(2 * ks + 1) * 32 + lane] =
+            g < G ? pack_bf16(q_s[g * D + c + 8], q_s[g * D + c + 9]) : 0u;
       }
-      const float dot = transpose_sum<NV>(part, lane);
-      const float z = masked ? -INFINITY : dot * scale + bias;
-      float zmax = z;
-      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 4));
-      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 8));
-      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 16));
-      const float mn = fmaxf(m_p[p], zmax);
-      float pr, alpha;
+    }
+    __syncthreads();
+    float acc[NT][2];  // O[head g][8n + 2t4], O[g][8n + 2t4 + 1]
+    float z2 = 0.f, z3 = 0.f;  // rows 8..15 of every O tile: always zero
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = 0.f;
+    float m_h = -INFINITY, l_h = 0.f;  // head g's running max and sum (this warp)
+    const int key0 = wid * 8 + 2 * t4;  // this lane's two keys of the unit
+    for (int i = 0; i < nu; ++i) {
+      const int slot = i % NKV;
+      const int u = unit_of(i);
+      const bool cur = (u == kk);
+      const float bias = (!cur && gated) ? key_score(fin[u]) - lse : 0.f;
+      mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
+      const uint32_t kt = smem_u32(U + (size_t)slot * kvslot);
+      const uint32_t vt = kt + TILE * sizeof(T);
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t b0, b1;
+        const int c = ks * 16 + 2 * t4;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b0) : "r"(kt + sw_off(wid * 8 + g, c)));
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(b1) : "r"(kt + sw_off(wid * 8 + g, c + 8)));
+        mma_16816(sc, qf[(2 * ks) * 32 + lane], qf[(2 * ks + 1) * 32 + lane], b0, b1);
+      }
+      const float z0 = (cur && key0 >= ncur) ? -INFINITY : sc[0] * scale + bias;
+      const float z1 = (cur && key0 + 1 >= ncur) ? -INFINITY : sc[1] * scale + bias;
+      float zmax = fmaxf(z0, z1);
+      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 1));
+      zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 2));
+      const float mn = fmaxf(m_h, zmax);
+      float p0, p1, alpha;
       if (mn == -INFINITY) {  // every key seen so far is masked
-        pr = 0.f;
+        p0 = p1 = 0.f;
         alpha = 1.f;
       } else {
-        pr = __expf(z - mn);
-        alpha = __expf(m_p[p] - mn);
+        p0 = __expf(z0 - mn);
+        p1 = __expf(z1 - mn);
+        alpha = __expf(m_h - mn);
       }
-      m_p[p] = mn;
-      float ps = pr;
-      ps += __shfl_xor_sync(FULL, ps, 4);
-      ps += __shfl_xor_sync(FULL, ps, 8);
-      ps += __shfl_xor_sync(FULL, ps, 16);
-      l_p[p] = l_p[p] * alpha + ps;
-      const int h = p * GP + hp;
-      if (uniq) {
-        pw[jj * G + h] = pr;
-        if (jj == 0) aw[h] = alpha;
+      m_h = mn;
+      float ps = p0 + p1;
+      ps += __shfl_xor_sync(FULL, ps, 1);
+      ps += __shfl_xor_sync(FULL, ps, 2);
+      l_h = l_h * alpha + ps;
+      const uint32_t pa = pack_bf16(p0, p1);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        acc[n][0] *= alpha;
+        acc[n][1] *= alpha;
+      }
+#pragma unroll
+      for (int nq = 0; nq < NT / 4; ++nq) {
+        uint32_t vb[4];
+        ldsm_x4_t(vb, vt + sw_off(wid * 8 + (lane & 7), (nq * 4 + (lane >> 3)) * 8));
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) mma_1688(acc[nq * 4 + mm], z2, z3, pa, vb[mm]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
+        mbar_wait(&empty[slot], (uint32_t)((i / NKV) & 1), err);
+        issue_unit(i + NKV);
       }
     }
-    __syncwarp();
-    {
-      float al[G];
-      loadg<G>(aw, al);
+    __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
+    if (g < G) {  // this warp's state of head g: (m, l) and acc, into [warp][head][D]
+      float* w = wst + (size_t)(wid * G + g) * D;
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[h][c] *= al[h];
+      for (int n = 0; n < NT; ++n)
+        *reinterpret_cast<float2*>(w + n * 8 + 2 * t4) = make_float2(acc[n][0], acc[n][1]);
+      if (t4 == 0) mlw[g * FD_WARPS + wid] = make_float2(m_h, l_h);
     }
-#pragma unroll
-    for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys
-      float pk[G], v[CPL];
-      loadg<G>(pw + k8 * G, pk);
-      loadn<CPL>(vt + (size_t)k8 * D + lane * CPL, v);
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk[h], pk[h], v[c], v[c + 1]);
+  } else {
+    // Each warp takes 8 keys of every unit (keys wid*8 .. wid*8+7) and keeps
+    // its own online-softmax state per head. Lane l holds columns
+    // [l*CPL, l*CPL + CPL) of q and of the accumulators of every head. The
+    // q.k partial sums of the warp's 8 keys x GP heads (one pass per group of
+    // at most 4 heads) are summed over the lanes by a transposing reduction:
+    // each shuffle stage halves the values a lane carries, so 8*GP sums cost
+    // fewer than 8*GP shuffles and lane l ends with the sum of key l/4 and
+    // head (l%4)/(4/GP) of the pass (lanes holding the same pair agree).
+    constexpr int GP = G < 4 ? G : 4;  // heads per pass
+    constexpr int HP = G / GP;         // passes
+    constexpr int NV = 8 * GP;         // partial sums per lane per pass
+    float qr[G][CPL], acc[G][CPL], m_p[HP], l_p[HP];
+  #pragma unroll
+    for (int h = 0; h < G; ++h) {
+  #pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        qr[h][c] = q_s[h * D + lane * CPL + c];
+        acc[h][c] = 0.f;
+      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
-    if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
-      mbar_wait(&empty[slot], (uint32_t)((i / NKV) & 1), err);
-      issue_unit(i + NKV);
+  #pragma unroll
+    for (int p = 0; p < HP; ++p) {
+      m_p[p] = -INFINITY;
+      l_p[p] = 0.f;
+    }
+    const int jj = lane >> 2;                                  // this lane's key of the 8
+    const int hp = (lane & 3) / (4 / GP);                      // and head within a pass
+    const bool uniq = (lane & (4 / GP - 1)) == 0;              // first lane holding the pair
+    float* pw = zp + wid * (2 * 8 * G);                        // [8 keys][G] p of this warp
+    float* aw = pw + 8 * G;                                    // [G] rescale factors
+    for (int i = 0; i < nu; ++i) {
+      const int slot = i % NKV;
+      const int u = unit_of(i);
+      const bool cur = (u == kk);
+      const float bias = (!cur && gated) ? key_score(fin[u]) - lse : 0.f;
+      mbar_wait_data(&full[slot], (uint32_t)((i / NKV) & 1), err);
+      const T* kt = reinterpret_cast<const T*>(U + (size_t)slot * kvslot) + (size_t)wid * 8 * D;
+      const T* vt = kt + TILE;
+      const bool masked = cur && (wid * 8 + jj >= ncur);
+  #pragma unroll
+      for (int p = 0; p < HP; ++p) {
+        float part[NV];
+  #pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          float kv[CPL];
+          loadn<CPL>(kt + (size_t)k8 * D + lane * CPL, kv);
+  #pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float a = 0.f;
+  #pragma unroll
+            for (int c = 0; c < CPL; ++c) a = fmaf(qr[p * GP + g][c], kv[c], a);
+            part[k8 * GP + g] = a;
+          }
+        }
+        const float dot = transpose_sum<NV>(part, lane);
+        const float z = masked ? -INFINITY : dot * scale + bias;
+        float zmax = z;
+        zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 4));
+        zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 8));
+        zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, 16));
+        const float mn = fmaxf(m_p[p], zmax);
+        float pr, alpha;
+        if (mn == -INFINITY) {  // every key seen so far is masked
+          pr = 0.f;
+          alpha = 1.f;
+        } else {
+          pr = __expf(z - mn);
+          alpha = __expf(m_p[p] - mn);
+        }
+        m_p[p] = mn;
+        float ps = pr;
+        ps += __shfl_xor_sync(FULL, ps, 4);
+        ps += __shfl_xor_sync(FULL, ps, 8);
+        ps += __shfl_xor_sync(FULL, ps, 16);
+        l_p[p] = l_p[p] * alpha + ps;
+        const int h = p * GP + hp;
+        if (uniq) {
+          pw[jj * G + h] = pr;
+          if (jj == 0) aw[h] = alpha;
+        }
+      }
+      __syncwarp();
+      {
+        float al[G];
+        loadg<G>(aw, al);
+  #pragma unroll
+        for (int h = 0; h < G; ++h)
+  #pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[h][c] *= al[h];
+      }
+  #pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8) {  // this warp's 8 keys
+        float pk[G], v[CPL];
+        loadg<G>(pw + k8 * G, pk);
+        loadn<CPL>(vt + (size_t)k8 * D + lane * CPL, v);
+  #pragma unroll
+        for (int h = 0; h < G; ++h)
+  #pragma unroll
+          for (int c = 0; c < CPL; c += 2) fma2(acc[h][c], acc[h][c + 1], pk[h], pk[h], v[c], v[c + 1]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (tid == 0 && i + NKV < nu) {  // refill the slot once every warp is done with it
+        mbar_wait(&empty[slot], (uint32_t)((i / NKV) & 1), err);
+        issue_unit(i + NKV);
+      }
+    }
+  
+
+  // ---- 5. fold the warp states per head; push head h's state into CTA h.
+    __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float* w = wst + (size_t)(wid * G + h) * D;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) w[lane * CPL + c] = acc[h][c];
+    }
+    if (lane < 4 && uniq) {  // the lanes of key 0 hold every head's (m, l) once
+#pragma unroll
+      for (int p = 0; p < HP; ++p) mlw[(p * GP + hp) * FD_WARPS + wid] = make_float2(m_p[p], l_p[p]);
     }
   }
-
   // ---- 5. fold the warp states per head; push head h's state into CTA h.
   // Every thread of the fold takes (head, 4 columns) and derives the 8 warp
   // weights itself from the warps' (m, l).
-  __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
-  float* wst = reinterpret_cast<float*>(U);  // [warp][head][D] acc
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float* w = wst + (size_t)(wid * G + h) * D;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) w[lane * CPL + c] = acc[h][c];
-  }
-  if (lane < 4 && uniq) {  // the lanes of key 0 hold every head's (m, l) once
-#pragma unroll
-    for (int p = 0; p < HP; ++p) mlw[(p * GP + hp) * FD_WARPS + wid] = make_float2(m_p[p], l_p[p]);
-  }
   __syncthreads();
   {
     const uint32_t cst_r = smem_u32(cst) + (uint32_t)(crank * D * 4);
@@ -933,10 +1108,21 @@ cudaError_t launch_fused_t(const void* q, const void* kc, const void* vc, const 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  // bf16 caches are read by TMA: the caches as 3-D tensors of 64 x 64 boxes
+  // (contiguous: planes of Lmax rows per (sequence, kv head); paged: planes of
+  // 64 rows per (page, kv head))
+  CUtensorMap km = {}, vm = {};
+  if (std::is_same<T, __nv_bfloat16>::value) {
+    const int rows = PAGED ? SAS_BLOCK : Lmax;
+    const int planes = PAGED ? npages * Hkv : B * Hkv;
+    if (!make_tma_map_bf16_3d(&km, kc, D, rows, planes) ||
+        !make_tma_map_bf16_3d(&vm, vc, D, rows, planes))
+      return cudaErrorInvalidValue;
+  }
   return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
                             static_cast<const T*>(vc), static_cast<const S*>(ksum), Hkv, Lmax,
                             lens, topk, gated, scale, per_max, ub, static_cast<T*>(o), idx_out,
-                            bt, npages);
+                            bt, npages, km, vm);
 }
 
 template <typename T, int D>

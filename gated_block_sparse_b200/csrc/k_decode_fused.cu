@@ -916,9 +916,6 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
         issue_unit(i + NKV);
       }
     }
-  
-
-  // ---- 5. fold the warp states per head; push head h's state into CTA h.
     __syncthreads();  // every warp left the loop and every copy was consumed: region u is free
 #pragma unroll
     for (int h = 0; h < G; ++h) {

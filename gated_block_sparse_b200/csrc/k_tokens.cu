@@ -9,7 +9,8 @@
 //
 // Selection: one CTA per (query block t, kv group r, sequence b) scores its
 // 64 token means against the C = t summaries (64 x 64 tiles, fp32), then one
-// warp per row takes the row's gate and its Top-K by rank counting.
+// warp per row takes the row's gate and its Top-K by a bitwise search for the
+// k-th largest score.
 // Attention: one CTA per (query block, head, sequence) walks the union of the
 // blocks its rows selected (built from the rows' lists in shared memory),
 // then the current block. Each row finds its bias for a unit by walking its
@@ -30,6 +31,87 @@ __device__ uint32_t g_tokens_err = 0;
 constexpr int TOK_CMAX = 512;  // history blocks of a query block at most
 
 // ------------------------------------------------------------------ selection
+// Order-preserving unsigned key of a score: a larger score has a larger key,
+// and -0 was mapped to +0 before, so equal scores have equal keys.
+__device__ __forceinline__ uint32_t score_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+}
+
+// One warp: the gate and the Top-K of one row's C scores si[0 .. C) (C <= 32
+// KPL). kk = min(topk, C) blocks are kept, ordered by (score desc, block
+// asc): tau, the kk-th largest key, is found bit by bit (the largest value
+// with at least kk keys at or above it); the keys above tau are kept, and of
+// the keys equal to tau the lowest-numbered ones until kk are reached. The
+// kept blocks and their log g = s - LSE(s) are written in ascending block
+// order, the rest of the row padded with -1 / 0.
+template <int KPL>
+__device__ __forceinline__ void select_row(const float* si, int C, int kk, int topk,
+                                           int32_t* __restrict__ idx_row,
+                                           float* __restrict__ logg_row,
+                                           int32_t* __restrict__ cnt_row) {
+  const int lane = threadIdx.x & 31;
+  float sv[KPL];
+  uint32_t kv[KPL];
+  float mx = -FLT_MAX;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int m = j * 32 + lane;
+    sv[j] = m < C ? si[m] : -FLT_MAX;
+    kv[j] = m < C ? score_key(sv[j]) : 0u;
+    mx = fmaxf(mx, sv[j]);
+  }
+  mx = warp_max(mx);
+  float z = 0.f;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j)
+    if (j * 32 + lane < C) z += __expf(sv[j] - mx);
+  z = warp_sum(z);
+  const float lse_i = mx + __logf(z);
+  uint32_t tau = 0u;  // keys of m >= C are 0 and every real key is above 0
+  if (kk > 0 && kk < C) {
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int n = 0;
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) n += kv[j] >= cand;
+      if ((int)__reduce_add_sync(0xffffffffu, (unsigned)n) >= kk) tau = cand;
+    }
+  }
+  int above = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) above += (j * 32 + lane < C) && kv[j] > tau;
+  above = (int)__reduce_add_sync(0xffffffffu, (unsigned)above);
+  const int need = kk > 0 ? kk - above : 0;  // keys equal to tau still to keep
+  int ties = 0, pos = 0;
+#pragma unroll
+  for (int j = 0; j < KPL; ++j) {
+    const int m = j * 32 + lane;
+    const bool in = m < C && kk > 0;
+    const bool eq = in && kv[j] == tau;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const int tr = ties + __popc(eqb & ((1u << lane) - 1u));
+    ties += __popc(eqb);
+    const bool sel = in && (kv[j] > tau || (eq && tr < need));
+    const unsigned bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int p = pos + __popc(bal & ((1u << lane) - 1u));
+      if (p < topk) {
+        idx_row[p] = m;
+        logg_row[p] = sv[j] - lse_i;
+      }
+    }
+    pos += __popc(bal);
+  }
+  pos = min(pos, topk);
+  for (int p = pos + lane; p < topk; p += 32) {
+    idx_row[p] = -1;
+    logg_row[p] = 0.f;
+  }
+  if (lane == 0) *cnt_row = pos;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(AT_THREADS) k_select_tokens(
     const T* __restrict__ q, const float* __restrict__ ksum, int Hq, int Hkv, int N, int topk,
@@ -74,44 +156,11 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_tokens(
   __syncthreads();
   const int kk = min(topk, C);
   for (int i = wid; i < nr; i += AT_THREADS / 32) {
-    const float* si = sc + i * CP;
     const size_t orow = ((size_t)b * Hkv + r) * N + row0 + i;
-    float mx = -FLT_MAX;
-    for (int m = lane; m < C; m += 32) mx = fmaxf(mx, si[m]);
-    mx = warp_max(mx);
-    float z = 0.f;
-    for (int m = lane; m < C; m += 32) z += __expf(si[m] - mx);
-    z = warp_sum(z);
-    const float lse_i = mx + __logf(z);
-    int pos = 0;  // kept blocks written so far, in ascending block order
-    for (int m0 = 0; m0 < C && kk > 0; m0 += 32) {
-      const int m = m0 + lane;
-      bool sel = false;
-      if (m < C) {
-        const float sv = si[m];
-        int above = 0;
-        for (int x = 0; x < C && above < kk; ++x) {
-          const float sx = si[x];
-          above += (sx > sv) || (sx == sv && x < m);
-        }
-        sel = above < kk;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, sel);
-      if (sel) {
-        const int p = pos + __popc(bal & ((1u << lane) - 1u));
-        if (p < topk) {
-          idx[orow * topk + p] = m;
-          logg[orow * topk + p] = si[m] - lse_i;
-        }
-      }
-      pos += __popc(bal);
-    }
-    pos = min(pos, topk);
-    for (int p = pos + lane; p < topk; p += 32) {
-      idx[orow * topk + p] = -1;
-      logg[orow * topk + p] = 0.f;
-    }
-    if (lane == 0) cnt[orow] = pos;
+    if (C <= 256) select_row<8>(sc + i * CP, C, kk, topk, idx + orow * topk, logg + orow * topk,
+                                cnt + orow);
+    else select_row<TOK_CMAX / 32>(sc + i * CP, C, kk, topk, idx + orow * topk,
+                                   logg + orow * topk, cnt + orow);
   }
 }
 

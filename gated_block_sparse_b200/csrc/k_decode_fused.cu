@@ -208,6 +208,32 @@ __device__ __forceinline__ float transpose_sum(float (&v)[NV], int lane) {
   return v[0];
 }
 
+// A step reads each summary and each kept K/V tile once: its copies carry an
+// L2 evict-first policy, so that the streamed bytes do not push out of L2 what
+// is reused from step to step (among it the kernel's own instructions).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_g2s_once(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(l2_evict_first())
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_once(void* dst, const CUtensorMap* map, int c0,
+                                                 int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)),
+      "l"(l2_evict_first())
+      : "memory");
+}
+
 // Warp MMAs on bf16 operands with fp32 accumulation (c += a b).
 __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
                                           uint32_t b1) {
@@ -380,12 +406,12 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       }
 #pragma unroll
       for (int bx = 0; bx < D / 64; ++bx) {
-        tc::tma_load_3d(dst + bx * 8192, &kmap, 64 * bx, row0, plane, bar);
-        tc::tma_load_3d(dst + TILE * sizeof(T) + bx * 8192, &vmap, 64 * bx, row0, plane, bar);
+        tma_load_3d_once(dst + bx * 8192, &kmap, 64 * bx, row0, plane, bar);
+        tma_load_3d_once(dst + TILE * sizeof(T) + bx * 8192, &vmap, 64 * bx, row0, plane, bar);
       }
     } else {
-      bulk_g2s(dst, kv_tile(kc, blk), TILE * sizeof(T), bar);
-      bulk_g2s(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), bar);
+      bulk_g2s_once(dst, kv_tile(kc, blk), TILE * sizeof(T), bar);
+      bulk_g2s_once(dst + TILE * sizeof(T), kv_tile(vc, blk), TILE * sizeof(T), bar);
     }
   };
   // summaries [first, first + cnt) of this CTA's range into ring slot `slot`:
@@ -396,12 +422,12 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       if (lane == 0) mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * sizeof(S)));
       __syncwarp();
       for (int j = lane; j < cnt; j += 32)
-        bulk_g2s(dst + (size_t)j * D, ksum + ((size_t)page_of(m0 + first + j) * Hkv + r) * D,
+        bulk_g2s_once(dst + (size_t)j * D, ksum + ((size_t)page_of(m0 + first + j) * Hkv + r) * D,
                  (uint32_t)(D * sizeof(S)), &sum_bar[slot]);
     } else {
       mbar_arrive_expect_tx(&sum_bar[slot], (uint32_t)(cnt * D * sizeof(S)));
-      bulk_g2s(dst, ks_row + (size_t)(m0 + first) * D, (uint32_t)(cnt * D * sizeof(S)),
-               &sum_bar[slot]);
+      bulk_g2s_once(dst, ks_row + (size_t)(m0 + first) * D, (uint32_t)(cnt * D * sizeof(S)),
+                    &sum_bar[slot]);
     }
   };
 
@@ -971,7 +997,7 @@ __global__ void __launch_bounds__(FD_THREADS, 2) k_decode_fused(
       const float M = warp_max(m);
       const float f = ok ? __expf(m - M) : 0.f;
       const float Ls = warp_sum(ok ? cml[2 * lane + 1] * f : 0.f);
-      if (lane < CS) cw[lane] = f / Ls;
+      if (lane < CS) cw[lane] = __fdividef(f, Ls);  // Ls >= 1: the max state has f = 1
     }
     __syncthreads();
     const int h = crank;

@@ -11,8 +11,10 @@
 //
 // One CTA per (query block t, kv group r, pair of query heads of the group):
 // an M = 128 tile (2 heads x 64 rows) that shares every K/V block it loads.
-//   warp 4     TMA producer: Q once (4 boxes of 64 rows x 64 columns, 128-byte
-//              swizzle), then K and V of each unit into a 2-stage ring;
+//   warp 4     TMA producers: lane 0 loads Q once (4 boxes of 64 rows x 64
+//              columns, 128-byte swizzle) and then K of each unit, lane 1 V
+//              of each unit, each into its own 2-stage ring (a K slot is
+//              released when S_j is done, a V slot when PV_j is);
 //   warp 5     one elected thread issues tcgen05.mma: S_j = Q K_j^T
 //              (M128 N64 K128, two TMEM buffers of 64 columns) and
 //              O += P_j V_j (M128 N128 K64, 128 TMEM columns);
@@ -64,7 +66,13 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy rescale threshold (log2 units)
 constexpr int TOK_UMAX = 512;         // history blocks of a query block at most (per-token mode)
 
-enum Bar { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 10, NBAR = 11 };
+// K_j and V_j have their own full/empty barriers: a K slot is free once S_j is
+// done, a V slot once PV_j is done, so the next K load starts a softmax earlier.
+enum Bar {
+  B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 10, B_VF = 11, B_VE = 13,
+  NBAR = 15
+};
+static_assert(NBAR * 8 + 4 <= 128, "barriers and the TMEM address fit their 128 bytes");
 
 }  // namespace
 
@@ -150,32 +158,39 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      tc::prefetch_map(&qmap);
-      tc::prefetch_map(&kmap);
-      tc::prefetch_map(&vmap);
-      mbar_arrive_expect_tx(&bars[B_Q], Q_BYTES);
-      for (int c = 0; c < 2; ++c)
-        for (int h = 0; h < 2; ++h)
-          tc::tma_load_3d(sm + OFF_Q + c * 16384 + h * 8192, &qmap, 64 * c, 64 * t,
-                          b * Hq + h0 + h, &bars[B_Q]);
+    // lane 0: Q, then K of every unit; lane 1: V of every unit
+    if (lane < 2) {
+      const bool kl = (lane == 0);
+      if (kl) {
+        tc::prefetch_map(&qmap);
+        tc::prefetch_map(&kmap);
+        mbar_arrive_expect_tx(&bars[B_Q], Q_BYTES);
+        for (int c = 0; c < 2; ++c)
+          for (int h = 0; h < 2; ++h)
+            tc::tma_load_3d(sm + OFF_Q + c * 16384 + h * 8192, &qmap, 64 * c, 64 * t,
+                            b * Hq + h0 + h, &bars[B_Q]);
+      } else {
+        tc::prefetch_map(&vmap);
+      }
+      const CUtensorMap* map = kl ? &kmap : &vmap;
+      uint64_t* fullb = &bars[kl ? B_KF : B_VF];
+      uint64_t* emptyb = &bars[kl ? B_KE : B_VE];
+      const uint32_t half = kl ? 0u : 16384u;
       int ucur = -1;  // per-token: the previous unit's block
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
-        if (j >= 2) mbar_wait_data(&bars[B_KVE + s], ((j >> 1) - 1) & 1, err);
+        if (j >= 2) mbar_wait_data(&emptyb[s], ((j >> 1) - 1) & 1, err);
         if (TOK && j < kk) ucur = next_unit(ucur + 1);
         int blk = (j < kk) ? (TOK ? ucur : idx_row[j]) : t;
         if (blk < 0 || blk >= t) {
-          if (j < kk) atomicOr(err, kErrBadIndex);
+          if (j < kk && kl) atomicOr(err, kErrBadIndex);
           blk = t;
         }
-        unsigned char* st = sm + OFF_KV + s * KV_STAGE_BYTES;
-        mbar_arrive_expect_tx(&bars[B_KVF + s], KV_STAGE_BYTES);
+        unsigned char* st = sm + OFF_KV + s * KV_STAGE_BYTES + half;
+        mbar_arrive_expect_tx(&fullb[s], KV_STAGE_BYTES / 2);
         const int plane = b * Hkv + r;
-        tc::tma_load_3d(st, &kmap, 0, 64 * blk, plane, &bars[B_KVF + s]);
-        tc::tma_load_3d(st + 8192, &kmap, 64, 64 * blk, plane, &bars[B_KVF + s]);
-        tc::tma_load_3d(st + 16384, &vmap, 0, 64 * blk, plane, &bars[B_KVF + s]);
-        tc::tma_load_3d(st + 24576, &vmap, 64, 64 * blk, plane, &bars[B_KVF + s]);
+        tc::tma_load_3d(st, map, 0, 64 * blk, plane, &fullb[s]);
+        tc::tma_load_3d(st + 8192, map, 64, 64 * blk, plane, &fullb[s]);
       }
     }
   } else if (warp == 5) {
@@ -188,6 +203,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       mbar_wait_data(&bars[B_Q], 0, err);
       auto pv = [&](int j) {  // O += P_j V_j
         mbar_wait(&bars[B_PF], j & 1, err);
+        mbar_wait_data(&bars[B_VF + (j & 1)], (j >> 1) & 1, err);
         tc::fence_after_sync();
         const uint32_t v_addr = smem_u32(sm + OFF_KV + (j & 1) * KV_STAGE_BYTES + 16384);
 #pragma unroll
@@ -197,11 +213,11 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
           tc::mma_bf16(tm_o, a, bd, ID_PV, (j > 0 || ks > 0) ? 1u : 0u);
         }
         tc::commit(&bars[B_OD]);
-        tc::commit(&bars[B_KVE + (j & 1)]);
+        tc::commit(&bars[B_VE + (j & 1)]);
       };
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
-        mbar_wait_data(&bars[B_KVF + s], (j >> 1) & 1, err);
+        mbar_wait_data(&bars[B_KF + s], (j >> 1) & 1, err);
         if (j >= 2) mbar_wait(&bars[B_SE + s], ((j >> 1) - 1) & 1, err);
         tc::fence_after_sync();
         const uint32_t k_addr = smem_u32(sm + OFF_KV + s * KV_STAGE_BYTES);
@@ -213,6 +229,7 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
           tc::mma_bf16(tm_s[s], a, bd, ID_QK, ks > 0 ? 1u : 0u);
         }
         tc::commit(&bars[B_SF + s]);
+        tc::commit(&bars[B_KE + s]);
         if (j >= 1) pv(j - 1);
       }
       pv(nunits - 1);

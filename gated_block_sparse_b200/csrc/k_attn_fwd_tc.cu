@@ -74,6 +74,35 @@ enum Bar {
 };
 static_assert(NBAR * 8 + 4 <= 128, "barriers and the TMEM address fit their 128 bytes");
 
+// (a0, a1) = (x0, x1) * c + (o, o) as one packed fp32x2 FMA
+__device__ __forceinline__ void fma2c(float& a0, float& a1, float x0, float x1, float c, float o) {
+  asm("{\n\t.reg .b64 x, c, o, a;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 c, {%4, %4};\n\t"
+      "mov.b64 o, {%5, %5};\n\t"
+      "fma.rn.f32x2 a, x, c, o;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(a0), "=f"(a1)
+      : "f"(x0), "f"(x1), "f"(c), "f"(o));
+}
+// (s0, s1) += (x0, x1) as one packed fp32x2 add
+__device__ __forceinline__ void add2(float& s0, float& s1, float x0, float x1) {
+  asm("{\n\t.reg .b64 s, x;\n\t"
+      "mov.b64 s, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "add.rn.f32x2 s, s, x;\n\t"
+      "mov.b64 {%0, %1}, s;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(x0), "f"(x1));
+}
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 }  // namespace
 
 template <bool TOK>
@@ -282,26 +311,37 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_SE + s]);
-      float mx = -INFINITY;
+      // the row max in the log2 domain: c1 > 0, so max_i (z_i c1 + bias) = c1 max_i z_i + bias
+      if (cur) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        float v = z[i] * c1 + bias;
-        if (cur && i > qr) v = -INFINITY;
-        z[i] = v;
-        mx = fmaxf(mx, v);
+        for (int i = 0; i < 64; ++i)
+          if (i > qr) z[i] = -INFINITY;  // causal mask of the current block
       }
+      float zm[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) zm[c] = fmaxf(z[2 * c], z[2 * c + 1]);
+#pragma unroll
+      for (int i = 8; i < 64; i += 8) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) zm[c] = max3(zm[c], z[i + 2 * c], z[i + 2 * c + 1]);
+      }
+      const float mx = max3(zm[0], zm[1], fmaxf(zm[2], zm[3])) * c1 + bias;
       const float mnew = fmaxf(m, mx);
       const bool grow = (j == 0) || (mnew > m + RESCALE_LOG2);
       const float muse = grow ? mnew : m;
-      float rs = 0.f;
+      const float off = bias - muse;  // -inf where the row masks the whole unit
+      float rs0 = 0.f, rs1 = 0.f;
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = tc::ex2(z[2 * i] - muse), p1 = tc::ex2(z[2 * i + 1] - muse);
-        rs += p0 + p1;
+        float a0, a1;
+        fma2c(a0, a1, z[2 * i], z[2 * i + 1], c1, off);
+        const float p0 = tc::ex2(a0), p1 = tc::ex2(a1);
+        add2(rs0, rs1, p0, p1);
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
       }
+      const float rs = rs0 + rs1;
       if (j > 0) {
         // PV_{j-1} must be done: O is stable and the P buffer is free
         mbar_wait_data(&bars[B_OD], (j - 1) & 1, err);

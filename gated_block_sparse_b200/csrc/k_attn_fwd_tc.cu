@@ -17,14 +17,16 @@
 //              released when S_j is done, a V slot when PV_j is);
 //   warp 5     one elected thread issues tcgen05.mma: S_j = Q K_j^T
 //              (M128 N64 K128, two TMEM buffers of 64 columns) and
-//              O += P_j V_j (M128 N128 K64, 128 TMEM columns);
+//              O += P_j V_j (M128 N128 K64, 128 TMEM columns, the A operand
+//              P_j read from TMEM); S_j waits until PV_{j-2} has read P_{j-2}
+//              from the buffer S_j overwrites;
 //   warps 0-3  softmax: thread i owns row i = TMEM lane i; loads S_j,
 //              applies scale, bias and the causal mask in the log2 domain,
 //              updates the running max lazily (O in TMEM is rescaled only when
-//              the max grows by more than 2^8), writes P_j as bf16 into shared
-//              memory in the 128-byte-swizzled K-major layout the MMA reads;
-//              at the end divides O by the row sum and writes o and lse.
-// About 113 KB of shared memory and 256 TMEM columns per CTA, so two CTAs
+//              the max grows by more than 2^8), writes P_j as bf16 (two per
+//              column) over the first half of S_j's TMEM buffer; at the end
+//              divides O by the row sum and writes o and lse.
+// About 97 KB of shared memory and 256 TMEM columns per CTA, so two CTAs
 // share an SM and overlap one's softmax with the other's MMAs. Every wait is
 // bounded.
 //
@@ -55,11 +57,9 @@ constexpr int FT_THREADS = 192;
 constexpr int D = 128;
 constexpr uint32_t Q_BYTES = 128 * D * 2;           // 32 KB
 constexpr uint32_t KV_STAGE_BYTES = 2 * 64 * D * 2;  // K + V block, 32 KB
-constexpr uint32_t P_BYTES = 128 * 64 * 2;          // 16 KB
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_P = OFF_KV + 2 * KV_STAGE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+constexpr uint32_t OFF_BAR = OFF_KV + 2 * KV_STAGE_BYTES;
 constexpr uint32_t OFF_UM = OFF_BAR + 128;  // per-token mode: union bitmask and its count
 constexpr uint32_t SMEM_BYTES = OFF_UM + 128;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -69,8 +69,7 @@ constexpr int TOK_UMAX = 512;         // history blocks of a query block at most
 // K_j and V_j have their own full/empty barriers: a K slot is free once S_j is
 // done, a V slot once PV_j is done, so the next K load starts a softmax earlier.
 enum Bar {
-  B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_SE = 7, B_PF = 9, B_OD = 10, B_VF = 11, B_VE = 13,
-  NBAR = 15
+  B_Q = 0, B_KF = 1, B_KE = 3, B_SF = 5, B_PF = 7, B_OD = 8, B_VF = 9, B_VE = 11, NBAR = 13
 };
 static_assert(NBAR * 8 + 4 <= 128, "barriers and the TMEM address fit their 128 bytes");
 
@@ -94,6 +93,32 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float x0, float x1) {
       "mov.b64 {%0, %1}, s;\n\t}"
       : "+f"(s0), "+f"(s1)
       : "f"(x0), "f"(x1));
+}
+
+// O += P V with the A operand (P, bf16, 128 lanes x 16 elements packed two
+// per 32-bit column) read from TMEM and B from shared memory.
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns from registers (lane of the warp's
+// quarter, columns taddr.col .. +31)
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+      "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 // max(a, b, c) in one instruction
@@ -172,9 +197,9 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
   };
   const int nunits = kk + 1;  // history units, then the current block
   if (tid == 0) {
-    // S-empty (both buffers) and P-full take one arrival per softmax warp
+    // P-full takes one arrival per softmax warp
     for (int i = 0; i < NBAR; ++i)
-      mbar_init(&bars[i], (i == B_SE || i == B_SE + 1 || i == B_PF) ? 4 : 1);
+      mbar_init(&bars[i], i == B_PF ? 4 : 1);
     fence_mbar_init();
   }
   if (warp == 5) tc::tmem_alloc(tmem_slot, 256);
@@ -228,7 +253,6 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       constexpr uint32_t ID_QK = tc::idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t ID_PV = tc::idesc_bf16(128, 128, 0, 1);
       const uint32_t q_addr = smem_u32(sm + OFF_Q);
-      const uint32_t p_addr = smem_u32(sm + OFF_P);
       mbar_wait_data(&bars[B_Q], 0, err);
       auto pv = [&](int j) {  // O += P_j V_j
         mbar_wait(&bars[B_PF], j & 1, err);
@@ -236,10 +260,9 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
         tc::fence_after_sync();
         const uint32_t v_addr = smem_u32(sm + OFF_KV + (j & 1) * KV_STAGE_BYTES + 16384);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t a = tc::sw128_desc(p_addr + ks * 32, 16, 1024);
+        for (int ks = 0; ks < 4; ++ks) {  // P_j: columns 8 ks .. 8 ks + 7 of S_j's buffer
           const uint64_t bd = tc::sw128_desc(v_addr + ks * 2048, 8192, 1024);
-          tc::mma_bf16(tm_o, a, bd, ID_PV, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_tmem_a(tm_o, tm_s[j & 1] + 8 * ks, bd, ID_PV, (j > 0 || ks > 0) ? 1u : 0u);
         }
         tc::commit(&bars[B_OD]);
         tc::commit(&bars[B_VE + (j & 1)]);
@@ -247,7 +270,8 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       for (int j = 0; j < nunits; ++j) {
         const int s = j & 1;
         mbar_wait_data(&bars[B_KF + s], (j >> 1) & 1, err);
-        if (j >= 2) mbar_wait(&bars[B_SE + s], ((j >> 1) - 1) & 1, err);
+        // S_j overwrites P_{j-2} (S_{j-2}'s buffer): PV_{j-2} must have read it
+        if (j >= 2) mbar_wait(&bars[B_OD], (j - 2) & 1, err);
         tc::fence_after_sync();
         const uint32_t k_addr = smem_u32(sm + OFF_KV + s * KV_STAGE_BYTES);
 #pragma unroll
@@ -271,7 +295,6 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c1 = scale * LOG2E;
     float m = -1e30f, l = 0.f;
-    unsigned char* prow = sm + OFF_P + row * 128;
     // per-token selection: this row's own list (ascending), walked as the
     // units advance; rows past the sequence end select nothing
     const size_t trow = tok0 + (pos < N ? qr : 0);
@@ -308,9 +331,6 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
           z[32 + i] = bb[i];
         }
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_SE + s]);
       // the row max in the log2 domain: c1 > 0, so max_i (z_i c1 + bias) = c1 max_i z_i + bias
       if (cur) {
 #pragma unroll
@@ -343,7 +363,9 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
       }
       const float rs = rs0 + rs1;
       if (j > 0) {
-        // PV_{j-1} must be done: O is stable and the P buffer is free
+        // PV_{j-1} done before O is rescaled. Waiting on every unit also keeps
+        // this thread within one phase of the O-done barrier, so that its
+        // parity waits (here and at the end) are never a phase behind.
         mbar_wait_data(&bars[B_OD], (j - 1) & 1, err);
         tc::fence_after_sync();
         const float alpha = grow ? tc::ex2(m - muse) : 1.f;
@@ -364,14 +386,10 @@ __global__ void __launch_bounds__(FT_THREADS, 2) k_attn_fwd_tc(
         l = rs;
       }
       m = muse;
-      // P row (64 bf16 = 8 chunks of 16 bytes), 128-byte swizzle: chunk c of
-      // row i sits at chunk position c ^ (i & 7)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
-      }
-      fence_proxy_async_smem();
+      // P_j (64 bf16, two per column) into the first 32 columns of S_j's
+      // buffer, this thread's lane: the A operand of O += P_j V_j
+      tmem_st32u(tm_s[s] + lane_off, pk);
+      tc::tmem_wait_st();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PF]);

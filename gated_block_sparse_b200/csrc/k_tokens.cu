@@ -724,6 +724,7 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
     }
     __syncthreads();
     // dqbar[i] += sum_m ds[i][m] kbar_m
+#pragma unroll 4
     for (int j = 0; j < nm; ++j) {
       float dsj[4];
 #pragma unroll
@@ -748,6 +749,7 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
       for (int g = 0; g < S::NG; ++g)
 #pragma unroll
         for (int e = 0; e < 4; ++e) a[jj][g][e] = 0.f;
+#pragma unroll 4
     for (int i2 = 0; i2 < nr; ++i2) {
       float wj[4];
 #pragma unroll

@@ -295,8 +295,6 @@ def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
     lens = h["lens"].to(dev)
     kc0, vc0 = h["kc"].to(dev), h["vc"].to(dev)
     bf16_sum = w.summary == "bf16"
-    if bf16_sum and paged:
-        raise SystemExit("bf16 summaries read contiguous caches only")
     ks0 = (sas.sas_block_summary_ex(kc0, torch.bfloat16) if bf16_sum
            else sas.sas_block_summary(kc0))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -326,15 +324,16 @@ def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
             return p
         for j in range(L):
             kcs[j], vcs[j] = pages(kcs[j]), pages(vcs[j])
-            kss[j] = sas.sas_block_summary(kcs[j]).view(B_ * nblk, Hkv, d_)
+            kss[j] = (sas.sas_block_summary_ex(kcs[j], torch.bfloat16) if bf16_sum
+                      else sas.sas_block_summary(kcs[j])).view(B_ * nblk, Hkv, d_)
     o = torch.empty_like(q)
     stream = torch.cuda.Stream(dev)
     clocks = clock_sampler(dev.index if dev.index is not None else 0)
 
     def decode(j, qq, out):
-        if bt is not None:
-            sas.sas_decode_paged(qq, kcs[j], vcs[j], kss[j], bt, lens, topk, gated=c["gated"],
-                                 out=out)
+        if bt is not None:  # sas_decode_paged_ex takes the summaries' dtype from kss[j]
+            sas.sas_decode_paged_ex(qq, kcs[j], vcs[j], kss[j], bt, lens, topk,
+                                    gated=c["gated"], out=out)
         elif bf16_sum:
             sas.sas_decode_ex(qq, kcs[j], vcs[j], lens, kss[j], topk, gated=c["gated"], out=out)
         else:
@@ -354,7 +353,8 @@ def bench_decode_ours(K: int, W: int, world: int, local: int, w: DecodeWorkload,
     kt = ms / K * 1e-3
     ach = w.step_bytes / kt / 1e9
     ach_sel = w.att_bytes / kt / 1e9
-    variant = "paged" if bt is not None else ("bf16_summaries" if bf16_sum else None)
+    variant = ("paged" if bt is not None else None, "bf16_summaries" if bf16_sum else None)
+    variant = "_".join(v for v in variant if v) or None
     roof = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(ach, 1),
             "peak": peaks["hbm"], "unit": "GB/s", "frac": round(ach / peaks["hbm"], 4),
             "traffic": (None if variant else
@@ -461,12 +461,14 @@ def finish_decode(sas, c, w, q, lens, kcs, vcs, kss, L, K, W, world, stream, o, 
     # eager step), a q copy alone and the kernel alone (the device-timed step)
     copy_ms = event_ms(lambda: qd.copy_(qh, non_blocking=True), E, stream)
     nb = q.numel() * q.element_size()
-    api = ({"paged": "sas_decode_paged with torch copies",
+    api = ({"paged": "sas_decode_paged_ex with torch copies",
+            "paged_bf16_summaries": "sas_decode_paged_ex with torch copies",
             "bf16_summaries": "sas_decode_ex with torch copies"}.get(variant) or
            "sas_decode_host (the step reading q from and writing o to pinned host memory)")
     value = D.whole_job_rate(w.step_bytes * K, world, ms) / 1e9
     cfg = {**w.describe(), "parallelism": f"replicas x{world}",
-           "cache": ("paged: 64-token pages in a random page order" if variant == "paged"
+           "cache": ("paged: 64-token pages in a random page order"
+                     if variant and variant.startswith("paged")
                      else "contiguous [B][Hkv][Lmax][d]"),
            "l2": f"rotating {L} layer copies of cache + summaries "
                  f"({w.step_bytes * L / 1e6:.0f} MB touched per rotation, L2 {l2 / 1e6:.0f} MB)"}
@@ -912,10 +914,14 @@ def run_one(name: str, cfg: str, opts: dict, K: int, W: int, world: int, rank: i
         rec = bench_prefill_ours(cfg, K, W, world, local, host=hosts[cfg])
         if rank == 0:
             rec["cpu_baseline"] = cpu_baseline_prefill(cfg, cpu_seconds, host=hosts[cfg])
+    parts = []
     if opts.get("paged"):
-        rec["config"]["variant"] = "paged KV cache (sas_decode_paged)"
+        parts.append("paged KV cache")
     if opts.get("summary") == "bf16":
-        rec["config"]["variant"] = "bf16 block summaries (sas_decode_ex)"
+        parts.append("bf16 block summaries")
+    if parts:
+        rec["config"]["variant"] = " + ".join(parts) + (
+            " (sas_decode_paged_ex)" if opts.get("paged") else " (sas_decode_ex)")
     return rec
 
 

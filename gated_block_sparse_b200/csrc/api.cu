@@ -448,14 +448,16 @@ sas_status sas_decode_host(const void* q_host, void* q_dev, const void* kc, cons
 }
 
 // ---------------------------------------------------------------- paged decode
-sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
-                            const float* kspool, sas_dtype dt, int B, int Hq, int Hkv, int npages,
-                            int d, const int32_t* block_table, int max_blocks,
-                            const int32_t* lens, int topk, int gated, float scale, void* o,
-                            int32_t* idx_out, sas_stream_t stream) {
-  g_last_error.clear();
+static sas_status decode_paged_impl(const char* fn, const void* q, const void* kpool,
+                                    const void* vpool, const void* kspool, sas_dtype sum_dt,
+                                    sas_dtype dt, int B, int Hq, int Hkv, int npages, int d,
+                                    const int32_t* block_table, int max_blocks,
+                                    const int32_t* lens, int topk, int gated, float scale,
+                                    void* o, int32_t* idx_out, sas_stream_t stream) {
   REQUIRE(max_blocks >= 1 && max_blocks <= (1 << 24), SAS_ERR_INVALID_ARG,
           "max_blocks must be in [1, 2^24] (got %d)", max_blocks);
+  REQUIRE(sum_dt == SAS_F32 || sum_dt == SAS_BF16, SAS_ERR_INVALID_ARG,
+          "summary dtype must be SAS_F32 or SAS_BF16 (got %d)", (int)sum_dt);
   sas_status s = check_decode(dt, B, Hq, Hkv, max_blocks * 64, d, topk, gated);
   if (s != SAS_OK) return s;
   REQUIRE(npages >= 1, SAS_ERR_INVALID_ARG, "npages must be >= 1 (got %d)", npages);
@@ -469,10 +471,33 @@ sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
   REQUIRE_PTR(o);
   if (idx_out) REQUIRE(aligned16(idx_out), SAS_ERR_INVALID_ARG, "idx_out must be 16-byte aligned");
   return cuda_status(sas::launch_decode_paged(q, kpool, vpool, dt == SAS_BF16, B, Hq, Hkv, npages,
-                                              d, block_table, max_blocks, lens, kspool, topk,
-                                              gated, resolve_scale(scale, d), o, idx_out,
+                                              d, block_table, max_blocks, lens, kspool,
+                                              sum_dt == SAS_BF16, topk, gated,
+                                              resolve_scale(scale, d), o, idx_out,
                                               (cudaStream_t)stream),
-                     "sas_decode_paged launch");
+                     fn);
+}
+
+sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
+                            const float* kspool, sas_dtype dt, int B, int Hq, int Hkv, int npages,
+                            int d, const int32_t* block_table, int max_blocks,
+                            const int32_t* lens, int topk, int gated, float scale, void* o,
+                            int32_t* idx_out, sas_stream_t stream) {
+  g_last_error.clear();
+  return decode_paged_impl("sas_decode_paged launch", q, kpool, vpool, kspool, SAS_F32, dt, B,
+                           Hq, Hkv, npages, d, block_table, max_blocks, lens, topk, gated, scale,
+                           o, idx_out, stream);
+}
+
+sas_status sas_decode_paged_ex(const void* q, const void* kpool, const void* vpool,
+                               const void* kspool, sas_dtype sum_dt, sas_dtype dt, int B, int Hq,
+                               int Hkv, int npages, int d, const int32_t* block_table,
+                               int max_blocks, const int32_t* lens, int topk, int gated,
+                               float scale, void* o, int32_t* idx_out, sas_stream_t stream) {
+  g_last_error.clear();
+  return decode_paged_impl("sas_decode_paged_ex launch", q, kpool, vpool, kspool, sum_dt, dt, B,
+                           Hq, Hkv, npages, d, block_table, max_blocks, lens, topk, gated, scale,
+                           o, idx_out, stream);
 }
 
 // ---------------------------------------------------------------- selector backward

@@ -1154,6 +1154,10 @@ cudaError_t launch_fused_g(int G, const void* q, const void* kc, const void* vc,
                            int gated, float scale, void* o, int32_t* idx_out, const int32_t* bt,
                            int npages, cudaStream_t st) {
 #define SAS_FD(GG)                                                                              \
+  if (bt && sum_bf16)                                                                           \
+    return launch_fused_t<T, D, GG, true, __nv_bfloat16>(q, kc, vc, ksum, B, Hkv, Lmax, lens,   \
+                                                         topk, gated, scale, o, idx_out, bt,    \
+                                                         npages, st);                           \
   if (bt)                                                                                       \
     return launch_fused_t<T, D, GG, true, float>(q, kc, vc, ksum, B, Hkv, Lmax, lens, topk,     \
                                                  gated, scale, o, idx_out, bt, npages, st);     \
@@ -1214,10 +1218,10 @@ cudaError_t launch_decode_fused_ex(const void* q, const void* kc, const void* vc
 cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vpool, int bf16,
                                 int B, int Hq, int Hkv, int npages, int d,
                                 const int32_t* block_table, int max_blocks, const int32_t* lens,
-                                const float* kspool, int topk, int gated, float scale, void* o,
-                                int32_t* idx_out, cudaStream_t st) {
+                                const void* kspool, int sum_bf16, int topk, int gated,
+                                float scale, void* o, int32_t* idx_out, cudaStream_t st) {
   return launch_fused(q, kpool, vpool, bf16, B, Hq, Hkv, max_blocks * SAS_BLOCK, d, lens, kspool,
-                      0, topk, gated, scale, o, idx_out, block_table, npages, st);
+                      sum_bf16, topk, gated, scale, o, idx_out, block_table, npages, st);
 }
 
 uint32_t* decode_fused_error_word() {

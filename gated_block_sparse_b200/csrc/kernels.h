@@ -124,12 +124,13 @@ cudaError_t launch_decode_fused_ex(const void* q, const void* kc, const void* vc
                                    const void* ksum, int sum_bf16, int topk, int gated,
                                    float scale, void* o, int32_t* idx_out, cudaStream_t st);
 // Paged caches: kpool, vpool [npages][Hkv][64][d], kspool [npages][Hkv][d]
-// fp32 (the summary of each page), block_table [B][max_blocks] page ids.
+// (the summary of each page; fp32, or bf16 with sum_bf16 = 1), block_table
+// [B][max_blocks] page ids.
 cudaError_t launch_decode_paged(const void* q, const void* kpool, const void* vpool, int bf16,
                                 int B, int Hq, int Hkv, int npages, int d,
                                 const int32_t* block_table, int max_blocks, const int32_t* lens,
-                                const float* kspool, int topk, int gated, float scale, void* o,
-                                int32_t* idx_out, cudaStream_t st);
+                                const void* kspool, int sum_bf16, int topk, int gated,
+                                float scale, void* o, int32_t* idx_out, cudaStream_t st);
 uint32_t* decode_fused_error_word();
 uint32_t* attn_simt_error_word();
 

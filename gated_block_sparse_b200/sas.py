@@ -46,6 +46,8 @@ SIGNATURES = {
                         _P]),
     "sas_decode_paged": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I, _F,
                               _P, _P, _P]),
+    "sas_decode_paged_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _I,
+                                 _F, _P, _P, _P]),
     "sas_decode_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I, _F, _P, _P,
                              _P, _P]),
     "sas_block_summary_ex": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _I, _P]),
@@ -410,6 +412,23 @@ def sas_decode_paged(q, kpool, vpool, kspool, block_table, lens, topk: int, gate
     _check("sas_decode_paged", lib.sas_decode_paged(
         _ptr(q), _ptr(kpool), _ptr(vpool), _ptr(kspool), _dt(q), B, Hq, Hkv, npages, d,
         _ptr(block_table), max_blocks, _ptr(lens), topk, int(gated), float(scale), _ptr(out),
+        _ptr(idx_out), _stream(stream)))
+    return out
+
+
+def sas_decode_paged_ex(q, kpool, vpool, kspool, block_table, lens, topk: int, gated: int = 1,
+                        scale: float = 0.0, out=None, idx_out=None, stream=None):
+    """sas_decode_paged with page summaries kspool [npages][Hkv][d] in fp32 or bf16
+    (the summaries' dtype is taken from kspool)."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    npages, Hkv = kpool.shape[0], kpool.shape[1]
+    max_blocks = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _check("sas_decode_paged_ex", lib.sas_decode_paged_ex(
+        _ptr(q), _ptr(kpool), _ptr(vpool), _ptr(kspool), _dt(kspool), _dt(q), B, Hq, Hkv, npages,
+        d, _ptr(block_table), max_blocks, _ptr(lens), topk, int(gated), float(scale), _ptr(out),
         _ptr(idx_out), _stream(stream)))
     return out
 

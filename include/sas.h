@@ -343,6 +343,20 @@ sas_status sas_decode_paged(const void* q, const void* kpool, const void* vpool,
                             int d, const int32_t* block_table, int max_blocks,
                             const int32_t* lens, int topk, int gated, float scale, void* o,
                             int32_t* idx_out, sas_stream_t stream);
+/*
+ * sas_decode_paged with the page summaries kspool [npages][Hkv][d] of type
+ * sum_dt: SAS_F32 (as sas_decode_paged) or SAS_BF16 (the bf16 summaries of
+ * sas_decode_ex: half the bytes of the summary scan; sas_block_summary_ex and
+ * sas_block_summary_last with a block table write them). The scores are
+ * computed from the stored summaries. sum_dt outside {SAS_F32, SAS_BF16} is
+ * SAS_ERR_INVALID_ARG; arguments, layouts and errors as sas_decode_paged
+ * otherwise.
+ */
+sas_status sas_decode_paged_ex(const void* q, const void* kpool, const void* vpool,
+                               const void* kspool, sas_dtype sum_dt, sas_dtype dt, int B, int Hq,
+                               int Hkv, int npages, int d, const int32_t* block_table,
+                               int max_blocks, const int32_t* lens, int topk, int gated,
+                               float scale, void* o, int32_t* idx_out, sas_stream_t stream);
 
 /*
  * Selector backward (SAS close reading, section 2.3, eq. 8, sparse scope),

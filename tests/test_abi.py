@@ -27,7 +27,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert len(names) == 31
+    assert len(names) == 32
     for n in names:
         assert hasattr(lib, n), n
         assert n in sas.SIGNATURES, n
@@ -107,6 +107,9 @@ def test_rejects_bad_summary_dtype(lib):
     assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
     st = lib.sas_decode_ex(FAKE, FAKE, FAKE, 1, 1, 32, 8, 65536, 128, FAKE, FAKE, 7, 15, 1, 0.0,
                            FAKE, None, None)
+    assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
+    st = lib.sas_decode_paged_ex(FAKE, FAKE, FAKE, FAKE, 7, 1, 1, 32, 8, 16, 128, FAKE, 16, FAKE,
+                                 15, 1, 0.0, FAKE, None, None)
     assert st == 1 and b"summary dtype" in lib.sas_last_error_message()
 
 def test_summary_upkeep_argument_checks(lib):

@@ -73,3 +73,32 @@ def test_decode_byte_accounting_matches_the_stated_figures():
     c = dict(c2, B=1)
     sel, att, step = b.decode_bytes(c, [65])
     assert att == 8 * (64 + 1) * 128 * 2 * 2 + 2 * 8192 and sel == 8 * 1 * 128 * 4 + 8192
+
+
+def test_prefill_flop_accounting_closed_form():
+    """c3 with every query block keeping min(t, 31) history blocks: per head,
+    sum_t 64 * 64 * min(t, 31) kept pairs plus 64 * 65 / 2 causal pairs of the
+    current block; 4 d FLOPs per pair forward, 10 d backward. These are the
+    0.508 / 1.270 TFLOP figures the c3 record is quoted on."""
+    import numpy as np
+    b = _bench()
+    N, Hq, Hkv, d, T = 16384, 32, 8, 128, 256
+    cnt = np.minimum(np.arange(T), 31)[None, None, :].repeat(Hkv, axis=1)
+    f, bw = b.prefill_flops(cnt, N, Hq, Hkv, d)
+    pairs = Hq * (sum(64 * 64 * min(t, 31) for t in range(T)) + T * 64 * 65 // 2)
+    assert f == 4 * d * pairs and bw == 10 * d * pairs
+    assert f == 508014100480 and bw == 1270035251200
+    # a ragged last block of 8 rows sees 8 * 64 keys per kept block and 8 * 9 / 2 causal pairs
+    f2, _ = b.prefill_flops(np.array([[[0, 1]]]), 72, 2, 1, 64)
+    assert f2 == 4 * 64 * 2 * (64 * 65 // 2 + 8 * 64 + 8 * 9 // 2)
+
+
+def test_prefill_flop_accounting_per_token_rows():
+    """Per-token rows: token i of a head sees 64 keys per kept block and the
+    i % 64 + 1 causal keys of its own block."""
+    import numpy as np
+    b = _bench()
+    cnt = np.array([[[0] * 64 + [1] * 64 + [2] * 64]])  # B = 1, Hkv = 1, N = 192
+    f, bw = b.prefill_flops_tokens(cnt, 192, 4, 1, 64)
+    pairs = 4 * (64 * (64 * 1 + 64 * 2) + 3 * (64 * 65 // 2))
+    assert f == 4 * 64 * pairs and bw == 10 * 64 * pairs

@@ -610,6 +610,35 @@ def test_decode_paged_matches_contiguous_and_oracle(gated):
     assert st == 0, msg
 
 
+@pytest.mark.parametrize("sum_dtype", [torch.bfloat16, torch.float32])
+def test_decode_paged_ex_summary_dtypes(sum_dtype):
+    """Paged decode reading page summaries of either dtype: identical to the
+    contiguous call reading the same summaries (sas_decode_ex), and against the
+    oracle selecting on the stored (for bf16: rounded) means."""
+    B, Hq, Hkv, Lmax, d, topk = 2, 16, 4, 8192, 128, 15
+    x = inputs.gen_decode(B, Hq, Hkv, Lmax, d, [8192, 6001], "bf16", seed=74, planted=16)
+    q, kc, vc, lens = x["q"], x["kc"], x["vc"], x["lens"]
+    kpool, vpool, bt = _to_pages(kc, vc, lens, seed=75)
+    kspool = sas.sas_block_summary_ex(dev(kpool.view(-1, Hkv, 64, d)), sum_dtype).view(-1, Hkv, d)
+    idx_p = torch.empty((B, Hkv, topk), dtype=torch.int32, device=DEV)
+    o_p = sas.sas_decode_paged_ex(dev(q), dev(kpool), dev(vpool), kspool,
+                                  dev(torch.from_numpy(bt)), dev(lens), topk, idx_out=idx_p)
+    ks = sas.sas_block_summary_ex(dev(kc), sum_dtype)
+    idx_c = torch.empty_like(idx_p)
+    o_c = sas.sas_decode_ex(dev(q), dev(kc), dev(vc), dev(lens), ks, topk, idx_out=idx_c)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_p, idx_c)
+    assert torch.equal(o_p, o_c)
+    oks = O.block_summary(kc)
+    if sum_dtype == torch.bfloat16:
+        oks = O.round_bf16(oks)
+    oo, oi, _, _ = O.decode(q, kc, vc, lens.numpy(), oks, Hkv, topk, gated=1)
+    assert np.array_equal(idx_p.cpu().numpy(), oi)
+    assert excess(np64(o_p), oo, 2e-2, True) <= 0
+    st, msg = sas.sas_device_status()
+    assert st == 0, msg
+
+
 def test_decode_host_buffers_match_device_call():
     """sas_decode_host gives the device call's output exactly, with pinned
     host q and o (read and written by the step over the bus) and with

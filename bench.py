@@ -56,6 +56,10 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn decode GB/s vs HBM peak; prefill fwd+bwd TFLOP/s vs bf16 peak"
 DEFAULT_STEPS = {"c1": 200, "c2": 100000, "c3": 200, "c4": 4000, "c5": 20000}
 DEFAULT_WARMUP = {"c1": 10, "c2": 1000, "c3": 3, "c4": 100, "c5": 500}
+# reference arm (the fp64 oracle on one core): steps without --steps, and the
+# most steps it times (an oracle step takes tens of milliseconds)
+REFERENCE_STEPS = 20
+REFERENCE_MAX_STEPS = 1000
 # (record name, config, options) of the default run; the first is the headline
 ALL_RECORDS = (("c5", "c5", {}), ("c5_bf16_summaries", "c5", {"summary": "bf16"}),
                ("c4", "c4", {}), ("c2", "c2", {}), ("c2_paged", "c2", {"paged": True}),
@@ -795,6 +799,58 @@ def cpu_baseline_decode(w: DecodeWorkload, seconds: float, all_cores: bool = Tru
     return res
 
 
+def reference_arm(cfg: str, summary: str, K: int, W: int) -> dict:
+    """The oracle as the reference arm: W untimed and K timed steps on one
+    core (one BLAS thread), each step a bounded sample of the workload: a
+    whole decode step (all rows) for decode workloads, one (sequence, kv
+    group, query block) unit's forward and backward, latest blocks first and
+    cycling, for prefill."""
+    from gated_block_sparse_b200 import inputs
+    from oracle import sas_oracle as O
+    c = inputs.CONFIGS[cfg]
+    with _one_thread():
+        if c["kind"] == "decode":
+            w = DecodeWorkload(cfg, summary)
+            h = w.host
+            ks = O.block_summary(h["kc"], lens=h["lens"].numpy())
+            if summary == "bf16":
+                ks = O.round_bf16(ks)
+            lens = h["lens"].numpy()
+
+            def step(i):
+                O.decode(h["q"], h["kc"], h["vc"], lens, ks, c["Hkv"], c["topk"], gated=c["gated"])
+                return w.step_bytes
+            unit, scale_to, what = "GB/s", 1e9, f"a whole decode step of {cfg} (all {w.rows} rows)"
+        else:
+            h = inputs.gen_config(cfg)
+            N, d, G = c["N"], c["d"], c["Hq"] // c["Hkv"]
+            ks = O.block_summary(h["k"])
+            idx, cnt, logg, _ = O.select_prefill(h["q"], ks, c["Hkv"], c["topk"])
+            T = idx.shape[2]
+            order = [(b, r, t) for t in range(T - 1, -1, -1) for b in range(c["B"])
+                     for r in range(c["Hkv"])]
+
+            def step(i):
+                b, r, t = order[i % len(order)]
+                O.query_block(h["q"], h["k"], h["v"], h["do"], idx, cnt, logg, b, r, t)
+                nr = min(64, N - 64 * t)
+                return 14 * d * (int(cnt[b, r, t]) * G * nr * 64 + G * nr * (nr + 1) // 2)
+            unit, scale_to = "TFLOP/s", 1e12
+            what = (f"one (sequence, kv group, query block) unit of {cfg}, forward + backward "
+                    "of all heads of the group")
+        for i in range(W):
+            step(i)
+        work, t0 = 0, time.perf_counter()
+        for i in range(K):
+            work += step(W + i)
+        el = time.perf_counter() - t0
+    value = round(work / el / scale_to, 6)
+    return {"value": value, "unit": unit, "steps": K, "warmup": W, "seconds": round(el, 3),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                             "sample": f"{K} steps, each {what}; fp64 numpy oracle, 1 BLAS thread",
+                             "cpu_model": cpu_model(), "nproc": os.cpu_count()}}
+
+
 def cpu_baseline_prefill(name: str, seconds: float, host=None, all_cores: bool = True) -> dict:
     """The oracle's forward+backward on whole query blocks of the workload
     (one core), and on all cores over (kv group, query block) units."""
@@ -960,18 +1016,18 @@ def main():
             return
         from gated_block_sparse_b200 import inputs
         name, cfg, opts = plan[0]
-        if inputs.CONFIGS[cfg]["kind"] == "decode":
-            base = cpu_baseline_decode(DecodeWorkload(cfg, opts.get("summary", "f32")), cpu_s)
-        else:
-            base = cpu_baseline_prefill(cfg, cpu_s)
+        K = min(args.steps or REFERENCE_STEPS, REFERENCE_MAX_STEPS)
+        W = min(args.warmup if args.warmup is not None else 1, REFERENCE_MAX_STEPS)
+        ref = reference_arm(cfg, opts.get("summary", "f32"), K, W)
         print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": base["value"], "unit": base["unit"],
-            "n_gpus": args.gpus, "steps": base.get("steps"), "warmup": 0,
+            "impl": "reference", "metric": METRIC, "value": ref["value"], "unit": ref["unit"],
+            "n_gpus": args.gpus, "steps": K, "warmup": W,
+            "ms_per_step": ref["seconds"] * 1e3 / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded, same generator)",
             "config": {"workload": f"{cfg}: {inputs.DESCRIPTIONS[cfg]}"},
-            "cpu_baseline": base,
-            "e2e": {"value": base["value"], "unit": base["unit"], "h2d_bytes_per_step": 0,
+            "cpu_baseline": ref["cpu_baseline"],
+            "e2e": {"value": ref["value"], "unit": ref["unit"], "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}))
         return
 

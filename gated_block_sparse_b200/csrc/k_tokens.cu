@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_tokens(
   float* sc = Kb + S::TILE;  // [64][C + 1] scores
   const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
   const int G = Hq / Hkv, nblk = N / SAS_BLOCK;
-  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15, lane = tid & 31, wid = tid >> 5;
+  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15, wid = tid >> 5;
   const int row0 = t * SAS_BLOCK, nr = min(SAS_BLOCK, N - row0);
   const int C = t, CP = t + 1;
   for (int e = tid; e < SAS_BLOCK * D; e += AT_THREADS) {

@@ -626,6 +626,25 @@ cudaError_t launch_attn_bwd_tokens(const void* q, const void* k, const void* v, 
 }
 
 // ------------------------------------------------------------------ selector backward
+// fp32 -> tf32 (round to nearest) and one m16n8k8 tf32 warp MMA (c += a b,
+// fp32 accumulation). Fragments: a0 = A[g][t], a1 = A[g + 8][t], a2 =
+// A[g][t + 4], a3 = A[g + 8][t + 4]; b0 = B[t][g], b1 = B[t + 4][g]; c0, c1 =
+// C[g][2t], C[g][2t + 1], c2, c3 = C[g + 8][2t], C[g + 8][2t + 1], with
+// g = lane / 4, t = lane % 4.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Eq. 8 (section 2.3, sparse scope) for per-token rows: for token i of kv
 // group r with C = i / 64, kept set I_i and g = softmax(s_i),
 //   ds_m = dlogg[slot of m] [m in I_i] - g_m sum_{l in I_i} dlogg[slot of l];
@@ -635,8 +654,12 @@ cudaError_t launch_attn_bwd_tokens(const void* q, const void* k, const void* v, 
 // kernel adds dkbar_m / 64 into each of block m's 64 keys of dk).
 // One CTA per (query block t, kv group r, sequence b): the rows' query means
 // and scores as in k_select_tokens, the gate and ds per row (one warp per
-// row), then dqbar = ds kbar over 64-block chunks (tile products in fp32)
-// and each chunk's ds^T qbar added into dkbar.
+// row), then dqbar = ds kbar over 64-block chunks and each chunk's
+// ds^T qbar added into dkbar. The three tile products run on the CUDA cores
+// in fp32 for fp32 inputs, and as tf32 warp MMAs (fp32 accumulation) for bf16
+// inputs, whose outputs are stored in bf16: each warp takes a 16-row slice
+// (warp % 4) and half of the columns (warp / 4) of every 64 x 64 or 64 x d
+// product.
 template <typename T, int D>
 __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
     const T* __restrict__ q, const float* __restrict__ ksum, int Hq, int Hkv, int N, int topk,
@@ -647,12 +670,15 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
   float* Qb = sm;            // [64][LD] the rows' query means
   float* Kb = Qb + S::TILE;  // [64][LD] 64 summaries
   float* sc = Kb + S::TILE;  // [64][C + 1] scores, then ds
+  constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int NT2 = D / 16;  // 8-column tiles of half of d (tensor-core path)
   const int t = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
   const int C = t, CP = t + 1;
   if (C == 0) return;  // no history: the selector has no gradient here
   const int G = Hq / Hkv, nblk = N / SAS_BLOCK;
   const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15, lane = tid & 31, wid = tid >> 5;
   const int row0 = t * SAS_BLOCK, nr = min(SAS_BLOCK, N - row0);
+  const int g8 = lane >> 2, t4 = lane & 3, mi = wid & 3, hw = wid >> 2;  // tensor-core path
   for (int e = tid; e < SAS_BLOCK * D; e += AT_THREADS) {
     const int i = e / D, c = e % D;
     float a = 0.f;
@@ -669,15 +695,44 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
       Kb[jj * S::LD + c] = (m0 + jj < C) ? krow[(size_t)(m0 + jj) * D + c] : 0.f;
     }
     __syncthreads();
-    float s[4][4];
-    tile_dot<D>(Qb, Kb, tr, tc, s);
+    if constexpr (TC) {
+      // rows 16 mi + g8 (+8) x summaries m0 + 32 hw + 8 nt + 2 t4 (+1)
+      float c4[4][4] = {};
+#pragma unroll 4
+      for (int k0 = 0; k0 < D; k0 += 8) {
+        const float* qa = Qb + (16 * mi + g8) * S::LD + k0 + t4;
+        const uint32_t a0 = to_tf32(qa[0]), a1 = to_tf32(qa[8 * S::LD]), a2 = to_tf32(qa[4]),
+                       a3 = to_tf32(qa[8 * S::LD + 4]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int m = m0 + tc + 16 * j;
-        if (m < C) sc[(tr + 16 * i) * CP + m] = s[i][j] * scale;
+        for (int nt = 0; nt < 4; ++nt) {
+          const float* kb = Kb + (32 * hw + 8 * nt + g8) * S::LD + k0 + t4;
+          mma_tf32(c4[nt], a0, a1, a2, a3, to_tf32(kb[0]), to_tf32(kb[4]));
+        }
       }
+      const int row = 16 * mi + g8;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int m = m0 + 32 * hw + 8 * nt + 2 * t4;
+        if (m < C) {
+          sc[row * CP + m] = c4[nt][0] * scale;
+          sc[(row + 8) * CP + m] = c4[nt][2] * scale;
+        }
+        if (m + 1 < C) {
+          sc[row * CP + m + 1] = c4[nt][1] * scale;
+          sc[(row + 8) * CP + m + 1] = c4[nt][3] * scale;
+        }
+      }
+    } else {
+      float s[4][4];
+      tile_dot<D>(Qb, Kb, tr, tc, s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = m0 + tc + 16 * j;
+          if (m < C) sc[(tr + 16 * i) * CP + m] = s[i][j] * scale;
+        }
+    }
   }
   __syncthreads();
   // ds per row (one warp per row); rows past the sequence end get ds = 0
@@ -714,6 +769,8 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
     for (int g = 0; g < S::NG; ++g)
 #pragma unroll
       for (int e = 0; e < 4; ++e) dqa[i][g][e] = 0.f;
+  // tensor-core path: rows 16 mi + g8 (+8) x columns (d / 2) hw + 8 nt + 2 t4 (+1)
+  float dqc[NT2][4] = {};
   float* dkb = dkbar + ((size_t)b * Hkv + r) * (size_t)nblk * D;
   for (int m0 = 0; m0 < C; m0 += SAS_BLOCK) {
     __syncthreads();  // ds written; the previous chunk's Kb consumed
@@ -723,78 +780,142 @@ __global__ void __launch_bounds__(AT_THREADS) k_select_bwd_tokens(
       Kb[jj * S::LD + c] = (jj < nm) ? krow[(size_t)(m0 + jj) * D + c] : 0.f;
     }
     __syncthreads();
-    // dqbar[i] += sum_m ds[i][m] kbar_m
-#pragma unroll 4
-    for (int j = 0; j < nm; ++j) {
-      float dsj[4];
+    if constexpr (TC) {
+      // dqbar[rows] += ds[rows][m0 + m] kbar[m], m over the chunk
+#pragma unroll 2
+      for (int k0 = 0; k0 < SAS_BLOCK; k0 += 8) {
+        const int ka = m0 + k0 + t4;
+        const float* da = sc + (16 * mi + g8) * CP;
+        const uint32_t a0 = to_tf32(ka < C ? da[ka] : 0.f);
+        const uint32_t a1 = to_tf32(ka < C ? da[8 * CP + ka] : 0.f);
+        const uint32_t a2 = to_tf32(ka + 4 < C ? da[ka + 4] : 0.f);
+        const uint32_t a3 = to_tf32(ka + 4 < C ? da[8 * CP + ka + 4] : 0.f);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dsj[i] = sc[(tr + 16 * i) * CP + m0 + j];
-#pragma unroll
-      for (int g = 0; g < S::NG; ++g) {
-        const float4 kv = *reinterpret_cast<const float4*>(Kb + j * S::LD + 4 * tc + 64 * g);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          dqa[i][g][0] += dsj[i] * kv.x;
-          dqa[i][g][1] += dsj[i] * kv.y;
-          dqa[i][g][2] += dsj[i] * kv.z;
-          dqa[i][g][3] += dsj[i] * kv.w;
+        for (int nt = 0; nt < NT2; ++nt) {
+          const float* kb = Kb + (k0 + t4) * S::LD + (D / 2) * hw + 8 * nt + g8;
+          mma_tf32(dqc[nt], a0, a1, a2, a3, to_tf32(kb[0]), to_tf32(kb[4 * S::LD]));
         }
       }
-    }
-    // dkbar[m] += scale sum_i ds[i][m] qbar_i (rows m = tr + 16 jj of the chunk)
-    float a[4][S::NG][4];
+      // dkbar[m0 + m] += scale sum_rows ds[row][m0 + m] qbar[row]
+      float dkc[NT2][4] = {};
+      const int mm = m0 + 16 * mi + g8;
+#pragma unroll 2
+      for (int k0 = 0; k0 < SAS_BLOCK; k0 += 8) {
+        const float* da = sc + (k0 + t4) * CP;
+        const uint32_t a0 = to_tf32(mm < C ? da[mm] : 0.f);
+        const uint32_t a1 = to_tf32(mm + 8 < C ? da[mm + 8] : 0.f);
+        const uint32_t a2 = to_tf32(mm < C ? da[4 * CP + mm] : 0.f);
+        const uint32_t a3 = to_tf32(mm + 8 < C ? da[4 * CP + mm + 8] : 0.f);
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
+        for (int nt = 0; nt < NT2; ++nt) {
+          const float* qb = Qb + (k0 + t4) * S::LD + (D / 2) * hw + 8 * nt + g8;
+          mma_tf32(dkc[nt], a0, a1, a2, a3, to_tf32(qb[0]), to_tf32(qb[4 * S::LD]));
+        }
+      }
 #pragma unroll
-      for (int g = 0; g < S::NG; ++g)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) a[jj][g][e] = 0.f;
+      for (int nt = 0; nt < NT2; ++nt) {
+        const int col = (D / 2) * hw + 8 * nt + 2 * t4;
+        if (mm < C)
+          atomicAdd(reinterpret_cast<float2*>(dkb + (size_t)mm * D + col),
+                    make_float2(dkc[nt][0] * scale, dkc[nt][1] * scale));
+        if (mm + 8 < C)
+          atomicAdd(reinterpret_cast<float2*>(dkb + (size_t)(mm + 8) * D + col),
+                    make_float2(dkc[nt][2] * scale, dkc[nt][3] * scale));
+      }
+    } else {
+      // dqbar[i] += sum_m ds[i][m] kbar_m
 #pragma unroll 4
-    for (int i2 = 0; i2 < nr; ++i2) {
-      float wj[4];
+      for (int j = 0; j < nm; ++j) {
+        float dsj[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dsj[i] = sc[(tr + 16 * i) * CP + m0 + j];
+#pragma unroll
+        for (int g = 0; g < S::NG; ++g) {
+          const float4 kv = *reinterpret_cast<const float4*>(Kb + j * S::LD + 4 * tc + 64 * g);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            dqa[i][g][0] += dsj[i] * kv.x;
+            dqa[i][g][1] += dsj[i] * kv.y;
+            dqa[i][g][2] += dsj[i] * kv.z;
+            dqa[i][g][3] += dsj[i] * kv.w;
+          }
+        }
+      }
+      // dkbar[m] += scale sum_i ds[i][m] qbar_i (rows m = tr + 16 jj of the chunk)
+      float a[4][S::NG][4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int g = 0; g < S::NG; ++g)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a[jj][g][e] = 0.f;
+#pragma unroll 4
+      for (int i2 = 0; i2 < nr; ++i2) {
+        float wj[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int m = tr + 16 * jj;
+          wj[jj] = m < nm ? sc[i2 * CP + m0 + m] : 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < S::NG; ++g) {
+          const float4 xv = *reinterpret_cast<const float4*>(Qb + i2 * S::LD + 4 * tc + 64 * g);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            a[jj][g][0] += wj[jj] * xv.x;
+            a[jj][g][1] += wj[jj] * xv.y;
+            a[jj][g][2] += wj[jj] * xv.z;
+            a[jj][g][3] += wj[jj] * xv.w;
+          }
+        }
+      }
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int m = tr + 16 * jj;
-        wj[jj] = m < nm ? sc[i2 * CP + m0 + m] : 0.f;
+        if (m >= nm) continue;
+        float* drow = dkb + (size_t)(m0 + m) * D;
+#pragma unroll
+        for (int g = 0; g < S::NG; ++g)
+          atomicAdd(reinterpret_cast<float4*>(drow + 4 * tc + 64 * g),
+                    make_float4(a[jj][g][0] * scale, a[jj][g][1] * scale, a[jj][g][2] * scale,
+                                a[jj][g][3] * scale));
       }
-#pragma unroll
-      for (int g = 0; g < S::NG; ++g) {
-        const float4 xv = *reinterpret_cast<const float4*>(Qb + i2 * S::LD + 4 * tc + 64 * g);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          a[jj][g][0] += wj[jj] * xv.x;
-          a[jj][g][1] += wj[jj] * xv.y;
-          a[jj][g][2] += wj[jj] * xv.z;
-          a[jj][g][3] += wj[jj] * xv.w;
-        }
-      }
-    }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int m = tr + 16 * jj;
-      if (m >= nm) continue;
-      float* drow = dkb + (size_t)(m0 + m) * D;
-#pragma unroll
-      for (int g = 0; g < S::NG; ++g)
-        atomicAdd(reinterpret_cast<float4*>(drow + 4 * tc + 64 * g),
-                  make_float4(a[jj][g][0] * scale, a[jj][g][1] * scale, a[jj][g][2] * scale,
-                              a[jj][g][3] * scale));
     }
   }
   const float fq = scale / (float)G;
+  if constexpr (TC) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int ri = tr + 16 * i;
-    if (ri >= nr) continue;
-    for (int g = 0; g < G; ++g) {
-      T* drow = dq + (((size_t)b * Hq + r * G + g) * N + row0 + ri) * D;
+    for (int hf = 0; hf < 2; ++hf) {
+      const int ri = 16 * mi + g8 + 8 * hf;
+      if (ri >= nr) continue;
+      for (int g = 0; g < G; ++g) {
+        T* drow = dq + (((size_t)b * Hq + r * G + g) * N + row0 + ri) * D;
 #pragma unroll
-      for (int gg = 0; gg < S::NG; ++gg)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * tc + 64 * gg + e;
-          drow[c] = from_f<T>(to_f(drow[c]) + dqa[i][gg][e] * fq);
+        for (int nt = 0; nt < NT2; ++nt) {
+          __nv_bfloat162* p2 =
+              reinterpret_cast<__nv_bfloat162*>(drow + (D / 2) * hw + 8 * nt + 2 * t4);
+          float2 v = __bfloat1622float2(*p2);
+          v.x += dqc[nt][2 * hf] * fq;
+          v.y += dqc[nt][2 * hf + 1] * fq;
+          *p2 = __float22bfloat162_rn(v);
         }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int ri = tr + 16 * i;
+      if (ri >= nr) continue;
+      for (int g = 0; g < G; ++g) {
+        T* drow = dq + (((size_t)b * Hq + r * G + g) * N + row0 + ri) * D;
+#pragma unroll
+        for (int gg = 0; gg < S::NG; ++gg)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * tc + 64 * gg + e;
+            drow[c] = from_f<T>(to_f(drow[c]) + dqa[i][gg][e] * fq);
+          }
+      }
     }
   }
 }

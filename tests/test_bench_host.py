@@ -102,3 +102,13 @@ def test_prefill_flop_accounting_per_token_rows():
     f, bw = b.prefill_flops_tokens(cnt, 192, 4, 1, 64)
     pairs = 4 * (64 * (64 * 1 + 64 * 2) + 3 * (64 * 65 // 2))
     assert f == 4 * 64 * pairs and bw == 10 * 64 * pairs
+
+
+def test_reference_arm_times_exactly_k_steps():
+    """--impl reference: W untimed and K timed oracle steps, each a bounded
+    sample (here one query-block unit of the tiny prefill workload)."""
+    b = _bench()
+    got = b.reference_arm("c1", "f32", 3, 1)
+    assert got["steps"] == 3 and got["warmup"] == 1
+    assert got["value"] > 0 and got["unit"] == "TFLOP/s"
+    assert got["cpu_baseline"]["kind"] == "oracle" and got["cpu_baseline"]["cores"] == 1
